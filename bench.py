@@ -1,0 +1,487 @@
+#!/usr/bin/env python
+"""Benchmark of the W8A8 scaled-FP8 Linear on B200.
+
+A step is one pass of the whole hot path over one DiT block: for every
+distinct activation of the block, per-token FP8 quantization (tfq kernel),
+then every Linear reading it as a scaled FP8 GEMM with the fused
+scale/bias/BF16 epilogue (tfq kernel).  Weights are quantized once per
+channel before timing (the offline converter step).  The metric is the
+block's GEMM FLOPs divided by the step time, which includes the activation
+quantizers ("TFLOP/s incl. act quant").
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+    python bench.py --impl reference ...     # the CPU oracle on a bounded sample
+
+Prints ONE JSON line (rank 0).  Multi-GPU: one process per GPU (torchrun);
+each rank runs an independent replica of the workload (weak scaling, no
+data-path collective); time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "scaled-FP8 Linear TFLOP/s incl. act quant, % of B200 FP8 dense peak"
+FP8_SPEC_TFLOPS = 4500.0
+FP8_OVER_BF16 = 2.0      # nominal dense ratio fp8 / bf16 (4.5 / 2.25 PFLOP/s)
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+L2_BYTES = 126 * 1024 * 1024
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="video_dit_block",
+                    choices=["video_dit_block", "image_dit_block", "reduced_qmax_ffn_out", "tiny_w8a8_linear"])
+    ap.add_argument("--impl", default="tfq", choices=["tfq", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle sample")
+    return ap.parse_args()
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as fh:
+            d = json.load(fh)
+        return d, "measured"
+    except (OSError, ValueError):
+        return {"hbm_gbs": FALLBACK_HBM_GBS, "bf16_tflops": FALLBACK_BF16_TFLOPS,
+                "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms."""
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(prefix="clocks", suffix=".csv")
+            os.close(fd)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.QUERY}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.fh, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.fh.close()
+        rows = []
+        with open(self.path) as fh:
+            for line in fh:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        def num(v):
+            try:
+                return float(v)
+            except ValueError:
+                return None
+        sm = [num(r[1]) for r in rows if num(r[1]) is not None]
+        pw = [num(r[3]) for r in rows if num(r[3]) is not None]
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            for name, v in zip(names, r[5:9]):
+                if v.strip().lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": num(rows[0][2]),
+                "power_w_max": max(pw) if pw else None,
+                "samples": len(rows),
+                "reasons": sorted(reasons)}
+
+
+# --------------------------------------------------------- multi-rank
+def max_over_ranks(value: float, device) -> float:
+    """Max of a per-rank timing over all ranks (the only collective: plumbing,
+    not data path).  `device` is where the backend wants the tensor."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_throughput(world: int, flops_per_step: int, ms_per_step_max: float) -> float:
+    """Whole-job TFLOP/s: every rank runs one replica of the workload per
+    step (weak scaling), timed by the slowest rank."""
+    return world * flops_per_step / (ms_per_step_max * 1e-3) / 1e12
+
+
+# ------------------------------------------------------------ GPU arm
+def build_block(wl, dev):
+    """Device-resident inputs, quantized weights and outputs of one block."""
+    import torch
+    from int8_w8a8_quantized_b200 import tfq_quant_weight_per_channel
+
+    xs = {name: wl.make_x(name, device=dev) for name in sorted(wl.x_shapes())}
+    lins = []
+    for lin in wl.linears:
+        w = wl.make_w(lin, device=dev)
+        Wq, sw = tfq_quant_weight_per_channel(w, "fp8", 448.0)
+        del w
+        b = wl.make_bias(lin, device=dev)
+        lins.append((lin, Wq, sw, b))
+    aq = {(name, q): (torch.empty_like(x, dtype=torch.uint8), torch.empty(x.shape[0], device=dev))
+          for name, x in xs.items() for q in wl.act_qmax}
+    ys = {(lin.name, q): torch.empty((wl.M, lin.N), dtype=torch.bfloat16, device=dev)
+          for lin in wl.linears for q in wl.act_qmax}
+    torch.cuda.synchronize()
+    return xs, lins, aq, ys
+
+
+def gpu_arm(args, wl, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    from int8_w8a8_quantized_b200 import _capi
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    lib = _capi.load_library()
+    stream = torch.cuda.current_stream()
+    sh = int(stream.cuda_stream)
+    xs, lins, aq, ys = build_block(wl, dev)
+
+    # per-kernel events, recorded on the launching stream
+    ev = {"quant": [], "gemm": []}
+    launches = [0]
+
+    def check(st, what):
+        if st != 0:
+            raise RuntimeError(f"{what}: {_capi.status_string(st)}: {_capi.last_error_message()}")
+
+    def step(record):
+        for q in wl.act_qmax:
+            for name, x in xs.items():
+                A, sa = aq[(name, q)]
+                if record:
+                    e0 = torch.cuda.Event(enable_timing=True); e0.record(stream)
+                check(lib.tfq_quant_act_fp8_per_token(x.data_ptr(), x.shape[0], x.shape[1], float(q),
+                                                      A.data_ptr(), sa.data_ptr(), sh), "quant")
+                launches[0] += 1
+                if record:
+                    e1 = torch.cuda.Event(enable_timing=True); e1.record(stream)
+                    # algorithmic bytes: read bf16, write e4m3 codes, 4 B of scale per row
+                    ev["quant"].append((e0, e1, 3 * x.numel() + 4 * x.shape[0]))
+            for lin, Wq, sw, b in lins:
+                A, sa = aq[(lin.x, q)]
+                y = ys[(lin.name, q)]
+                if record:
+                    e0 = torch.cuda.Event(enable_timing=True); e0.record(stream)
+                check(lib.tfq_scaled_fp8_linear(A.data_ptr(), sa.data_ptr(), Wq.data_ptr(), sw.data_ptr(),
+                                                None if b is None else b.data_ptr(), wl.M, lin.N, lin.K,
+                                                y.data_ptr(), sh), "gemm")
+                launches[0] += 1
+                if record:
+                    e1 = torch.cuda.Event(enable_timing=True); e1.record(stream)
+                    ev["gemm"].append((e0, e1, (wl.M, lin.N, lin.K)))
+
+    for _ in range(args.warmup):
+        step(False)
+    torch.cuda.synchronize()
+    check(lib.tfq_device_error(sh), "device error after warm-up")
+
+    clocks = ClockSampler(local_rank)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    launches[0] = 0
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(args.steps):
+        step(True)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    if world > 1:
+        dist.barrier()
+    check(lib.tfq_device_error(sh), "device error in the timed region")
+    ms = max_over_ranks(t0.elapsed_time(t1), dev) if world > 1 else t0.elapsed_time(t1)
+    ms_per_step = ms / args.steps
+
+    gemm_ms = [a.elapsed_time(b) for a, b, _ in ev["gemm"]]
+    quant_ms = [a.elapsed_time(b) for a, b, _ in ev["quant"]]
+    gemm_flops = [2 * m * n * k for _, _, (m, n, k) in ev["gemm"]]
+    quant_bytes = [nbytes for _, _, nbytes in ev["quant"]]
+    out = {
+        "ms_per_step": ms_per_step,
+        "gemm_ms_total": sum(gemm_ms), "gemm_flops_total": sum(gemm_flops),
+        "quant_ms_total": sum(quant_ms), "quant_bytes_total": sum(quant_bytes),
+        "gemm_launches": len(gemm_ms), "quant_launches": len(quant_ms),
+        "gpu_launches": launches[0], "clocks": clk,
+        "per_linear": {},
+    }
+    for (a, b, (m, n, k)) in ev["gemm"]:
+        key = f"{m}x{n}x{k}"
+        out["per_linear"].setdefault(key, []).append(a.elapsed_time(b))
+
+    # -------- end-to-end through the C ABI with host buffers
+    e2e = None
+    if not args.no_e2e:
+        e2e = e2e_arm(args, wl, lib, xs, lins, aq, ys, stream, sh, check)
+    return out, e2e
+
+
+def e2e_arm(args, wl, lib, xs, lins, aq, ys, stream, sh, check):
+    """Every step: H2D copy of the block's activations from pinned host
+    memory, the quantizers and GEMMs, D2H copy of every output."""
+    import torch
+    hx = {n: torch.empty(x.shape, dtype=x.dtype, pin_memory=True) for n, x in xs.items()}
+    for n, x in xs.items():
+        hx[n].copy_(x)
+    hy = {k: torch.empty(y.shape, dtype=y.dtype, pin_memory=True) for k, y in ys.items()}
+    h2d = sum(t.numel() * t.element_size() for t in hx.values())
+    d2h = sum(t.numel() * t.element_size() for t in hy.values())
+
+    def step():
+        for n, x in xs.items():
+            x.copy_(hx[n], non_blocking=True)
+        for q in wl.act_qmax:
+            for n, x in xs.items():
+                A, sa = aq[(n, q)]
+                check(lib.tfq_quant_act_fp8_per_token(x.data_ptr(), x.shape[0], x.shape[1], float(q),
+                                                      A.data_ptr(), sa.data_ptr(), sh), "quant")
+            for lin, Wq, sw, b in lins:
+                A, sa = aq[(lin.x, q)]
+                y = ys[(lin.name, q)]
+                check(lib.tfq_scaled_fp8_linear(A.data_ptr(), sa.data_ptr(), Wq.data_ptr(), sw.data_ptr(),
+                                                None if b is None else b.data_ptr(), wl.M, lin.N, lin.K,
+                                                y.data_ptr(), sh), "gemm")
+        for k, y in ys.items():
+            hy[k].copy_(y, non_blocking=True)
+
+    step()
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(args.e2e_steps):
+        step()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    ms = t0.elapsed_time(t1) / args.e2e_steps
+    return {"value": wl.flops() / (ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": ms,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": args.e2e_steps,
+            "host_buffers": "pinned"}
+
+
+# ------------------------------------------------------------ CPU oracle
+def oracle_sample(wl, seconds: float, seed: int = 0):
+    """Runs the oracle (quantizer + double GEMM) on a bounded sample of the
+    workload's rows; returns (flops_done, seconds_taken, description)."""
+    import numpy as np
+    import torch
+    import oracle
+
+    rng = np.random.default_rng(seed)
+    # Rows are independent, so a sample of rows is a sample of the job: each
+    # pass quantizes `threads` fresh rows per Linear (drawn with the same
+    # recipe) and multiplies them by the full per-channel FP8 weight, which
+    # keeps every OpenMP thread of the oracle busy.
+    rows_per_linear = oracle.num_threads()
+    total_flops = 0
+    t_total = 0.0
+    done = []
+    cache = {}
+    while t_total < seconds:
+        for lin in wl.linears:
+            key = lin.name
+            if key not in cache:
+                w = wl.make_w(lin)
+                wbits = w.contiguous().view(torch.int16).numpy().view(np.uint16)
+                Wq, sw = oracle.quant_rows_fp8(wbits, 448.0)
+                b = wl.make_bias(lin)
+                bbits = None if b is None else b.contiguous().view(torch.int16).numpy().view(np.uint16)
+                cache[key] = (Wq, sw, bbits)
+            Wq, sw, bbits = cache[key]
+            x = _x_rows(wl, lin, rows_per_linear, int(rng.integers(1 << 30)))
+            for q in wl.act_qmax:
+                t0 = time.perf_counter()
+                A, sa = oracle.quant_rows_fp8(x, q)
+                oracle.scaled_fp8_linear(A, sa, Wq, sw, bbits)
+                t_total += time.perf_counter() - t0
+                total_flops += 2 * x.shape[0] * lin.N * lin.K
+                done.append(x.shape[0])
+    desc = (f"{sum(done)} rows (per-token quantization + double-accumulated GEMM against the full "
+            f"per-channel FP8 weight) over the {len(wl.linears)} Linears of {wl.name}; "
+            f"FLOPs of the sample / oracle time")
+    return total_flops, t_total, desc
+
+
+def _x_rows(wl, lin, n, seed):
+    import numpy as np
+    import torch
+    from int8_w8a8_quantized_b200 import workloads
+    r = wl.x_recipe
+    x = workloads.activations(n, lin.K, seed=seed, nu=r.nu, amplitude=r.amplitude,
+                              outlier_cols=int(round(r.outlier_frac * lin.K)), outlier_mult=r.outlier_mult)
+    return x.contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def cpu_baseline(wl, seconds):
+    import oracle
+    flops, secs, desc = oracle_sample(wl, seconds)
+    return {"value": flops / secs / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": desc, "seconds": secs}
+
+
+# ------------------------------------------------------------------ main
+def main():
+    args = parse_args()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    from int8_w8a8_quantized_b200 import workloads
+    wl = workloads.WORKLOADS[args.workload]
+    cfg = {"workload": wl.name, "M": wl.M,
+           "linears": [f"{l.name}:{l.K}->{l.N}" for l in wl.linears],
+           "act_qmax": list(wl.act_qmax), "weight_qmax": 448.0, "bias": wl.has_bias,
+           "l2": "inputs larger than L2 (126 MB)" if wl.M * min(l.K for l in wl.linears) * 2 > L2_BYTES
+           else "working set of one step larger than L2; no flush",
+           "parallelism": f"replicas x{world}"}
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        reference_arm(args, wl, cfg, world)
+        return 0
+
+    import torch
+    import torch.distributed as dist
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    res, e2e = gpu_arm(args, wl, rank, world, local_rank)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+
+    peaks, peak_src = measured_peaks()
+    flops_step = wl.flops()
+    value = aggregate_throughput(world, flops_step, res["ms_per_step"])
+    gemm_avg_ms = res["gemm_ms_total"] / max(1, res["gemm_launches"])
+    gemm_tflops = res["gemm_flops_total"] / (res["gemm_ms_total"] * 1e-3) / 1e12
+    timed_s = res["ms_per_step"] * args.steps * 1e-3
+    sustained = timed_s >= 1.0
+    bf16 = peaks.get("bf16_tflops_sustained" if sustained else "bf16_tflops", FALLBACK_BF16_TFLOPS)
+    fp8_peak = bf16 * FP8_OVER_BF16
+    quant_gbs = res["quant_bytes_total"] / (res["quant_ms_total"] * 1e-3) / 1e9 if res["quant_ms_total"] else None
+    line = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "TFLOP/s",
+        "pct_fp8_dense_peak": round(100.0 * value / (world * FP8_SPEC_TFLOPS), 2),
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(res["ms_per_step"], 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "e4m3",
+        "data": "synthetic",
+        "config": cfg,
+        "roofline": {
+            "kernel": "scaled_fp8_gemm_kernel",
+            "bound": "tensor",
+            "achieved": round(gemm_tflops, 1),
+            "peak": round(fp8_peak, 1),
+            "unit": "TFLOP/s",
+            "frac": round(gemm_tflops / fp8_peak, 4),
+            "traffic": None,
+            "peak_source": f"{peak_src} bf16 {'sustained' if sustained else 'burst'} x {FP8_OVER_BF16} "
+                           f"(nominal fp8/bf16 dense ratio)",
+            "avg_launch_ms": round(gemm_avg_ms, 4),
+            "frac_of_fp8_spec": round(gemm_tflops / FP8_SPEC_TFLOPS, 4),
+        },
+        "quantizer": {
+            "kernel": "quant_rows_kernel",
+            "bound": "hbm",
+            "achieved": None if quant_gbs is None else round(quant_gbs, 1),
+            "peak": peaks.get("hbm_gbs", FALLBACK_HBM_GBS),
+            "unit": "GB/s",
+            "frac": None if quant_gbs is None else round(quant_gbs / peaks.get("hbm_gbs", FALLBACK_HBM_GBS), 4),
+            "share_of_step": round(res["quant_ms_total"] / (res["ms_per_step"] * args.steps), 4),
+        },
+        "per_linear_ms": {k: round(statistics.median(v), 4) for k, v in res["per_linear"].items()},
+        "gpu_launches": res["gpu_launches"],
+        "clocks": res["clocks"],
+    }
+    if e2e is not None:
+        e2e["value"] = round(world * e2e["value"], 3)
+        line["e2e"] = e2e
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(wl, args.cpu_seconds)
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def reference_arm(args, wl, cfg, world):
+    """The oracle, as it stands, timed on the host cores; each step is a
+    bounded sample of the workload."""
+    import oracle
+    per_step = max(2.0, min(15.0, 150.0 / max(1, args.steps + args.warmup)))
+    for i in range(args.warmup):
+        oracle_sample(wl, per_step, seed=1000 + i)
+    flops = 0
+    secs = 0.0
+    desc = ""
+    for i in range(args.steps):
+        f, s, desc = oracle_sample(wl, per_step, seed=i)
+        flops += f
+        secs += s
+    value = flops / secs / 1e12
+    line = {
+        "metric": METRIC, "impl": "reference", "value": value, "unit": "TFLOP/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * secs / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": cfg,
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
+                         "sample": "each step: " + desc},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,144 @@
+/*
+ * tfq.h -- C ABI of libtfq.so, a B200 (sm_100a) W8A8 scaled-FP8 Linear.
+ *
+ * The Linear the source pages describe is two steps:
+ *   1. per-token dynamic absmax quantization of BF16 activations to E4M3FN,
+ *        s[m] = max_k |x[m,k]| / qmax,  q[m,k] = cast_E4M3FN(clamp(x[m,k] / s[m]))
+ *      (TeleFuser "Quantization" page, section "Scaled FP8 checkpoints: W8A8";
+ *       qmax 14 and 7 from the LightX2V "模型量化技术" page, section
+ *       "MiniMax-H3 FP8 FP16 累加");
+ *   2. a scaled GEMM against per-output-channel FP8 weights with BF16 output,
+ *        y[m,n] = s_a[m] * s_w[n] * sum_k q_a[m,k] * q_w[n,k]  (+ bias[n])
+ *      (same TeleFuser page, sections "Scaled FP8 checkpoints" and
+ *       "tf-kernel FP8: online W8A8").
+ * The per-output-channel weight converter (FP8, or INT8 with
+ *   s = max|x| / 127, q = clamp(round(x / s), -128, 127),
+ * TeleFuser "Quantization" page, sections "Core ideas" and "Offline
+ * conversion") ships in the same library.
+ *
+ * Conventions shared by every entry point:
+ *  - Every data pointer is a DEVICE pointer owned by the caller; the library
+ *    never frees or keeps it.  Matrices are dense and row-major; a row is
+ *    K contiguous elements.  E4M3FN codes and INT8 codes are bytes with the
+ *    same bit patterns as torch.float8_e4m3fn / torch.int8.  Scales are fp32.
+ *  - Every data pointer must be 16-byte aligned, and K must be a multiple
+ *    of 16 (rows are then 16-byte aligned too).
+ *  - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
+ *    stream of the current device).  Work is enqueued asynchronously on it
+ *    on the CURRENT device; the call returns once the launch is enqueued.
+ *  - Return value: TFQ_OK, or an error detected before any launch
+ *    (TFQ_EINVAL for bad arguments, TFQ_EUNSUPPORTED for a device that is
+ *    not sm_100 or a size beyond a stated limit), or TFQ_ECUDA when the CUDA
+ *    runtime reports a launch error.  Nothing is launched when an argument
+ *    check fails.
+ *  - Device-side failures: every wait inside the kernels is bounded; a wait
+ *    that runs out sets a per-device error word and the kernel returns.
+ *    tfq_device_error() reports and clears it (TFQ_ETIMEOUT).
+ *  - Rounding is fixed so that results are reproducible bit for bit:
+ *    the scale is the fp32 IEEE quotient max(amax, 1e-12) / qmax, the
+ *    element quotient x / s is an fp32 IEEE division, the FP8 cast rounds
+ *    to nearest even and saturates, the INT8 rounding is half-to-even.
+ *  - Thread safety: calls may come from several host threads; the library
+ *    keeps per-device state (launch attributes, the error word, a small
+ *    TMA-descriptor cache) behind a mutex.
+ */
+#ifndef TFQ_H_
+#define TFQ_H_
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define TFQ_API __attribute__((visibility("default")))
+#else
+#define TFQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum tfq_status {
+    TFQ_OK = 0,
+    TFQ_EINVAL = 1,        /* null/misaligned pointer, bad size or qmax      */
+    TFQ_EUNSUPPORTED = 2,  /* not an sm_100 device, or a size beyond a limit  */
+    TFQ_ECUDA = 3,         /* the CUDA runtime reported an error              */
+    TFQ_ETIMEOUT = 4       /* a bounded device-side wait ran out             */
+} tfq_status;
+
+/* Output element type of the per-row weight quantizer. */
+enum { TFQ_DTYPE_FP8_E4M3 = 0, TFQ_DTYPE_INT8 = 1 };
+
+/* Largest K (row length) the row quantizers accept: a row is staged whole
+ * in shared memory.  Larger K returns TFQ_EUNSUPPORTED. */
+#define TFQ_QUANT_MAX_K 32768
+
+/*
+ * Per-token FP8 activation quantization (step 1 above).
+ *   x_bf16 : [M, K] bf16, read only.
+ *   qmax   : fp32, 1 <= qmax <= 448 (the pages use 448, 14 and 7).
+ *   q_e4m3 : [M, K] bytes, written: E4M3FN codes of clamp(x/s, -qmax, qmax).
+ *   s      : [M] fp32, written: s[m] = fl32(max(amax_m, 1e-12f) / qmax).
+ * M == 0 is a no-op.  K == 0 writes s only (amax of an empty row is 0).
+ * Errors: TFQ_EINVAL (null or misaligned pointer with M > 0, M or K < 0,
+ * K % 16 != 0, qmax outside [1, 448] or not finite), TFQ_EUNSUPPORTED
+ * (K > TFQ_QUANT_MAX_K, M >= 2^31, not sm_100).
+ */
+TFQ_API tfq_status tfq_quant_act_fp8_per_token(const void *x_bf16, int64_t M, int64_t K, float qmax,
+                                       void *q_e4m3, float *s, void *stream);
+
+/*
+ * Per-output-channel weight quantization: the same row quantizer applied to
+ * the rows (output channels) of an nn.Linear weight [N, K].
+ *   dtype == TFQ_DTYPE_FP8_E4M3 : as tfq_quant_act_fp8_per_token, qmax in [1, 448];
+ *   dtype == TFQ_DTYPE_INT8     : s[n] = fl32(max(amax_n, 1e-12f) / qmax),
+ *                                 q = clamp(round_half_even(fl32(w / s)), -128, 127),
+ *                                 qmax in [1, 127] (the pages use 127).
+ *   q : [N, K] bytes (E4M3FN codes or int8), s : [N] fp32.
+ * Errors as for tfq_quant_act_fp8_per_token; an unknown dtype is TFQ_EINVAL.
+ */
+TFQ_API tfq_status tfq_quant_weight_per_channel(const void *w_bf16, int64_t N, int64_t K, int dtype,
+                                        float qmax, void *q, float *s, void *stream);
+
+/*
+ * Scaled FP8 Linear (step 2 above), "TN": both operands K-contiguous.
+ *   A_q  : [M, K] E4M3FN codes (per-token quantized activations).
+ *   s_a  : [M] fp32 per-token scales.
+ *   W_q  : [N, K] E4M3FN codes (per-output-channel quantized weight).
+ *   s_w  : [N] fp32 per-channel scales.
+ *   bias_bf16 : [N] bf16, or NULL for no bias.
+ *   out_bf16  : [M, N] bf16, written:
+ *       out[m,n] = bf16_rn(fp32(sum_k A_q[m,k] W_q[n,k]) * s_a[m] * s_w[n] + bias[n]).
+ * The products are accumulated in fp32 on the tensor cores; the result is
+ * within |y - y_exact| <= 2^-7 |y_exact| + 1e-3 rms(y_exact) of the exact
+ * value (the tests check this bound).
+ * M == 0 or N == 0 is a no-op.
+ * Errors: TFQ_EINVAL (null/misaligned pointer, K <= 0, K % 16 != 0,
+ * N % 8 != 0, negative sizes), TFQ_EUNSUPPORTED (M, N or K >= 2^31,
+ * not sm_100).
+ */
+TFQ_API tfq_status tfq_scaled_fp8_linear(const void *A_q, const float *s_a, const void *W_q,
+                                 const float *s_w, const void *bias_bf16, int64_t M, int64_t N,
+                                 int64_t K, void *out_bf16, void *stream);
+
+/*
+ * Synchronizes `stream`, then reads and clears the current device's error
+ * word.  Returns TFQ_ETIMEOUT if a bounded wait inside a kernel ran out
+ * since the last call (the outputs of that launch are then incomplete),
+ * TFQ_ECUDA if the synchronization itself failed, TFQ_OK otherwise.
+ */
+TFQ_API tfq_status tfq_device_error(void *stream);
+
+/* Static string naming a status ("TFQ_OK", ...); "unknown" otherwise. */
+TFQ_API const char *tfq_status_string(int status);
+
+/* Thread-local text of the last error this thread's calls returned. */
+TFQ_API const char *tfq_last_error_message(void);
+
+/* ABI version: 100 * major + minor. */
+TFQ_API int tfq_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TFQ_H_ */

@@ -1,0 +1,40 @@
+"""B200-native (sm_100a) W8A8 scaled-FP8 Linear.
+
+The computation lives in libtfq.so (include/tfq.h): a per-row absmax
+quantizer (BF16 -> E4M3FN or INT8 with one fp32 scale per row) and a
+tcgen05/TMEM/TMA scaled FP8 GEMM with a fused scale/bias/BF16 epilogue.
+This package is its Python binding; torch supplies device memory and
+streams.  Build the library with ``python -m int8_w8a8_quantized_b200.build``.
+"""
+from ._capi import (  # noqa: F401
+    LIB_PATH,
+    SIGNATURES,
+    TFQ_DTYPE_FP8_E4M3,
+    TFQ_DTYPE_INT8,
+    TFQ_EINVAL,
+    TFQ_ECUDA,
+    TFQ_ETIMEOUT,
+    TFQ_EUNSUPPORTED,
+    TFQ_OK,
+    TFQ_QUANT_MAX_K,
+    TfqError,
+    last_error_message,
+    load_library,
+    raw,
+    status_string,
+    tfq_device_error,
+    tfq_quant_act_fp8_per_token,
+    tfq_quant_weight_per_channel,
+    tfq_scaled_fp8_linear,
+    w8a8_linear,
+)
+
+__all__ = [
+    "tfq_quant_act_fp8_per_token",
+    "tfq_quant_weight_per_channel",
+    "tfq_scaled_fp8_linear",
+    "tfq_device_error",
+    "w8a8_linear",
+    "TfqError",
+    "raw",
+]

@@ -1,0 +1,198 @@
+"""ctypes binding of libtfq.so (include/tfq.h).
+
+Two layers, both argument marshalling only (every step runs in the CUDA
+library):
+
+* ``raw``: the C functions with their C signatures (integers for pointers,
+  a stream handle as an integer); the tests call the library through these;
+* functions named like the C entry points that take torch CUDA tensors,
+  check dtypes/shapes/devices, allocate outputs when none are given, pass
+  ``data_ptr()`` and the current CUDA stream, and raise ``TfqError`` on a
+  non-zero status.
+
+There is no fallback: if libtfq.so is missing or cannot be loaded, every
+call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "libtfq.so")
+
+TFQ_OK, TFQ_EINVAL, TFQ_EUNSUPPORTED, TFQ_ECUDA, TFQ_ETIMEOUT = range(5)
+TFQ_DTYPE_FP8_E4M3, TFQ_DTYPE_INT8 = 0, 1
+TFQ_QUANT_MAX_K = 32768
+
+# name -> (restype, argtypes), in the order include/tfq.h declares them
+_P, _I64, _F, _I = ctypes.c_void_p, ctypes.c_int64, ctypes.c_float, ctypes.c_int
+SIGNATURES = {
+    "tfq_quant_act_fp8_per_token": (_I, [_P, _I64, _I64, _F, _P, _P, _P]),
+    "tfq_quant_weight_per_channel": (_I, [_P, _I64, _I64, _I, _F, _P, _P, _P]),
+    "tfq_scaled_fp8_linear": (_I, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _P]),
+    "tfq_device_error": (_I, [_P]),
+    "tfq_status_string": (ctypes.c_char_p, [_I]),
+    "tfq_last_error_message": (ctypes.c_char_p, []),
+    "tfq_version": (_I, []),
+}
+
+_lock = threading.Lock()
+_lib = None
+
+
+class TfqError(RuntimeError):
+    def __init__(self, status: int, where: str, message: str):
+        super().__init__(f"{where}: {status_string(status)}: {message}")
+        self.status = status
+
+
+def load_library(path: str | None = None) -> ctypes.CDLL:
+    """Loads libtfq.so (once).  Raises if it is missing: there is no fallback."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        p = path or LIB_PATH
+        if not os.path.exists(p):
+            raise RuntimeError(f"{p} is not built; run `python -m int8_w8a8_quantized_b200.build`")
+        lib = ctypes.CDLL(p)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = lib
+        return lib
+
+
+class _Raw:
+    """The C entry points with their C signatures."""
+
+    def __getattr__(self, name):
+        if name not in SIGNATURES:
+            raise AttributeError(name)
+        return getattr(load_library(), name)
+
+
+raw = _Raw()
+
+
+def status_string(status: int) -> str:
+    return load_library().tfq_status_string(int(status)).decode()
+
+
+def last_error_message() -> str:
+    return load_library().tfq_last_error_message().decode()
+
+
+def _check(status: int, where: str) -> None:
+    if status != TFQ_OK:
+        raise TfqError(status, where, last_error_message())
+
+
+def _stream_handle(stream) -> int:
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(stream.cuda_stream) if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _require(t, dtype, ndim, name):
+    import torch
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.dim() != ndim:
+        raise ValueError(f"{name} must be {ndim}-D")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def tfq_quant_act_fp8_per_token(x, qmax: float = 448.0, q=None, s=None, stream=None):
+    """x bf16 [M, K] -> (q uint8 [M, K] E4M3FN codes, s fp32 [M])."""
+    import torch
+    _require(x, torch.bfloat16, 2, "x")
+    M, K = x.shape
+    if q is None:
+        q = torch.empty((M, K), dtype=torch.uint8, device=x.device)
+    if s is None:
+        s = torch.empty((M,), dtype=torch.float32, device=x.device)
+    _require(q, torch.uint8, 2, "q")
+    _require(s, torch.float32, 1, "s")
+    if tuple(q.shape) != (M, K) or tuple(s.shape) != (M,):
+        raise ValueError("output shapes do not match x")
+    with torch.cuda.device(x.device):
+        st = raw.tfq_quant_act_fp8_per_token(x.data_ptr(), M, K, float(qmax), q.data_ptr(), s.data_ptr(),
+                                             _stream_handle(stream))
+    _check(st, "tfq_quant_act_fp8_per_token")
+    return q, s
+
+
+def tfq_quant_weight_per_channel(w, dtype: str = "fp8", qmax: float | None = None, q=None, s=None, stream=None):
+    """w bf16 [N, K] -> (codes [N, K] (uint8 E4M3FN or int8), s fp32 [N])."""
+    import torch
+    _require(w, torch.bfloat16, 2, "w")
+    N, K = w.shape
+    if dtype == "fp8":
+        code, qdt, qmax = TFQ_DTYPE_FP8_E4M3, torch.uint8, 448.0 if qmax is None else qmax
+    elif dtype == "int8":
+        code, qdt, qmax = TFQ_DTYPE_INT8, torch.int8, 127.0 if qmax is None else qmax
+    else:
+        raise ValueError("dtype must be 'fp8' or 'int8'")
+    if q is None:
+        q = torch.empty((N, K), dtype=qdt, device=w.device)
+    if s is None:
+        s = torch.empty((N,), dtype=torch.float32, device=w.device)
+    _require(q, qdt, 2, "q")
+    _require(s, torch.float32, 1, "s")
+    if tuple(q.shape) != (N, K) or tuple(s.shape) != (N,):
+        raise ValueError("output shapes do not match w")
+    with torch.cuda.device(w.device):
+        st = raw.tfq_quant_weight_per_channel(w.data_ptr(), N, K, code, float(qmax), q.data_ptr(), s.data_ptr(),
+                                              _stream_handle(stream))
+    _check(st, "tfq_quant_weight_per_channel")
+    return q, s
+
+
+def tfq_scaled_fp8_linear(A_q, s_a, W_q, s_w, bias=None, out=None, stream=None):
+    """A_q uint8 [M, K], s_a fp32 [M], W_q uint8 [N, K], s_w fp32 [N], bias bf16 [N] or None
+    -> out bf16 [M, N]."""
+    import torch
+    _require(A_q, torch.uint8, 2, "A_q")
+    _require(W_q, torch.uint8, 2, "W_q")
+    _require(s_a, torch.float32, 1, "s_a")
+    _require(s_w, torch.float32, 1, "s_w")
+    M, K = A_q.shape
+    N, K2 = W_q.shape
+    if K2 != K or s_a.shape[0] != M or s_w.shape[0] != N:
+        raise ValueError("shape mismatch")
+    if bias is not None:
+        _require(bias, torch.bfloat16, 1, "bias")
+        if bias.shape[0] != N:
+            raise ValueError("bias shape")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=A_q.device)
+    _require(out, torch.bfloat16, 2, "out")
+    if tuple(out.shape) != (M, N):
+        raise ValueError("out shape")
+    with torch.cuda.device(A_q.device):
+        st = raw.tfq_scaled_fp8_linear(A_q.data_ptr(), s_a.data_ptr(), W_q.data_ptr(), s_w.data_ptr(),
+                                       None if bias is None else bias.data_ptr(), M, N, K, out.data_ptr(),
+                                       _stream_handle(stream))
+    _check(st, "tfq_scaled_fp8_linear")
+    return out
+
+
+def tfq_device_error(stream=None) -> None:
+    """Raises TfqError(TFQ_ETIMEOUT) if a bounded device wait ran out."""
+    _check(raw.tfq_device_error(_stream_handle(stream)), "tfq_device_error")
+
+
+def w8a8_linear(x, W_q, s_w, bias=None, qmax: float = 448.0, stream=None):
+    """The whole Linear: per-token FP8 quantization of x, then the scaled GEMM."""
+    A_q, s_a = tfq_quant_act_fp8_per_token(x, qmax, stream=stream)
+    return tfq_scaled_fp8_linear(A_q, s_a, W_q, s_w, bias, stream=stream)

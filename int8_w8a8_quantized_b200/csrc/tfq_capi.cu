@@ -1,0 +1,203 @@
+// tfq_capi.cu -- the extern "C" entry points of libtfq.so: argument
+// validation, per-device state, TMA descriptor encoding, launches.
+// See include/tfq.h for the contract of every function.
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <mutex>
+
+#include "tfq_internal.h"
+
+namespace tfq {
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_mutex;
+DeviceState g_states[kMaxDevices];
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+thread_local char g_last_error[512] = "";
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+tfq_status resolve_encode() {
+    if (g_encode != nullptr) return TFQ_OK;
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    const cudaError_t e = cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000,
+                                                           cudaEnableDefault, &q);
+    if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || fn == nullptr)
+        return fail(TFQ_ECUDA, "cannot resolve cuTensorMapEncodeTiled: %s", cudaGetErrorString(e));
+    g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    return TFQ_OK;
+}
+
+}  // namespace
+
+tfq_status fail(tfq_status st, const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_last_error, sizeof g_last_error, fmt, ap);
+    va_end(ap);
+    return st;
+}
+
+DeviceState* current_device_state(tfq_status* st) {
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) {
+        *st = fail(TFQ_ECUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+        return nullptr;
+    }
+    if (dev < 0 || dev >= kMaxDevices) {
+        *st = fail(TFQ_EUNSUPPORTED, "device ordinal %d out of range", dev);
+        return nullptr;
+    }
+    std::lock_guard<std::mutex> lock(g_mutex);
+    DeviceState* ds = &g_states[dev];
+    if (ds->device < 0) {
+        cudaDeviceProp prop;
+        e = cudaGetDeviceProperties(&prop, dev);
+        if (e != cudaSuccess) {
+            *st = fail(TFQ_ECUDA, "cudaGetDeviceProperties: %s", cudaGetErrorString(e));
+            return nullptr;
+        }
+        if (prop.major != 10 || prop.minor != 0) {
+            *st = fail(TFQ_EUNSUPPORTED, "device %d is sm_%d%d; this library is built for sm_100a", dev, prop.major,
+                       prop.minor);
+            return nullptr;
+        }
+        uint32_t* err_word = nullptr;
+        e = cudaMalloc(&err_word, sizeof(uint32_t));
+        if (e == cudaSuccess) e = cudaMemset(err_word, 0, sizeof(uint32_t));
+        if (e != cudaSuccess) {
+            *st = fail(TFQ_ECUDA, "allocating the device error word: %s", cudaGetErrorString(e));
+            return nullptr;
+        }
+        tfq_status rs = resolve_encode();
+        if (rs != TFQ_OK) {
+            *st = rs;
+            return nullptr;
+        }
+        ds->sm_count = prop.multiProcessorCount;
+        ds->cc_major = prop.major;
+        ds->cc_minor = prop.minor;
+        ds->smem_optin = prop.sharedMemPerBlockOptin;
+        ds->err_word = err_word;
+        ds->device = dev;
+    }
+    *st = TFQ_OK;
+    return ds;
+}
+
+tfq_status encode_tensor_map_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, uint64_t inner,
+                                uint64_t outer, uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer,
+                                CUtensorMapSwizzle swizzle) {
+    const cuuint64_t dims[2] = {inner, outer};
+    const cuuint64_t strides[1] = {row_stride_bytes};
+    const cuuint32_t box[2] = {box_inner, box_outer};
+    const cuuint32_t estride[2] = {1, 1};
+    const CUresult r = g_encode(map, dtype, 2, const_cast<void*>(base), dims, strides, box, estride,
+                                CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(TFQ_ECUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+    return TFQ_OK;
+}
+
+}  // namespace tfq
+
+using namespace tfq;
+
+namespace {
+
+tfq_status check_quant_args(const void* x, int64_t M, int64_t K, const void* q, const float* s, float qmax,
+                            float qmax_hi) {
+    if (M < 0 || K < 0) return fail(TFQ_EINVAL, "negative size (M=%lld, K=%lld)", (long long)M, (long long)K);
+    if (K % 16 != 0) return fail(TFQ_EINVAL, "K=%lld is not a multiple of 16", (long long)K);
+    if (!std::isfinite(qmax) || qmax < 1.0f || qmax > qmax_hi)
+        return fail(TFQ_EINVAL, "qmax=%g outside [1, %g]", (double)qmax, (double)qmax_hi);
+    if (K > TFQ_QUANT_MAX_K) return fail(TFQ_EUNSUPPORTED, "K=%lld above %d", (long long)K, TFQ_QUANT_MAX_K);
+    if (M >= (int64_t(1) << 31)) return fail(TFQ_EUNSUPPORTED, "M=%lld too large", (long long)M);
+    if (M == 0) return TFQ_OK;
+    if (s == nullptr || (K > 0 && (x == nullptr || q == nullptr)))
+        return fail(TFQ_EINVAL, "null pointer");
+    if (!aligned16(x) || !aligned16(q) || !aligned16(s)) return fail(TFQ_EINVAL, "pointer not 16-byte aligned");
+    return TFQ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+tfq_status tfq_quant_act_fp8_per_token(const void* x_bf16, int64_t M, int64_t K, float qmax, void* q_e4m3,
+                                       float* s, void* stream) {
+    tfq_status st = check_quant_args(x_bf16, M, K, q_e4m3, s, qmax, 448.0f);
+    if (st != TFQ_OK || M == 0) return st;
+    DeviceState* ds = current_device_state(&st);
+    if (ds == nullptr) return st;
+    return launch_quant_rows(x_bf16, M, K, qmax, false, q_e4m3, s, static_cast<cudaStream_t>(stream), ds);
+}
+
+tfq_status tfq_quant_weight_per_channel(const void* w_bf16, int64_t N, int64_t K, int dtype, float qmax, void* q,
+                                        float* s, void* stream) {
+    if (dtype != TFQ_DTYPE_FP8_E4M3 && dtype != TFQ_DTYPE_INT8) return fail(TFQ_EINVAL, "unknown dtype %d", dtype);
+    const bool is_int8 = dtype == TFQ_DTYPE_INT8;
+    tfq_status st = check_quant_args(w_bf16, N, K, q, s, qmax, is_int8 ? 127.0f : 448.0f);
+    if (st != TFQ_OK || N == 0) return st;
+    DeviceState* ds = current_device_state(&st);
+    if (ds == nullptr) return st;
+    return launch_quant_rows(w_bf16, N, K, qmax, is_int8, q, s, static_cast<cudaStream_t>(stream), ds);
+}
+
+tfq_status tfq_scaled_fp8_linear(const void* A_q, const float* s_a, const void* W_q, const float* s_w,
+                                 const void* bias_bf16, int64_t M, int64_t N, int64_t K, void* out_bf16,
+                                 void* stream) {
+    if (M < 0 || N < 0 || K < 0) return fail(TFQ_EINVAL, "negative size");
+    if (K == 0 || K % 16 != 0) return fail(TFQ_EINVAL, "K=%lld must be a positive multiple of 16", (long long)K);
+    if (N % 8 != 0) return fail(TFQ_EINVAL, "N=%lld is not a multiple of 8", (long long)N);
+    const int64_t lim = int64_t(1) << 31;
+    if (M >= lim || N >= lim || K >= lim) return fail(TFQ_EUNSUPPORTED, "size too large");
+    if (M == 0 || N == 0) return TFQ_OK;
+    if (A_q == nullptr || s_a == nullptr || W_q == nullptr || s_w == nullptr || out_bf16 == nullptr)
+        return fail(TFQ_EINVAL, "null pointer");
+    if (!aligned16(A_q) || !aligned16(s_a) || !aligned16(W_q) || !aligned16(s_w) || !aligned16(out_bf16) ||
+        (bias_bf16 != nullptr && !aligned16(bias_bf16)))
+        return fail(TFQ_EINVAL, "pointer not 16-byte aligned");
+    tfq_status st;
+    DeviceState* ds = current_device_state(&st);
+    if (ds == nullptr) return st;
+    return launch_scaled_fp8_gemm(A_q, s_a, W_q, s_w, bias_bf16, M, N, K, out_bf16,
+                                  static_cast<cudaStream_t>(stream), ds);
+}
+
+tfq_status tfq_device_error(void* stream) {
+    tfq_status st;
+    DeviceState* ds = current_device_state(&st);
+    if (ds == nullptr) return st;
+    cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return fail(TFQ_ECUDA, "cudaStreamSynchronize: %s", cudaGetErrorString(e));
+    uint32_t word = 0;
+    e = cudaMemcpy(&word, ds->err_word, sizeof word, cudaMemcpyDeviceToHost);
+    if (e == cudaSuccess && word != 0) e = cudaMemset(ds->err_word, 0, sizeof(uint32_t));
+    if (e != cudaSuccess) return fail(TFQ_ECUDA, "reading the error word: %s", cudaGetErrorString(e));
+    if (word != 0) return fail(TFQ_ETIMEOUT, "a bounded device wait ran out (error bits 0x%x)", word);
+    return TFQ_OK;
+}
+
+const char* tfq_status_string(int status) {
+    switch (status) {
+        case TFQ_OK: return "TFQ_OK";
+        case TFQ_EINVAL: return "TFQ_EINVAL";
+        case TFQ_EUNSUPPORTED: return "TFQ_EUNSUPPORTED";
+        case TFQ_ECUDA: return "TFQ_ECUDA";
+        case TFQ_ETIMEOUT: return "TFQ_ETIMEOUT";
+        default: return "unknown";
+    }
+}
+
+const char* tfq_last_error_message(void) { return g_last_error; }
+
+int tfq_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,351 @@
+// tfq_gemm.cu -- scaled FP8 GEMM with fused epilogue on 5th-generation
+// tensor cores (tcgen05, sm_100a).
+//
+// Computes out[m,n] = bf16_rn(acc[m,n] * s_a[m] * s_w[n] + bias[n]) with
+// acc[m,n] = sum_k e4m3(A[m,k]) * e4m3(W[n,k]) accumulated in fp32: the
+// scaled GEMM of the TeleFuser "Quantization" page (sections "Scaled FP8
+// checkpoints" and "tf-kernel FP8: online W8A8": per-token activation
+// scales, per-output-channel weight scales, BF16 output).
+//
+// Kernel structure (one persistent CTA per SM, 192 threads):
+//   warp 0      TMA producer: streams 128x128 A tiles and 256x128 B tiles
+//               (K-major, 128-byte swizzle) into a 4-stage shared-memory
+//               ring, completion counted on "full" mbarriers.
+//   warp 1      allocates 512 TMEM columns (two 128x256 fp32 accumulators)
+//               and, from one thread, issues tcgen05.mma kind::f8f6f4
+//               (M=128, N=256, K=32 per instruction, 4 per stage); each
+//               stage is released to the producer by tcgen05.commit onto its
+//               "empty" mbarrier, each finished tile by a commit onto the
+//               accumulator's "tmem_full" mbarrier.
+//   warps 2..5  epilogue: tcgen05.ld a 32-row quarter of the accumulator
+//               (warp w may read TMEM lanes 32*(w%4)..+31), apply s_a, s_w
+//               and bias in fp32, round to bf16, write 64-column chunks into
+//               a 128-byte-swizzled staging buffer and TMA-store them; the
+//               accumulator is handed back through "tmem_empty" so the MMA
+//               of the next tile overlaps this epilogue.
+// Tiles are visited in M-grouped raster order so that the CTAs running at
+// the same time share A and B panels in L2.  M and N tails are handled by
+// TMA (zero fill on load, clipping on store); K tails by zero fill.
+// Every wait is bounded (see tfq_ptx.cuh); a CTA that gives up records it in
+// the error word, drains its own outstanding copies and MMAs, frees TMEM and
+// returns.
+#include <cuda_bf16.h>
+
+#include <algorithm>
+
+#include "tfq_internal.h"
+#include "tfq_ptx.cuh"
+
+namespace tfq {
+namespace {
+
+constexpr int BM = 128;            // tile rows (tokens)
+constexpr int BN = 256;            // tile columns (output channels)
+constexpr int BK = 128;            // K elements (= bytes) per stage: one 128-byte swizzle atom
+constexpr int UMMA_K = 32;         // K per tcgen05.mma for 8-bit operands
+constexpr int STAGES = 4;
+constexpr int A_STAGE_BYTES = BM * BK;  // 16 KiB
+constexpr int B_STAGE_BYTES = BN * BK;  // 32 KiB
+constexpr int EPI_WARPS = 4;
+constexpr int EPI_COLS = 64;                         // bf16 columns per TMA store (128 bytes)
+constexpr int EPI_BUF_BYTES = 32 * EPI_COLS * 2;     // 4 KiB per staging buffer
+constexpr int THREADS = 64 + EPI_WARPS * 32;         // producer warp, MMA warp, epilogue warps
+constexpr int TMEM_COLS = 2 * BN;                    // double-buffered accumulator
+constexpr int GROUP_M = 16;
+
+constexpr size_t SMEM_RING = static_cast<size_t>(STAGES) * (A_STAGE_BYTES + B_STAGE_BYTES);
+constexpr size_t SMEM_EPI = static_cast<size_t>(EPI_WARPS) * 2 * EPI_BUF_BYTES;
+constexpr size_t SMEM_BARS = (2 * STAGES + 4 + 1) * 8 + 16;
+constexpr size_t SMEM_BYTES = 1024 /* alignment slack */ + SMEM_RING + SMEM_EPI + SMEM_BARS;
+static_assert(SMEM_BYTES <= 232448, "shared memory budget exceeded");
+
+// Instruction descriptor of tcgen05.mma kind::f8f6f4: fp32 accumulator
+// (bits 4-5 = 1), A and B E4M3 (format 0 in bits 7-9 and 10-12), both
+// K-major (bits 15, 16 = 0), N >> 3 in bits 17-22, M >> 4 in bits 24-28.
+constexpr uint32_t IDESC = (1u << 4) | (static_cast<uint32_t>(BN >> 3) << 17) | (static_cast<uint32_t>(BM >> 4) << 24);
+
+struct GemmArgs {
+    const float* s_a;
+    const float* s_w;
+    const uint16_t* bias;  // may be null
+    int M, N, K;
+    int m_tiles, n_tiles, k_blocks;
+    uint32_t* err;
+};
+
+__device__ __forceinline__ void tile_coords(int t, const GemmArgs& p, int& tm, int& tn) {
+    const int per_group = GROUP_M * p.n_tiles;
+    const int gid = t / per_group;
+    const int first_m = gid * GROUP_M;
+    const int gsize = min(p.m_tiles - first_m, GROUP_M);
+    const int r = t - gid * per_group;
+    tm = first_m + r % gsize;
+    tn = r / gsize;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    uint32_t d;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
+    return d;
+}
+
+__device__ __forceinline__ void give_up(volatile int* abort_flag, uint32_t* err, uint32_t bit) {
+    *abort_flag = 1;
+    atomicOr(err, bit);
+}
+
+__global__ void __launch_bounds__(THREADS, 1)
+    scaled_fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                           const __grid_constant__ CUtensorMap tmY, GemmArgs p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* sA = smem;
+    uint8_t* sB = sA + STAGES * A_STAGE_BYTES;
+    uint8_t* sE = sB + STAGES * B_STAGE_BYTES;
+    uint64_t* full = reinterpret_cast<uint64_t*>(sE + SMEM_EPI);
+    uint64_t* empty = full + STAGES;
+    uint64_t* tmem_full = empty + STAGES;
+    uint64_t* tmem_empty = tmem_full + 2;
+    uint64_t* drain = tmem_empty + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int total_tiles = p.m_tiles * p.n_tiles;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < STAGES; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&tmem_full[i], 1);
+            mbar_init(&tmem_empty[i], EPI_WARPS);
+        }
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+        prefetch_tensormap(&tmA);
+        prefetch_tensormap(&tmB);
+        prefetch_tensormap(&tmY);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == 0) {
+        // ---------------------------------------------------- TMA producer
+        if (lane == 0) {
+            int it = 0;
+            int issued_phase[STAGES];
+            for (int i = 0; i < STAGES; ++i) issued_phase[i] = -1;
+            bool ok = true;
+            for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
+                int tm, tn;
+                tile_coords(t, p, tm, tn);
+                for (int kb = 0; kb < p.k_blocks; ++kb, ++it) {
+                    const int st = it % STAGES;
+                    const uint32_t ph = static_cast<uint32_t>(it / STAGES) & 1u;
+                    if (!mbar_wait(&empty[st], ph ^ 1u, abort_flag)) {
+                        give_up(abort_flag, p.err, kErrGemmProducer);
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&full[st], A_STAGE_BYTES + B_STAGE_BYTES);
+                    tma_load_2d(sA + st * A_STAGE_BYTES, &tmA, kb * BK, tm * BM, &full[st]);
+                    tma_load_2d(sB + st * B_STAGE_BYTES, &tmB, kb * BK, tn * BN, &full[st]);
+                    issued_phase[st] = static_cast<int>(ph);
+                }
+            }
+            // Outstanding loads must land before the CTA may exit.
+            for (int i = 0; i < STAGES; ++i)
+                if (issued_phase[i] >= 0 && !mbar_wait(&full[i], static_cast<uint32_t>(issued_phase[i]), nullptr))
+                    atomicOr(p.err, kErrGemmDrain);
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            int it = 0, tcount = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x, ++tcount) {
+                const int buf = tcount & 1;
+                const uint32_t use = static_cast<uint32_t>(tcount >> 1);
+                if (!mbar_wait(&tmem_empty[buf], (use & 1u) ^ 1u, abort_flag)) {
+                    give_up(abort_flag, p.err, kErrGemmMma);
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * BN);
+                for (int kb = 0; kb < p.k_blocks; ++kb, ++it) {
+                    const int st = it % STAGES;
+                    const uint32_t ph = static_cast<uint32_t>(it / STAGES) & 1u;
+                    if (!mbar_wait(&full[st], ph, abort_flag)) {
+                        give_up(abort_flag, p.err, kErrGemmMma);
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint64_t a_desc = sw128_kmajor_desc(sA + st * A_STAGE_BYTES);
+                    const uint64_t b_desc = sw128_kmajor_desc(sB + st * B_STAGE_BYTES);
+#pragma unroll
+                    for (int k = 0; k < BK / UMMA_K; ++k) {
+                        // advance the start address by k * 32 bytes inside the swizzle atom
+                        const uint64_t koff = static_cast<uint64_t>((k * UMMA_K) >> 4);
+                        mma_e4m3(d_tmem, a_desc + koff, b_desc + koff, IDESC, (kb | k) != 0 ? 1u : 0u);
+                    }
+                    mma_commit(&empty[st]);
+                }
+                if (ok) mma_commit(&tmem_full[buf]);
+            }
+            // Every MMA issued above must finish before TMEM is freed.
+            mma_commit(drain);
+            if (!mbar_wait(drain, 0, nullptr)) atomicOr(p.err, kErrGemmDrain);
+        }
+    } else {
+        // -------------------------------------------------------- epilogue
+        const int ew = warp - 2;         // 0..3: staging buffers
+        const int quarter = warp & 3;    // TMEM lanes this warp may read
+        uint8_t* ebuf0 = sE + static_cast<size_t>(ew) * 2 * EPI_BUF_BYTES;
+        int tcount = 0, chunk = 0;
+        for (int t = blockIdx.x; t < total_tiles; t += gridDim.x, ++tcount) {
+            int tm, tn;
+            tile_coords(t, p, tm, tn);
+            const int buf = tcount & 1;
+            const uint32_t use = static_cast<uint32_t>(tcount >> 1);
+            if (!mbar_wait_warp(&tmem_full[buf], use & 1u, abort_flag)) {
+                if (lane == 0) give_up(abort_flag, p.err, kErrGemmEpilogue);
+                break;
+            }
+            tc_fence_after();
+            const int row0 = tm * BM + quarter * 32;
+            const int m = row0 + lane;
+            const float sa = (m < p.M) ? __ldg(p.s_a + m) : 0.0f;
+            const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
+                                   static_cast<uint32_t>(buf * BN);
+#pragma unroll 1
+            for (int c = 0; c < BN / EPI_COLS; ++c) {
+                const int n0 = tn * BN + c * EPI_COLS;
+                if (n0 >= p.N) break;  // uniform across the warp
+                uint32_t acc[2][32];
+                tmem_ld_32x32b_x32(t_row + c * EPI_COLS, acc[0]);
+                tmem_ld_32x32b_x32(t_row + c * EPI_COLS + 32, acc[1]);
+                tmem_ld_wait();
+                uint8_t* ebuf = ebuf0 + (chunk & 1) * EPI_BUF_BYTES;
+                // The staging buffer written two chunks ago must have been read by its TMA store.
+                if (lane == 0) bulk_wait_read<1>();
+                __syncwarp();
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+#pragma unroll
+                    for (int g = 0; g < 4; ++g) {  // 8 columns -> one 16-byte unit
+                        const int nl = h * 32 + g * 8;
+                        float sw[8], bb[8];
+                        if (n0 + nl < p.N) {  // N % 8 == 0: a group is all valid or all out
+                            const float4 w0 = __ldg(reinterpret_cast<const float4*>(p.s_w + n0 + nl));
+                            const float4 w1 = __ldg(reinterpret_cast<const float4*>(p.s_w + n0 + nl + 4));
+                            sw[0] = w0.x; sw[1] = w0.y; sw[2] = w0.z; sw[3] = w0.w;
+                            sw[4] = w1.x; sw[5] = w1.y; sw[6] = w1.z; sw[7] = w1.w;
+                            if (p.bias != nullptr) {
+                                const uint4 bv = __ldg(reinterpret_cast<const uint4*>(p.bias + n0 + nl));
+                                const uint32_t bw[4] = {bv.x, bv.y, bv.z, bv.w};
+#pragma unroll
+                                for (int j = 0; j < 4; ++j) {
+                                    bb[2 * j] = __uint_as_float(bw[j] << 16);
+                                    bb[2 * j + 1] = __uint_as_float(bw[j] & 0xFFFF0000u);
+                                }
+                            } else {
+#pragma unroll
+                                for (int j = 0; j < 8; ++j) bb[j] = 0.0f;
+                            }
+                        } else {
+#pragma unroll
+                            for (int j = 0; j < 8; ++j) sw[j] = bb[j] = 0.0f;
+                        }
+                        uint32_t packed[4];
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            const float y0 = fmaf(__uint_as_float(acc[h][g * 8 + 2 * j]) * sa, sw[2 * j], bb[2 * j]);
+                            const float y1 =
+                                fmaf(__uint_as_float(acc[h][g * 8 + 2 * j + 1]) * sa, sw[2 * j + 1], bb[2 * j + 1]);
+                            packed[j] = pack_bf16x2(y0, y1);
+                        }
+                        // 128-byte swizzle: 16-byte unit u of row r lives at unit u ^ (r % 8).
+                        const int unit = h * 4 + g;
+                        uint4* dst = reinterpret_cast<uint4*>(ebuf + lane * 128 + ((unit ^ (lane & 7)) << 4));
+                        *dst = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+                    }
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    tma_store_2d(&tmY, ebuf, n0, row0);
+                    bulk_commit();
+                }
+                ++chunk;
+            }
+            // All of this warp's TMEM reads of `buf` are complete: hand it back.
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tmem_empty[buf]);
+        }
+        if (lane == 0) bulk_wait<0>();
+        __syncwarp();
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem_base, TMEM_COLS);
+    }
+}
+
+}  // namespace
+
+tfq_status launch_scaled_fp8_gemm(const void* A, const float* s_a, const void* W, const float* s_w,
+                                  const void* bias, int64_t M, int64_t N, int64_t K, void* out,
+                                  cudaStream_t stream, DeviceState* ds) {
+    if (M == 0 || N == 0) return TFQ_OK;
+    CUtensorMap tmA, tmB, tmY;
+    tfq_status st = encode_tensor_map_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, A, K, M, K, BK, BM,
+                                         CU_TENSOR_MAP_SWIZZLE_128B);
+    if (st != TFQ_OK) return st;
+    st = encode_tensor_map_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, W, K, N, K, BK, BN, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (st != TFQ_OK) return st;
+    st = encode_tensor_map_2d(&tmY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, out, N, M, N * 2, EPI_COLS, 32,
+                              CU_TENSOR_MAP_SWIZZLE_128B);
+    if (st != TFQ_OK) return st;
+    if (!ds->gemm_attr_set) {
+        const cudaError_t e = cudaFuncSetAttribute(scaled_fp8_gemm_kernel,
+                                                   cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                   static_cast<int>(SMEM_BYTES));
+        if (e != cudaSuccess) return fail(TFQ_ECUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+        ds->gemm_attr_set = true;
+    }
+    GemmArgs a;
+    a.s_a = s_a;
+    a.s_w = s_w;
+    a.bias = static_cast<const uint16_t*>(bias);
+    a.M = static_cast<int>(M);
+    a.N = static_cast<int>(N);
+    a.K = static_cast<int>(K);
+    a.m_tiles = static_cast<int>((M + BM - 1) / BM);
+    a.n_tiles = static_cast<int>((N + BN - 1) / BN);
+    a.k_blocks = static_cast<int>((K + BK - 1) / BK);
+    a.err = ds->err_word;
+    const int64_t tiles = static_cast<int64_t>(a.m_tiles) * a.n_tiles;
+    if (tiles > INT32_MAX) return fail(TFQ_EUNSUPPORTED, "too many output tiles");
+    const int grid = static_cast<int>(std::min<int64_t>(tiles, ds->sm_count));
+    scaled_fp8_gemm_kernel<<<grid, THREADS, SMEM_BYTES, stream>>>(tmA, tmB, tmY, a);
+    const cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? TFQ_OK : fail(TFQ_ECUDA, "GEMM launch: %s", cudaGetErrorString(e));
+}
+
+}  // namespace tfq

@@ -1,0 +1,54 @@
+// tfq_internal.h -- declarations shared by the C-ABI layer and the kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "tfq.h"
+
+namespace tfq {
+
+// Bits of the per-device error word (which role of which kernel gave up).
+enum : uint32_t {
+    kErrQuantProducer = 1u << 0,
+    kErrQuantConsumer = 1u << 1,
+    kErrGemmProducer = 1u << 4,
+    kErrGemmMma = 1u << 5,
+    kErrGemmEpilogue = 1u << 6,
+    kErrGemmDrain = 1u << 7,
+};
+
+struct DeviceState {
+    int device = -1;
+    int sm_count = 0;
+    int cc_major = 0, cc_minor = 0;
+    size_t smem_optin = 0;          // max dynamic shared memory per block
+    uint32_t* err_word = nullptr;   // device memory, one 32-bit word
+    bool quant_attr_set[2] = {false, false};
+    bool gemm_attr_set = false;
+};
+
+// Per-device state of the current device, created on first use.  Returns
+// nullptr and sets *st on failure.
+DeviceState* current_device_state(tfq_status* st);
+
+// Records a message for tfq_last_error_message() and returns `st`.
+tfq_status fail(tfq_status st, const char* fmt, ...);
+
+// cuTensorMapEncodeTiled, resolved through the runtime's driver entry point.
+tfq_status encode_tensor_map_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, uint64_t inner,
+                                uint64_t outer, uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer,
+                                CUtensorMapSwizzle swizzle);
+
+// Row quantizer: out_int8 == false -> E4M3FN codes, true -> INT8 codes.
+tfq_status launch_quant_rows(const void* x, int64_t rows, int64_t K, float qmax, bool out_int8, void* q, float* s,
+                             cudaStream_t stream, DeviceState* ds);
+
+// Scaled FP8 GEMM with the fused scale/bias/BF16 epilogue.
+tfq_status launch_scaled_fp8_gemm(const void* A, const float* s_a, const void* W, const float* s_w,
+                                  const void* bias, int64_t M, int64_t N, int64_t K, void* out,
+                                  cudaStream_t stream, DeviceState* ds);
+
+}  // namespace tfq

@@ -1,0 +1,110 @@
+"""Helpers for the GPU parity tests: calls through the raw C ABI (pointers,
+sizes, stream handle), buffers from torch, expected values from the oracle."""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import oracle
+from int8_w8a8_quantized_b200 import _capi, build
+
+GUARD = 64  # guard bytes/elements after every output buffer
+
+
+def lib():
+    build.build()
+    return _capi.load_library()
+
+
+def stream_handle() -> int:
+    return int(torch.cuda.current_stream().cuda_stream)
+
+
+def check_device_error():
+    st = _capi.raw.tfq_device_error(stream_handle())
+    assert st == _capi.TFQ_OK, (_capi.status_string(st), _capi.last_error_message())
+
+
+def guarded(n: int, dtype, fill) -> torch.Tensor:
+    """A CUDA buffer of n elements followed by GUARD elements set to `fill`."""
+    t = torch.empty(n + GUARD, dtype=dtype, device="cuda")
+    t.fill_(fill)
+    return t
+
+
+def quant_act_fp8(x: torch.Tensor, qmax: float):
+    """GPU per-token FP8 quantization through the C ABI; checks guard bytes."""
+    M, K = x.shape
+    q = guarded(M * K, torch.uint8, 0xA5)
+    s = guarded(M, torch.float32, -7.0)
+    st = _capi.raw.tfq_quant_act_fp8_per_token(x.data_ptr(), M, K, float(qmax), q.data_ptr(), s.data_ptr(),
+                                                stream_handle())
+    assert st == _capi.TFQ_OK, _capi.last_error_message()
+    check_device_error()
+    assert torch.all(q[M * K:] == 0xA5) and torch.all(s[M:] == -7.0), "write past the end of an output"
+    return q[:M * K].view(M, K), s[:M]
+
+
+def quant_weight(w: torch.Tensor, dtype: int, qmax: float):
+    N, K = w.shape
+    q = guarded(N * K, torch.uint8, 0x5A)
+    s = guarded(N, torch.float32, -7.0)
+    st = _capi.raw.tfq_quant_weight_per_channel(w.data_ptr(), N, K, dtype, float(qmax), q.data_ptr(),
+                                                 s.data_ptr(), stream_handle())
+    assert st == _capi.TFQ_OK, _capi.last_error_message()
+    check_device_error()
+    assert torch.all(q[N * K:] == 0x5A) and torch.all(s[N:] == -7.0), "write past the end of an output"
+    return q[:N * K].view(N, K), s[:N]
+
+
+def scaled_linear(A_q, s_a, W_q, s_w, bias):
+    M, K = A_q.shape
+    N = W_q.shape[0]
+    out = guarded(M * N, torch.bfloat16, 12345.0)
+    st = _capi.raw.tfq_scaled_fp8_linear(A_q.data_ptr(), s_a.data_ptr(), W_q.data_ptr(), s_w.data_ptr(),
+                                          None if bias is None else bias.data_ptr(), M, N, K, out.data_ptr(),
+                                          stream_handle())
+    assert st == _capi.TFQ_OK, _capi.last_error_message()
+    check_device_error()
+    assert torch.all(out[M * N:] == 12345.0), "write past the end of the output"
+    return out[:M * N].view(M, N)
+
+
+def bf16_bits_np(t: torch.Tensor) -> np.ndarray:
+    return t.detach().contiguous().cpu().view(torch.int16).numpy().view(np.uint16)
+
+
+def gemm_tolerance_check(y_gpu: torch.Tensor, y_ref: np.ndarray, what: str = ""):
+    """|y - y_ref| <= 2^-7 |y_ref| + 1e-3 rms(y_ref), element by element."""
+    y = y_gpu.float().cpu().numpy().astype(np.float64)
+    assert y.shape == y_ref.shape
+    rms = float(np.sqrt(np.mean(y_ref ** 2))) if y_ref.size else 0.0
+    err = np.abs(y - y_ref)
+    bound = 2.0 ** -7 * np.abs(y_ref) + 1e-3 * rms
+    bad = err > bound
+    assert np.isfinite(y).all(), f"{what}: non-finite output"
+    if bad.any():
+        i = np.argwhere(bad)[0]
+        raise AssertionError(f"{what}: {int(bad.sum())} of {bad.size} outside tolerance; first at {tuple(i)}: "
+                             f"gpu {y[tuple(i)]} ref {y_ref[tuple(i)]} bound {bound[tuple(i)]}")
+    e_max = float(err.max()) if err.size else 0.0
+    e_rel = float(np.linalg.norm(y - y_ref) / max(np.linalg.norm(y_ref), 1e-300))
+    return e_max, e_rel
+
+
+def oracle_quant_fp8(x: torch.Tensor, qmax: float, rows=None):
+    bits = bf16_bits_np(x if rows is None else x[torch.as_tensor(rows, device=x.device)])
+    return oracle.quant_rows_fp8(bits, qmax)
+
+
+def oracle_quant_int8(x: torch.Tensor, qmax: float, rows=None):
+    bits = bf16_bits_np(x if rows is None else x[torch.as_tensor(rows, device=x.device)])
+    return oracle.quant_rows_int8(bits, qmax)
+
+
+def sample_rows(M: int, n: int, seed: int, tail: int = 128) -> np.ndarray:
+    """n seeded random rows plus the last rows of the final (ragged) tile."""
+    rng = np.random.default_rng(seed)
+    pick = rng.choice(M, size=min(n, M), replace=False)
+    last = np.arange(max(0, M - (M % tail or tail)), M)
+    return np.unique(np.concatenate([pick, last, [0]])).astype(np.int64)

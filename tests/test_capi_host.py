@@ -1,0 +1,110 @@
+"""Host-side checks of the C ABI (no GPU needed).
+
+* libtfq.so loads and exports every function include/tfq.h declares, and the
+  binding declares the same set;
+* argument validation rejects bad calls before touching the GPU;
+* on a machine without a GPU a valid call fails loudly (TFQ_ECUDA), it never
+  falls back to anything.
+"""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+import torch
+
+from int8_w8a8_quantized_b200 import _capi, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "tfq.h")
+
+
+def _declared():
+    src = open(HEADER, encoding="utf-8").read()
+    return re.findall(r"TFQ_API\s+[\w\s\*]+?\b(tfq_\w+)\s*\(", src)
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return _capi.load_library()
+
+
+def test_header_declarations_match_binding():
+    names = _declared()
+    assert len(names) == len(set(names)) and names
+    assert set(names) == set(_capi.SIGNATURES)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", _capi.LIB_PATH], capture_output=True, text=True,
+                         check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if line.strip()}
+    for name in _declared():
+        assert name in exported, name
+        assert hasattr(lib, name)
+
+
+def test_status_strings(lib):
+    assert _capi.status_string(0) == "TFQ_OK"
+    assert _capi.status_string(4) == "TFQ_ETIMEOUT"
+    assert _capi.status_string(99) == "unknown"
+    assert lib.tfq_version() == 100
+
+
+ALIGNED = 0x10000  # a fake, 16-byte aligned address: never dereferenced by a rejected call
+
+
+@pytest.mark.parametrize("args,status", [
+    ((ALIGNED, 4, 24, 448.0, ALIGNED, ALIGNED, None), _capi.TFQ_EINVAL),        # K % 16
+    ((ALIGNED, 4, 32, 500.0, ALIGNED, ALIGNED, None), _capi.TFQ_EINVAL),        # qmax > 448
+    ((ALIGNED, 4, 32, 0.5, ALIGNED, ALIGNED, None), _capi.TFQ_EINVAL),          # qmax < 1
+    ((ALIGNED, 4, 32, float("nan"), ALIGNED, ALIGNED, None), _capi.TFQ_EINVAL),
+    ((None, 4, 32, 448.0, ALIGNED, ALIGNED, None), _capi.TFQ_EINVAL),           # null x
+    ((ALIGNED, 4, 32, 448.0, ALIGNED, None, None), _capi.TFQ_EINVAL),           # null s
+    ((ALIGNED + 8, 4, 32, 448.0, ALIGNED, ALIGNED, None), _capi.TFQ_EINVAL),    # misaligned
+    ((ALIGNED, -1, 32, 448.0, ALIGNED, ALIGNED, None), _capi.TFQ_EINVAL),
+    ((ALIGNED, 4, 32768 + 16, 448.0, ALIGNED, ALIGNED, None), _capi.TFQ_EUNSUPPORTED),
+    ((ALIGNED, 0, 32, 448.0, None, None, None), _capi.TFQ_OK),                  # M == 0: no-op
+])
+def test_quant_act_validation(lib, args, status):
+    assert lib.tfq_quant_act_fp8_per_token(*args) == status
+    if status != _capi.TFQ_OK:
+        assert _capi.last_error_message()
+
+
+def test_quant_weight_validation(lib):
+    f = lib.tfq_quant_weight_per_channel
+    assert f(ALIGNED, 4, 32, 7, 448.0, ALIGNED, ALIGNED, None) == _capi.TFQ_EINVAL            # dtype
+    assert f(ALIGNED, 4, 32, _capi.TFQ_DTYPE_INT8, 200.0, ALIGNED, ALIGNED, None) == _capi.TFQ_EINVAL
+    assert f(ALIGNED, 4, 40, _capi.TFQ_DTYPE_FP8_E4M3, 448.0, ALIGNED, ALIGNED, None) == _capi.TFQ_EINVAL
+    assert f(ALIGNED, 0, 32, _capi.TFQ_DTYPE_INT8, 127.0, None, None, None) == _capi.TFQ_OK
+
+
+@pytest.mark.parametrize("M,N,K,status", [
+    (4, 16, 24, _capi.TFQ_EINVAL),     # K % 16
+    (4, 16, 0, _capi.TFQ_EINVAL),      # K == 0
+    (4, 12, 32, _capi.TFQ_EINVAL),     # N % 8
+    (-1, 16, 32, _capi.TFQ_EINVAL),
+    (1 << 31, 16, 32, _capi.TFQ_EUNSUPPORTED),
+    (0, 16, 32, _capi.TFQ_OK),         # empty: no-op
+    (4, 0, 32, _capi.TFQ_OK),
+])
+def test_gemm_validation(lib, M, N, K, status):
+    assert lib.tfq_scaled_fp8_linear(ALIGNED, ALIGNED, ALIGNED, ALIGNED, None, M, N, K, ALIGNED, None) == status
+
+
+def test_gemm_rejects_null_and_misaligned(lib):
+    f = lib.tfq_scaled_fp8_linear
+    assert f(None, ALIGNED, ALIGNED, ALIGNED, None, 4, 16, 32, ALIGNED, None) == _capi.TFQ_EINVAL
+    assert f(ALIGNED, ALIGNED, ALIGNED, ALIGNED, ALIGNED + 2, 4, 16, 32, ALIGNED, None) == _capi.TFQ_EINVAL
+    assert f(ALIGNED, ALIGNED, ALIGNED, ALIGNED, None, 4, 16, 32, ALIGNED + 4, None) == _capi.TFQ_EINVAL
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU behaviour")
+def test_valid_call_without_gpu_fails_loudly(lib):
+    st = lib.tfq_quant_act_fp8_per_token(ALIGNED, 4, 32, 448.0, ALIGNED, ALIGNED, None)
+    assert st in (_capi.TFQ_ECUDA, _capi.TFQ_EUNSUPPORTED)
+    assert lib.tfq_scaled_fp8_linear(ALIGNED, ALIGNED, ALIGNED, ALIGNED, None, 4, 16, 32, ALIGNED, None) \
+        in (_capi.TFQ_ECUDA, _capi.TFQ_EUNSUPPORTED)

@@ -1,0 +1,133 @@
+"""GPU parity of the scaled FP8 GEMM against the oracle, within the stated
+tolerance |y - y_ref| <= 2^-7 |y_ref| + 1e-3 rms(y_ref) element by element:
+full comparisons on small and ragged shapes, sampled rows at the full DiT
+sizes (same launch configuration as the benchmark)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from int8_w8a8_quantized_b200 import _capi, workloads
+from tests import _gpu
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    _gpu.lib()
+
+
+def _rand_codes(gen, shape, max_code=0x6F):
+    """Finite E4M3 codes with magnitudes up to dec(max_code), random signs."""
+    mag = torch.randint(0, max_code + 1, shape, generator=gen, dtype=torch.int32)
+    sign = torch.randint(0, 2, shape, generator=gen, dtype=torch.int32) << 7
+    return (mag | sign).to(torch.uint8)
+
+
+def _run_case(M, N, K, with_bias, seed):
+    g = torch.Generator().manual_seed(seed)
+    A = _rand_codes(g, (M, K))
+    W = _rand_codes(g, (N, K))
+    sa = (torch.rand(M, generator=g) * 0.01 + 1e-4).float()
+    sw = (torch.rand(N, generator=g) * 0.01 + 1e-4).float()
+    bias = (torch.randn(N, generator=g) * 0.5).to(torch.bfloat16) if with_bias else None
+    y = _gpu.scaled_linear(A.cuda(), sa.cuda(), W.cuda(), sw.cuda(), None if bias is None else bias.cuda())
+    y_ref = oracle.scaled_fp8_linear(A.numpy(), sa.numpy(), W.numpy(), sw.numpy(),
+                                     None if bias is None else _gpu.bf16_bits_np(bias))
+    return _gpu.gemm_tolerance_check(y, y_ref, f"M={M} N={N} K={K}")
+
+
+@pytest.mark.parametrize("M,N,K", [(128, 256, 128), (1, 8, 16), (100, 136, 48), (129, 264, 144),
+                                   (300, 520, 1024), (257, 256, 32), (64, 128, 256), (640, 1024, 2048)])
+@pytest.mark.parametrize("with_bias", [True, False])
+def test_ragged_full_compare(M, N, K, with_bias):
+    _run_case(M, N, K, with_bias, seed=M + N + K)
+
+
+def test_many_tiles_persistent():
+    """More tiles than SMs, several tiles per CTA, both accumulator buffers."""
+    _run_case(1100, 2048, 512, True, seed=3)
+
+
+def test_tiny_config_end_to_end():
+    """Tiny W8A8 Linear: X [64,256], W [128,256] N(0,0.02), qmax 448, bias."""
+    wl = workloads.TINY
+    lin = wl.linears[0]
+    x = wl.make_x("x", device="cuda")
+    w = wl.make_w(lin, device="cuda")
+    b = wl.make_bias(lin, device="cuda")
+    A, sa = _gpu.quant_act_fp8(x, 448.0)
+    Wq, sw = _gpu.quant_weight(w, _capi.TFQ_DTYPE_FP8_E4M3, 448.0)
+    A_ref, sa_ref = _gpu.oracle_quant_fp8(x, 448.0)
+    W_ref, sw_ref = _gpu.oracle_quant_fp8(w, 448.0)
+    np.testing.assert_array_equal(A.cpu().numpy(), A_ref)
+    np.testing.assert_array_equal(Wq.cpu().numpy(), W_ref)
+    np.testing.assert_array_equal(sa.cpu().numpy(), sa_ref)
+    np.testing.assert_array_equal(sw.cpu().numpy(), sw_ref)
+    y = _gpu.scaled_linear(A, sa, Wq, sw, b)
+    y_ref = oracle.scaled_fp8_linear(A_ref, sa_ref, W_ref, sw_ref, _gpu.bf16_bits_np(b))
+    _gpu.gemm_tolerance_check(y, y_ref, "tiny")
+
+
+def test_extreme_codes():
+    """Largest codes (+-448) everywhere: sums up to K * 448^2 stay exact-ish in fp32."""
+    M, N, K = 130, 264, 512
+    A = torch.full((M, K), 0x7E, dtype=torch.uint8)
+    A[::2, ::3] = 0xFE
+    W = torch.full((N, K), 0x7E, dtype=torch.uint8)
+    W[1::2, 1::5] = 0x01  # smallest subnormal
+    sa = torch.full((M,), 1e-3)
+    sw = torch.full((N,), 2e-3)
+    y = _gpu.scaled_linear(A.cuda(), sa.cuda(), W.cuda(), sw.cuda(), None)
+    y_ref = oracle.scaled_fp8_linear(A.numpy(), sa.numpy(), W.numpy(), sw.numpy())
+    _gpu.gemm_tolerance_check(y, y_ref, "extreme")
+
+
+def test_zero_activation_gives_bias():
+    M, N, K = 200, 264, 64
+    A = torch.zeros((M, K), dtype=torch.uint8, device="cuda")
+    W = _rand_codes(torch.Generator().manual_seed(1), (N, K)).cuda()
+    b = (torch.randn(N) * 3).to(torch.bfloat16).cuda()
+    y = _gpu.scaled_linear(A, torch.ones(M, device="cuda"), W, torch.ones(N, device="cuda"), b)
+    assert torch.equal(y, b.expand(M, N))
+
+
+@pytest.mark.parametrize("name", ["image_dit_block", "video_dit_block", "reduced_qmax_ffn_out"])
+def test_full_size_linears_sampled(name):
+    """Every Linear of the DiT workloads at full size: GPU quantizer + GPU
+    GEMM; the oracle recomputes a sample of rows (plus the ragged tail)."""
+    wl = workloads.WORKLOADS[name]
+    xs = {}
+    for lin in wl.linears:
+        if lin.x not in xs:
+            xs[lin.x] = wl.make_x(lin.x, device="cuda")
+        x = xs[lin.x]
+        w = wl.make_w(lin, device="cuda")
+        b = wl.make_bias(lin, device="cuda")
+        Wq, sw = _gpu.quant_weight(w, _capi.TFQ_DTYPE_FP8_E4M3, 448.0)
+        rows = _gpu.sample_rows(wl.M, 96, seed=lin.N + lin.K)
+        for qmax in wl.act_qmax:
+            A, sa = _gpu.quant_act_fp8(x, qmax)
+            y = _gpu.scaled_linear(A, sa, Wq, sw, b)
+            ridx = torch.as_tensor(rows, device="cuda")
+            y_ref = oracle.scaled_fp8_linear(A.cpu().numpy(), sa.cpu().numpy(), Wq.cpu().numpy(),
+                                             sw.cpu().numpy(), None if b is None else _gpu.bf16_bits_np(b),
+                                             rows=rows)
+            _gpu.gemm_tolerance_check(y[ridx], y_ref, f"{name}/{lin.name}/q{qmax:g}")
+            del A, sa, y
+        del w, Wq
+    del xs
+    torch.cuda.empty_cache()
+
+
+def test_tensor_wrapper_linear():
+    from int8_w8a8_quantized_b200 import tfq_quant_weight_per_channel, w8a8_linear
+    x = workloads.activations(300, 512, seed=9, device="cuda")
+    w = workloads.weights(264, 512, seed=10, std=0.02, device="cuda")
+    b = workloads.bias(264, seed=11, device="cuda")
+    Wq, sw = tfq_quant_weight_per_channel(w, "fp8")
+    y = w8a8_linear(x, Wq, sw, b, qmax=448.0)
+    A_ref, sa_ref = _gpu.oracle_quant_fp8(x, 448.0)
+    y_ref = oracle.scaled_fp8_linear(A_ref, sa_ref, Wq.cpu().numpy(), sw.cpu().numpy(), _gpu.bf16_bits_np(b))
+    _gpu.gemm_tolerance_check(y, y_ref, "wrapper")

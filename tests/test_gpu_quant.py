@@ -1,0 +1,129 @@
+"""GPU parity of the row quantizers against the oracle: codes and scales
+bit-exact, on the workloads' shapes and distributions, ragged sizes and the
+degenerate cases (zero rows, K = 0, M = 0, tiny magnitudes, rounding ties)."""
+import numpy as np
+import pytest
+import torch
+
+from int8_w8a8_quantized_b200 import _capi, workloads
+from tests import _gpu
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    _gpu.lib()
+
+
+def _assert_fp8_equal(x, qmax, rows=None):
+    q, s = _gpu.quant_act_fp8(x, qmax)
+    q_ref, s_ref = _gpu.oracle_quant_fp8(x, qmax, rows)
+    qg = q.cpu().numpy() if rows is None else q[torch.as_tensor(rows, device="cuda")].cpu().numpy()
+    sg = s.cpu().numpy() if rows is None else s[torch.as_tensor(rows, device="cuda")].cpu().numpy()
+    np.testing.assert_array_equal(sg.view(np.uint32), s_ref.view(np.uint32))
+    mism = np.argwhere(qg != q_ref)
+    assert mism.size == 0, f"{len(mism)} code mismatches, first {tuple(mism[0])}: gpu {qg[tuple(mism[0])]:#x} " \
+                           f"oracle {q_ref[tuple(mism[0])]:#x}"
+
+
+def test_tiny_config_activation():
+    x = workloads.TINY.make_x("x", device="cuda")
+    _assert_fp8_equal(x, 448.0)
+
+
+@pytest.mark.parametrize("qmax", [448.0, 14.0, 7.0])
+@pytest.mark.parametrize("M,K", [(1, 16), (3, 48), (37, 256), (129, 1024), (65, 3072), (33, 5120),
+                                 (17, 12288), (9, 13824), (5, 32768), (300, 160)])
+def test_ragged_shapes(M, K, qmax):
+    x = workloads.activations(M, K, seed=M * 7 + K, nu=3, amplitude=4.0, outlier_cols=max(1, K // 100),
+                              outlier_mult=30.0, zero_rows=1 if M > 2 else 0, device="cuda")
+    _assert_fp8_equal(x, qmax)
+
+
+def test_quantizer_config_fp8_and_int8():
+    """Activation-quantizer workload: [8192, 3072], 1 % outlier columns x50,
+    16 all-zero rows; per-token FP8 (448) and per-row INT8 (127)."""
+    x = workloads.quantizer_input(device="cuda")
+    _assert_fp8_equal(x, 448.0)
+    q, s = _gpu.quant_weight(x, _capi.TFQ_DTYPE_INT8, 127.0)
+    q_ref, s_ref = _gpu.oracle_quant_int8(x, 127.0)
+    np.testing.assert_array_equal(s.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
+    np.testing.assert_array_equal(q.cpu().numpy().view(np.int8), q_ref)
+    zero = (x == 0).all(dim=1)
+    assert int(zero.sum()) == 16
+    assert torch.all(s[zero] == torch.tensor(np.float32(1e-12) / np.float32(127.0), device="cuda"))
+
+
+@pytest.mark.parametrize("qmax", [448.0, 14.0, 7.0])
+def test_weight_fp8_per_channel(qmax):
+    w = workloads.weights(520, 1024, seed=11, std=0.02, device="cuda")
+    q, s = _gpu.quant_weight(w, _capi.TFQ_DTYPE_FP8_E4M3, qmax)
+    q_ref, s_ref = _gpu.oracle_quant_fp8(w, qmax)
+    np.testing.assert_array_equal(s.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
+    np.testing.assert_array_equal(q.cpu().numpy(), q_ref)
+
+
+@pytest.mark.parametrize("K", [16, 256, 5120, 13824])
+def test_int8_ragged(K):
+    x = workloads.activations(77, K, seed=K, nu=4, outlier_cols=3, outlier_mult=20.0, zero_rows=2, device="cuda")
+    q, s = _gpu.quant_weight(x, _capi.TFQ_DTYPE_INT8, 127.0)
+    q_ref, s_ref = _gpu.oracle_quant_int8(x, 127.0)
+    np.testing.assert_array_equal(s.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
+    np.testing.assert_array_equal(q.cpu().numpy().view(np.int8), q_ref)
+
+
+def test_rounding_edges():
+    """Rows built so that x/s hits E4M3 midpoints, subnormals, signed zeros,
+    saturation and tiny magnitudes below the 1e-12 floor."""
+    grid = torch.tensor(np.r_[0:0x7F].astype(np.uint8)).view(torch.float8_e4m3fn).float()
+    mids = (grid[:-1] + grid[1:]) / 2
+    row = torch.cat([torch.tensor([448.0]), grid, -grid, mids, -mids, torch.tensor([-0.0, 0.0, 1e-30, -1e-30])])
+    K = ((row.numel() + 15) // 16) * 16
+    x = torch.zeros(6, K)
+    x[0, :row.numel()] = row                       # s = 1: t = x exactly
+    x[1, :row.numel()] = row * 2.0 ** -20          # scaled copy (still exact in bf16 where representable)
+    x[2, :row.numel()] = row / 448.0 * 14.0
+    x[3] = -0.0                                    # all negative zeros
+    x[4, :8] = torch.tensor([1e-13, -3e-13, 2e-13, 0, 0, 0, 0, -1e-14])   # below the floor
+    x[5, :row.numel()] = row * 3.0                 # a non-power-of-two scale
+    x = x.to(torch.bfloat16).cuda()
+    for qmax in (448.0, 14.0, 7.0):
+        _assert_fp8_equal(x, qmax)
+
+
+def test_empty_and_k0():
+    x = torch.empty((0, 64), dtype=torch.bfloat16, device="cuda")
+    st = _capi.raw.tfq_quant_act_fp8_per_token(x.data_ptr(), 0, 64, 448.0, 0, 0, _gpu.stream_handle())
+    assert st == _capi.TFQ_OK
+    s = torch.full((5,), -1.0, device="cuda")
+    x0 = torch.empty((5, 0), dtype=torch.bfloat16, device="cuda")
+    q0 = torch.empty((5, 0), dtype=torch.uint8, device="cuda")
+    st = _capi.raw.tfq_quant_act_fp8_per_token(x0.data_ptr() or 16, 5, 0, 7.0, q0.data_ptr() or 16, s.data_ptr(),
+                                                _gpu.stream_handle())
+    assert st == _capi.TFQ_OK
+    _gpu.check_device_error()
+    assert torch.all(s == torch.tensor(np.float32(1e-12) / np.float32(7.0), device="cuda"))
+
+
+@pytest.mark.parametrize("name", ["image_dit_block", "video_dit_block", "reduced_qmax_ffn_out"])
+def test_full_size_activations_sampled(name):
+    """Full-size DiT activations, bench launch configuration; the oracle
+    checks a seeded sample of rows plus the ragged tail."""
+    wl = workloads.WORKLOADS[name]
+    for xname in sorted(wl.x_shapes()):
+        x = wl.make_x(xname, device="cuda")
+        rows = _gpu.sample_rows(wl.M, 384, seed=len(xname))
+        for qmax in wl.act_qmax:
+            _assert_fp8_equal(x, qmax, rows)
+        del x
+        torch.cuda.empty_cache()
+
+
+def test_tensor_wrappers_match_raw():
+    x = workloads.activations(100, 512, seed=5, device="cuda")
+    q1, s1 = _gpu.quant_act_fp8(x, 14.0)
+    from int8_w8a8_quantized_b200 import tfq_quant_act_fp8_per_token
+    q2, s2 = tfq_quant_act_fp8_per_token(x, 14.0)
+    torch.cuda.synchronize()
+    assert torch.equal(q1, q2) and torch.equal(s1, s2)
