@@ -121,6 +121,43 @@ TFQ_API tfq_status tfq_scaled_fp8_linear(const void *A_q, const float *s_a, cons
                                  int64_t K, void *out_bf16, void *stream);
 
 /*
+ * Bytes of the static device array used by tfq_scaled_fp8_linear_noalloc.
+ * Every GPU that loads the library holds this array until the process exits.
+ */
+#define TFQ_NOALLOC_SCRATCH_BYTES 256
+
+/*
+ * tfq_scaled_fp8_linear without any device allocation.  (An addition of this
+ * library for callers that cannot allocate; the pages have no counterpart.)
+ *
+ * Same arguments, preconditions, result and errors as tfq_scaled_fp8_linear.
+ * The regular entry points cudaMalloc one device word per device on their
+ * first call (where a kernel records a bounded wait that ran out).  Callers
+ * that must not allocate device memory -- a framework that owns all device
+ * memory through its own pool, a process that has reserved nearly all of
+ * HBM, code running where a possibly synchronizing CUDA call is not allowed
+ * -- call this one instead: that word lives in a file-scope __device__ array
+ * of TFQ_NOALLOC_SCRATCH_BYTES bytes, and no call allocates (no cudaMalloc,
+ * cudaFree or allocating library routine).
+ *  - The caller still owns and passes every input and output.
+ *  - A call needs 4 bytes of the array whatever M, N and K; a call needing
+ *    more than the array holds is rejected with TFQ_EUNSUPPORTED.
+ *  - The first call on a device does a one-time set-up with that device
+ *    current (device checks, cudaGetSymbolAddress of the array, which may
+ *    load the library's device code into the context); make that first call
+ *    before any stream capture.
+ *  - Every call on a device shares the array, which keeps the last call's
+ *    contents; each call clears the word on `stream` before its kernel.
+ *    Calls that overlap on the GPU (on different streams) race on the word.
+ *  - A bounded wait that runs out is recorded in the array's word only:
+ *    this entry point does not read it back (that would need a host
+ *    synchronization), and tfq_device_error() does not see it.
+ */
+TFQ_API tfq_status tfq_scaled_fp8_linear_noalloc(const void *A_q, const float *s_a, const void *W_q,
+                                                 const float *s_w, const void *bias_bf16, int64_t M,
+                                                 int64_t N, int64_t K, void *out_bf16, void *stream);
+
+/*
  * Synchronizes `stream`, then reads and clears the current device's error
  * word.  Returns TFQ_ETIMEOUT if a bounded wait inside a kernel ran out
  * since the last call (the outputs of that launch are then incomplete),

@@ -19,9 +19,14 @@ DeviceState g_states[kMaxDevices];
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 thread_local char g_last_error[512] = "";
 
+std::mutex g_encode_mutex;
+
+}  // namespace
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 tfq_status resolve_encode() {
+    std::lock_guard<std::mutex> lock(g_encode_mutex);
     if (g_encode != nullptr) return TFQ_OK;
     void* fn = nullptr;
     cudaDriverEntryPointQueryResult q;
@@ -32,8 +37,6 @@ tfq_status resolve_encode() {
     g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
     return TFQ_OK;
 }
-
-}  // namespace
 
 tfq_status fail(tfq_status st, const char* fmt, ...) {
     va_list ap;

@@ -34,6 +34,12 @@ struct DeviceState {
 // nullptr and sets *st on failure.
 DeviceState* current_device_state(tfq_status* st);
 
+// Resolves cuTensorMapEncodeTiled through the runtime (once; thread safe).
+tfq_status resolve_encode();
+
+// True when p is 16-byte aligned.
+bool aligned16(const void* p);
+
 // Records a message for tfq_last_error_message() and returns `st`.
 tfq_status fail(tfq_status st, const char* fmt, ...);
 
