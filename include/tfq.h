@@ -158,6 +158,22 @@ TFQ_API tfq_status tfq_scaled_fp8_linear_noalloc(const void *A_q, const float *s
                                                  int64_t N, int64_t K, void *out_bf16, void *stream);
 
 /*
+ * Self-check of the division the quantizers use (a branch-free correctly
+ * rounded fp32 division from the row's reciprocal, Markstein's method; the
+ * pages fix x / s, see the conventions above).  For i < n writes
+ *   ours[i] = the quantizers' quotient a[i] / b[i],
+ *   ieee[i] = the CUDA IEEE round-to-nearest quotient __fdiv_rn(a[i], b[i]);
+ * the two agree bit for bit when |a| >= 2^-102 and 2^-49 <= b <= 2^125
+ * (every row scale the quantizers use this division for); for smaller |a|
+ * both quotients are below 2^-53 in magnitude with the sign of a, so they
+ * give the same E4M3 and INT8 codes.  All pointers are device
+ * pointers of n floats, 4-byte aligned.  Errors: TFQ_EINVAL (n < 0, null
+ * pointer with n > 0).
+ */
+TFQ_API tfq_status tfq_selftest_div_rn(const float *a, const float *b, int64_t n, float *ours, float *ieee,
+                                       void *stream);
+
+/*
  * Synchronizes `stream`, then reads and clears the current device's error
  * word.  Returns TFQ_ETIMEOUT if a bounded wait inside a kernel ran out
  * since the last call (the outputs of that launch are then incomplete),

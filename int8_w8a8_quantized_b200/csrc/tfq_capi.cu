@@ -174,6 +174,17 @@ tfq_status tfq_scaled_fp8_linear(const void* A_q, const float* s_a, const void* 
                                   static_cast<cudaStream_t>(stream), ds);
 }
 
+tfq_status tfq_selftest_div_rn(const float* a, const float* b, int64_t n, float* ours, float* ieee,
+                               void* stream) {
+    if (n < 0) return fail(TFQ_EINVAL, "negative n");
+    if (n == 0) return TFQ_OK;
+    if (a == nullptr || b == nullptr || ours == nullptr || ieee == nullptr) return fail(TFQ_EINVAL, "null pointer");
+    tfq_status st;
+    DeviceState* ds = current_device_state(&st);
+    if (ds == nullptr) return st;
+    return launch_div_selftest(a, b, n, ours, ieee, static_cast<cudaStream_t>(stream));
+}
+
 tfq_status tfq_device_error(void* stream) {
     tfq_status st;
     DeviceState* ds = current_device_state(&st);

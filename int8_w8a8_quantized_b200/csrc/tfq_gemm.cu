@@ -94,6 +94,78 @@ __device__ __forceinline__ void give_up(volatile int* abort_flag, uint32_t* err,
     atomicOr(err, bit);
 }
 
+// Epilogue of one 32-row slice of a finished tile: TMEM -> registers ->
+// y = acc * s_a[m] * s_w[n] + bias[n] in fp32 -> bf16 -> 128-byte swizzled
+// staging buffer -> TMA store, EPI_COLS columns at a time.  `t_row` is the
+// TMEM address of this warp's 32 lanes at the tile's first column; `chunk`
+// counts stores of this warp (selects the staging buffer).
+template <int kBN>
+__device__ __forceinline__ void store_tile_rows(const GemmArgs& p, const CUtensorMap& tmY, uint32_t t_row,
+                                                uint8_t* ebuf0, int& chunk, int n_tile0, int row0, float sa,
+                                                int lane) {
+#pragma unroll 1
+    for (int c = 0; c < kBN / EPI_COLS; ++c) {
+        const int n0 = n_tile0 + c * EPI_COLS;
+        if (n0 >= p.N) break;  // uniform across the warp
+        uint32_t acc[2][32];
+        tmem_ld_32x32b_x32(t_row + c * EPI_COLS, acc[0]);
+        tmem_ld_32x32b_x32(t_row + c * EPI_COLS + 32, acc[1]);
+        tmem_ld_wait();
+        uint8_t* ebuf = ebuf0 + (chunk & 1) * EPI_BUF_BYTES;
+        // The staging buffer written two chunks ago must have been read by its TMA store.
+        if (lane == 0) bulk_wait_read<1>();
+        __syncwarp();
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+#pragma unroll
+            for (int g = 0; g < 4; ++g) {  // 8 columns -> one 16-byte unit
+                const int nl = h * 32 + g * 8;
+                float sw[8], bb[8];
+                if (n0 + nl < p.N) {  // N % 8 == 0: a group is all valid or all out
+                    const float4 w0 = __ldg(reinterpret_cast<const float4*>(p.s_w + n0 + nl));
+                    const float4 w1 = __ldg(reinterpret_cast<const float4*>(p.s_w + n0 + nl + 4));
+                    sw[0] = w0.x; sw[1] = w0.y; sw[2] = w0.z; sw[3] = w0.w;
+                    sw[4] = w1.x; sw[5] = w1.y; sw[6] = w1.z; sw[7] = w1.w;
+                    if (p.bias != nullptr) {
+                        const uint4 bv = __ldg(reinterpret_cast<const uint4*>(p.bias + n0 + nl));
+                        const uint32_t bw[4] = {bv.x, bv.y, bv.z, bv.w};
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            bb[2 * j] = __uint_as_float(bw[j] << 16);
+                            bb[2 * j + 1] = __uint_as_float(bw[j] & 0xFFFF0000u);
+                        }
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) bb[j] = 0.0f;
+                    }
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) sw[j] = bb[j] = 0.0f;
+                }
+                uint32_t packed[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const float y0 = fmaf(__uint_as_float(acc[h][g * 8 + 2 * j]) * sa, sw[2 * j], bb[2 * j]);
+                    const float y1 =
+                        fmaf(__uint_as_float(acc[h][g * 8 + 2 * j + 1]) * sa, sw[2 * j + 1], bb[2 * j + 1]);
+                    packed[j] = pack_bf16x2(y0, y1);
+                }
+                // 128-byte swizzle: 16-byte unit u of row r lives at unit u ^ (r % 8).
+                const int unit = h * 4 + g;
+                uint4* dst = reinterpret_cast<uint4*>(ebuf + lane * 128 + ((unit ^ (lane & 7)) << 4));
+                *dst = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+            }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+            tma_store_2d(&tmY, ebuf, n0, row0);
+            bulk_commit();
+        }
+        ++chunk;
+    }
+}
+
 __global__ void __launch_bounds__(THREADS, 1)
     scaled_fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                            const __grid_constant__ CUtensorMap tmY, GemmArgs p) {
@@ -228,67 +300,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             const float sa = (m < p.M) ? __ldg(p.s_a + m) : 0.0f;
             const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
                                    static_cast<uint32_t>(buf * BN);
-#pragma unroll 1
-            for (int c = 0; c < BN / EPI_COLS; ++c) {
-                const int n0 = tn * BN + c * EPI_COLS;
-                if (n0 >= p.N) break;  // uniform across the warp
-                uint32_t acc[2][32];
-                tmem_ld_32x32b_x32(t_row + c * EPI_COLS, acc[0]);
-                tmem_ld_32x32b_x32(t_row + c * EPI_COLS + 32, acc[1]);
-                tmem_ld_wait();
-                uint8_t* ebuf = ebuf0 + (chunk & 1) * EPI_BUF_BYTES;
-                // The staging buffer written two chunks ago must have been read by its TMA store.
-                if (lane == 0) bulk_wait_read<1>();
-                __syncwarp();
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
-#pragma unroll
-                    for (int g = 0; g < 4; ++g) {  // 8 columns -> one 16-byte unit
-                        const int nl = h * 32 + g * 8;
-                        float sw[8], bb[8];
-                        if (n0 + nl < p.N) {  // N % 8 == 0: a group is all valid or all out
-                            const float4 w0 = __ldg(reinterpret_cast<const float4*>(p.s_w + n0 + nl));
-                            const float4 w1 = __ldg(reinterpret_cast<const float4*>(p.s_w + n0 + nl + 4));
-                            sw[0] = w0.x; sw[1] = w0.y; sw[2] = w0.z; sw[3] = w0.w;
-                            sw[4] = w1.x; sw[5] = w1.y; sw[6] = w1.z; sw[7] = w1.w;
-                            if (p.bias != nullptr) {
-                                const uint4 bv = __ldg(reinterpret_cast<const uint4*>(p.bias + n0 + nl));
-                                const uint32_t bw[4] = {bv.x, bv.y, bv.z, bv.w};
-#pragma unroll
-                                for (int j = 0; j < 4; ++j) {
-                                    bb[2 * j] = __uint_as_float(bw[j] << 16);
-                                    bb[2 * j + 1] = __uint_as_float(bw[j] & 0xFFFF0000u);
-                                }
-                            } else {
-#pragma unroll
-                                for (int j = 0; j < 8; ++j) bb[j] = 0.0f;
-                            }
-                        } else {
-#pragma unroll
-                            for (int j = 0; j < 8; ++j) sw[j] = bb[j] = 0.0f;
-                        }
-                        uint32_t packed[4];
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            const float y0 = fmaf(__uint_as_float(acc[h][g * 8 + 2 * j]) * sa, sw[2 * j], bb[2 * j]);
-                            const float y1 =
-                                fmaf(__uint_as_float(acc[h][g * 8 + 2 * j + 1]) * sa, sw[2 * j + 1], bb[2 * j + 1]);
-                            packed[j] = pack_bf16x2(y0, y1);
-                        }
-                        // 128-byte swizzle: 16-byte unit u of row r lives at unit u ^ (r % 8).
-                        const int unit = h * 4 + g;
-                        uint4* dst = reinterpret_cast<uint4*>(ebuf + lane * 128 + ((unit ^ (lane & 7)) << 4));
-                        *dst = make_uint4(packed[0], packed[1], packed[2], packed[3]);
-                    }
-                }
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) {
-                    tma_store_2d(&tmY, ebuf, n0, row0);
-                    bulk_commit();
-                }
-                ++chunk;
-            }
+            store_tile_rows<BN>(p, tmY, t_row, ebuf0, chunk, tn * BN, row0, sa, lane);
             // All of this warp's TMEM reads of `buf` are complete: hand it back.
             tc_fence_before();
             __syncwarp();
@@ -307,6 +319,221 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
 }
 
+// ---------------------------------------------------------------------------
+// CTA-pair kernel (cta_group::2): a cluster of two CTAs on two SMs computes a
+// 256 x PBN tile.  CTA r of the pair loads rows [128 r, 128 r + 128) of the
+// tile's A panel and rows [PBN/2 r, PBN/2 (r + 1)) of its B panel into its
+// own shared memory; the even CTA's single MMA thread issues
+// tcgen05.mma.cta_group::2 (M = 256, N = PBN, K = 32), which reads both
+// CTAs' halves and leaves rows [128 r, 128 r + 128) of the accumulator in
+// CTA r's TMEM.  Per CTA a stage is 16 KiB of A + PBN/2 x 128 B of B (32 KiB
+// at PBN = 256 instead of 48 KiB), so six stages fit and each SM pulls a
+// third less data from L2 per FLOP.  Both CTAs' loads complete on the even
+// CTA's "full" barrier (which expects the bytes of both); the MMA thread
+// releases each stage and each accumulator to both CTAs with a multicast
+// commit; both CTAs' epilogue warps hand the accumulator back on the even
+// CTA's "tmem_empty" barrier.  The epilogue is the same as above.
+constexpr int PAIR_STAGES = 6;
+constexpr int PAIR_GROUP_M = 8;  // pair tiles per M group (2048 rows)
+
+template <int PBN>
+struct PairCfg {
+    static constexpr int kBHalf = PBN / 2;                      // B rows per CTA
+    static constexpr int kAStage = 128 * BK;                    // 16 KiB
+    static constexpr int kBStage = kBHalf * BK;
+    static constexpr int kTmemCols = 512;                       // two PBN-column accumulators, power of 2
+    static constexpr size_t kRing = static_cast<size_t>(PAIR_STAGES) * (kAStage + kBStage);
+    static constexpr size_t kSmem = 1024 + kRing + SMEM_EPI + (2 * PAIR_STAGES + 4 + 1) * 8 + 16;
+    static constexpr uint32_t kIdesc =
+        (1u << 4) | (static_cast<uint32_t>(PBN >> 3) << 17) | (static_cast<uint32_t>(256 >> 4) << 24);
+    static_assert(kSmem <= 232448, "shared memory budget exceeded");
+    static_assert(2 * PBN <= kTmemCols, "two accumulators must fit in TMEM");
+    static_assert(PBN % 64 == 0 && PBN >= 64 && PBN <= 256, "N tile");
+};
+
+__device__ __forceinline__ void pair_tile_coords(int t, int m_tiles, int n_tiles, int& tm, int& tn) {
+    const int per_group = PAIR_GROUP_M * n_tiles;
+    const int gid = t / per_group;
+    const int first_m = gid * PAIR_GROUP_M;
+    const int gsize = min(m_tiles - first_m, PAIR_GROUP_M);
+    const int r = t - gid * per_group;
+    tm = first_m + r % gsize;
+    tn = r / gsize;
+}
+
+template <int PBN>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
+    scaled_fp8_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                                const __grid_constant__ CUtensorMap tmY, GemmArgs p) {
+    using C = PairCfg<PBN>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* sA = smem;
+    uint8_t* sB = sA + PAIR_STAGES * C::kAStage;
+    uint8_t* sE = sB + PAIR_STAGES * C::kBStage;
+    uint64_t* full = reinterpret_cast<uint64_t*>(sE + SMEM_EPI);
+    uint64_t* empty = full + PAIR_STAGES;
+    uint64_t* tmem_full = empty + PAIR_STAGES;
+    uint64_t* tmem_empty = tmem_full + 2;
+    uint64_t* drain = tmem_empty + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();
+    const int cluster = blockIdx.x >> 1;
+    const int n_clusters = gridDim.x >> 1;
+    const int m_tiles = (p.M + 255) / 256;
+    const int total_tiles = m_tiles * p.n_tiles;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < PAIR_STAGES; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&tmem_full[i], 1);
+            mbar_init(&tmem_empty[i], 2 * EPI_WARPS);
+        }
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+        prefetch_tensormap(&tmA);
+        prefetch_tensormap(&tmB);
+        prefetch_tensormap(&tmY);
+    }
+    if (warp == 1) {
+        tmem_alloc_pair(tmem_slot, C::kTmemCols);
+        tmem_relinquish_pair();
+    }
+    tc_fence_before();
+    cluster_sync_all();  // barriers of both CTAs initialised, TMEM allocated
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == 0) {
+        // ---------------------------------------------------- TMA producer
+        if (lane == 0) {
+            int it = 0;
+            int issued_phase[PAIR_STAGES];
+            for (int i = 0; i < PAIR_STAGES; ++i) issued_phase[i] = -1;
+            bool ok = true;
+            for (int t = cluster; t < total_tiles && ok; t += n_clusters) {
+                int tm, tn;
+                pair_tile_coords(t, m_tiles, p.n_tiles, tm, tn);
+                const int a_row = tm * 256 + static_cast<int>(rank) * 128;
+                const int b_row = tn * PBN + static_cast<int>(rank) * C::kBHalf;
+                for (int kb = 0; kb < p.k_blocks; ++kb, ++it) {
+                    const int st = it % PAIR_STAGES;
+                    const uint32_t ph = static_cast<uint32_t>(it / PAIR_STAGES) & 1u;
+                    if (!mbar_wait(&empty[st], ph ^ 1u, abort_flag)) {
+                        give_up(abort_flag, p.err, kErrGemmProducer);
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t full_leader = mapa_shared(smem_u32(&full[st]), 0);
+                    if (rank == 0) mbar_arrive_expect_tx(&full[st], 2 * (C::kAStage + C::kBStage));
+                    tma_load_2d_pair(sA + st * C::kAStage, &tmA, kb * BK, a_row, full_leader);
+                    tma_load_2d_pair(sB + st * C::kBStage, &tmB, kb * BK, b_row, full_leader);
+                    issued_phase[st] = static_cast<int>(ph);
+                }
+            }
+            // The even CTA's "full" barriers count both CTAs' loads: the even
+            // producer waits for everything in flight before the final
+            // cluster barrier lets either CTA exit.
+            if (rank == 0) {
+                for (int i = 0; i < PAIR_STAGES; ++i)
+                    if (issued_phase[i] >= 0 &&
+                        !mbar_wait(&full[i], static_cast<uint32_t>(issued_phase[i]), nullptr))
+                        atomicOr(p.err, kErrGemmDrain);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------- MMA issuer (even CTA)
+        if (lane == 0 && rank == 0) {
+            int it = 0, tcount = 0;
+            bool ok = true;
+            for (int t = cluster; t < total_tiles && ok; t += n_clusters, ++tcount) {
+                const int buf = tcount & 1;
+                const uint32_t use = static_cast<uint32_t>(tcount >> 1);
+                if (!mbar_wait(&tmem_empty[buf], (use & 1u) ^ 1u, abort_flag)) {
+                    give_up(abort_flag, p.err, kErrGemmMma);
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * PBN);
+                for (int kb = 0; kb < p.k_blocks; ++kb, ++it) {
+                    const int st = it % PAIR_STAGES;
+                    const uint32_t ph = static_cast<uint32_t>(it / PAIR_STAGES) & 1u;
+                    if (!mbar_wait(&full[st], ph, abort_flag)) {
+                        give_up(abort_flag, p.err, kErrGemmMma);
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint64_t a_desc = sw128_kmajor_desc(sA + st * C::kAStage);
+                    const uint64_t b_desc = sw128_kmajor_desc(sB + st * C::kBStage);
+#pragma unroll
+                    for (int k = 0; k < BK / UMMA_K; ++k) {
+                        const uint64_t koff = static_cast<uint64_t>((k * UMMA_K) >> 4);
+                        mma_e4m3_pair(d_tmem, a_desc + koff, b_desc + koff, C::kIdesc, (kb | k) != 0 ? 1u : 0u);
+                    }
+                    mma_commit_pair(&empty[st], 0x3);
+                }
+                if (ok) mma_commit_pair(&tmem_full[buf], 0x3);
+            }
+            mma_commit_pair(drain, 0x1);
+            if (!mbar_wait(drain, 0, nullptr)) atomicOr(p.err, kErrGemmDrain);
+        }
+    } else {
+        // ------------------------------------------- epilogue (both CTAs)
+        const int ew = warp - 2;
+        const int quarter = warp & 3;
+        uint8_t* ebuf0 = sE + static_cast<size_t>(ew) * 2 * EPI_BUF_BYTES;
+        const uint32_t tmem_empty_leader0 = mapa_shared(smem_u32(&tmem_empty[0]), 0);
+        const uint32_t tmem_empty_leader1 = mapa_shared(smem_u32(&tmem_empty[1]), 0);
+        int tcount = 0, chunk = 0;
+        for (int t = cluster; t < total_tiles; t += n_clusters, ++tcount) {
+            int tm, tn;
+            pair_tile_coords(t, m_tiles, p.n_tiles, tm, tn);
+            const int buf = tcount & 1;
+            const uint32_t use = static_cast<uint32_t>(tcount >> 1);
+            if (!mbar_wait_warp(&tmem_full[buf], use & 1u, abort_flag)) {
+                if (lane == 0) give_up(abort_flag, p.err, kErrGemmEpilogue);
+                break;
+            }
+            tc_fence_after();
+            const int row0 = tm * 256 + static_cast<int>(rank) * 128 + quarter * 32;
+            const int m = row0 + lane;
+            const float sa = (m < p.M) ? __ldg(p.s_a + m) : 0.0f;
+            const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
+                                   static_cast<uint32_t>(buf * PBN);
+            store_tile_rows<PBN>(p, tmY, t_row, ebuf0, chunk, tn * PBN, row0, sa, lane);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(buf == 0 ? tmem_empty_leader0 : tmem_empty_leader1);
+        }
+        if (lane == 0) bulk_wait<0>();
+        __syncwarp();
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync_all();  // neither CTA leaves while the pair may still touch its shared memory
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc_pair(tmem_base, C::kTmemCols);
+    }
+}
+
+#ifndef TFQ_GEMM_PAIR_MIN_M
+#define TFQ_GEMM_PAIR_MIN_M 512  // below this many rows the 1-CTA 128 x 256 tiles are used
+#endif
+
+bool use_pair_kernel(int64_t M, int sm_count) { return M >= TFQ_GEMM_PAIR_MIN_M && sm_count >= 2; }
+
 }  // namespace
 
 tfq_status launch_scaled_fp8_gemm(const void* A, const float* s_a, const void* W, const float* s_w,
@@ -323,9 +550,11 @@ tfq_status launch_scaled_fp8_gemm(const void* A, const float* s_a, const void* W
                               CU_TENSOR_MAP_SWIZZLE_128B);
     if (st != TFQ_OK) return st;
     if (!ds->gemm_attr_set) {
-        const cudaError_t e = cudaFuncSetAttribute(scaled_fp8_gemm_kernel,
-                                                   cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                   static_cast<int>(SMEM_BYTES));
+        cudaError_t e = cudaFuncSetAttribute(scaled_fp8_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(SMEM_BYTES));
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(scaled_fp8_gemm_pair_kernel<256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     static_cast<int>(PairCfg<256>::kSmem));
         if (e != cudaSuccess) return fail(TFQ_ECUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
         ds->gemm_attr_set = true;
     }
@@ -342,8 +571,19 @@ tfq_status launch_scaled_fp8_gemm(const void* A, const float* s_a, const void* W
     a.err = ds->err_word;
     const int64_t tiles = static_cast<int64_t>(a.m_tiles) * a.n_tiles;
     if (tiles > INT32_MAX) return fail(TFQ_EUNSUPPORTED, "too many output tiles");
-    const int grid = static_cast<int>(std::min<int64_t>(tiles, ds->sm_count));
-    scaled_fp8_gemm_kernel<<<grid, THREADS, SMEM_BYTES, stream>>>(tmA, tmB, tmY, a);
+    if (use_pair_kernel(M, ds->sm_count)) {
+        CUtensorMap tmBh;
+        st = encode_tensor_map_2d(&tmBh, CU_TENSOR_MAP_DATA_TYPE_UINT8, W, K, N, K, BK, PairCfg<256>::kBHalf,
+                                  CU_TENSOR_MAP_SWIZZLE_128B);
+        if (st != TFQ_OK) return st;
+        const int64_t pair_tiles = ((M + 255) / 256) * static_cast<int64_t>(a.n_tiles);
+        const int clusters = static_cast<int>(std::min<int64_t>(pair_tiles, ds->sm_count / 2));
+        scaled_fp8_gemm_pair_kernel<256>
+            <<<2 * clusters, THREADS, PairCfg<256>::kSmem, stream>>>(tmA, tmBh, tmY, a);
+    } else {
+        const int grid = static_cast<int>(std::min<int64_t>(tiles, ds->sm_count));
+        scaled_fp8_gemm_kernel<<<grid, THREADS, SMEM_BYTES, stream>>>(tmA, tmB, tmY, a);
+    }
     const cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? TFQ_OK : fail(TFQ_ECUDA, "GEMM launch: %s", cudaGetErrorString(e));
 }

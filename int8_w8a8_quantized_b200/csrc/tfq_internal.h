@@ -26,7 +26,7 @@ struct DeviceState {
     int cc_major = 0, cc_minor = 0;
     size_t smem_optin = 0;          // max dynamic shared memory per block
     uint32_t* err_word = nullptr;   // device memory, one 32-bit word
-    bool quant_attr_set[2] = {false, false};
+    bool quant_attr_set[3] = {false, false, false};
     bool gemm_attr_set = false;
 };
 
@@ -51,6 +51,10 @@ tfq_status encode_tensor_map_2d(CUtensorMap* map, CUtensorMapDataType dtype, con
 // Row quantizer: out_int8 == false -> E4M3FN codes, true -> INT8 codes.
 tfq_status launch_quant_rows(const void* x, int64_t rows, int64_t K, float qmax, bool out_int8, void* q, float* s,
                              cudaStream_t stream, DeviceState* ds);
+
+// Self-check: the quantizer's division next to the IEEE division.
+tfq_status launch_div_selftest(const float* a, const float* b, int64_t n, float* ours, float* ieee,
+                               cudaStream_t stream);
 
 // Scaled FP8 GEMM with the fused scale/bias/BF16 epilogue.
 tfq_status launch_scaled_fp8_gemm(const void* A, const float* s_a, const void* W, const float* s_w,

@@ -24,6 +24,7 @@
 #include <cuda_bf16.h>
 
 #include <algorithm>
+#include <cmath>
 
 #include "tfq_internal.h"
 #include "tfq_ptx.cuh"
@@ -33,8 +34,17 @@ namespace {
 
 constexpr int kComputeWarps = 8;
 constexpr int kThreads = (kComputeWarps + 1) * 32;  // + one producer warp
-constexpr uint32_t kStageTarget = 32 * 1024;        // bytes of x per stage (target)
-constexpr uint32_t kSmemTarget = 100 * 1024;        // ring size target: two CTAs per SM
+#ifndef TFQ_QUANT_STAGE_KB
+#define TFQ_QUANT_STAGE_KB 32   // bytes of x per stage (target), KiB
+#endif
+#ifndef TFQ_QUANT_RING_KB
+#define TFQ_QUANT_RING_KB 72    // ring size target per CTA, KiB (three CTAs per SM)
+#endif
+#ifndef TFQ_QUANT_CTAS_PER_SM
+#define TFQ_QUANT_CTAS_PER_SM 3
+#endif
+constexpr uint32_t kStageTarget = TFQ_QUANT_STAGE_KB * 1024;
+constexpr uint32_t kSmemTarget = TFQ_QUANT_RING_KB * 1024;
 constexpr uint32_t kBulkPiece = 32 * 1024;          // one cp.async.bulk moves at most this
 
 struct QuantConfig {
@@ -72,10 +82,11 @@ __host__ QuantConfig choose_config(int64_t K) {
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
-// Packed max of two bf16x2 values whose halves are non-negative.
-__device__ __forceinline__ uint32_t max_bf16x2(uint32_t a, uint32_t b) {
+// Packed max of magnitudes: each bf16 half of the result has magnitude
+// max(|a|, |b|) (its sign bit is the XOR of the inputs' signs and is ignored).
+__device__ __forceinline__ uint32_t max_abs_bf16x2(uint32_t a, uint32_t b) {
     uint32_t d;
-    asm("max.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
     return d;
 }
 
@@ -95,20 +106,61 @@ __device__ __forceinline__ uint32_t to_int8_byte(float t) {
     return static_cast<uint32_t>(i) & 0xFFu;
 }
 
-// Quantizes the 8 bf16 values of `v` with scale `sc`: 8 output bytes.
-template <bool kInt8>
-__device__ __forceinline__ uint2 quantize8(uint4 v, float sc, float qmax) {
+}  // namespace
+
+// Correctly rounded fp32 quotient a / b, given y = RN(1/b), by Markstein's
+// method (P. Markstein, "Computation of elementary functions on the IBM
+// RISC System/6000 processor", IBM J. Res. Dev. 34(1), 1990): if y is the
+// correctly rounded reciprocal of b and q is a faithful approximation of
+// a/b, then r = a - b*q is exact in one FMA and RN(q + r*y) = RN(a/b).
+// q0 = RN(a*y) is within 1.5 ulp of a/b; one correction step makes it
+// faithful (q1 is within 1/2 ulp plus a term of order 2^-23 ulp), the
+// second step rounds it correctly.  The argument needs y and the residuals
+// to be normal numbers, which holds for |a| >= 2^-102 and
+// 2^-49 <= b <= 2^125 (every row scale is >= 1e-12 / 448 > 2^-49; rows with
+// a larger scale take the IEEE division instead).  For |a| < 2^-102 the
+// quotient is below 2^-53 in magnitude, so only its sign reaches the codes;
+// the final copysign keeps it, also for a = +-0.  Five FMA-pipe
+// instructions, no branch.  Checked against the IEEE division __fdiv_rn by
+// tfq_selftest_div_rn.
+__device__ __forceinline__ float div_rn_from_rcp(float a, float b, float y) {
+    const float q0 = __fmul_rn(a, y);
+    const float r0 = __fmaf_rn(-q0, b, a);
+    const float q1 = __fmaf_rn(r0, y, q0);
+    const float r1 = __fmaf_rn(-q1, b, a);
+    const float q2 = __fmaf_rn(r1, y, q1);
+    return copysignf(q2, a);
+}
+
+namespace {
+
+// Quantizes the 8 bf16 values of `v` with scale `sc` (rcp = RN(1/sc)): 8
+// output bytes.  kClamp: clamp x/s to +-qmax before the cast.  The clamp is
+// skipped when qmax is an E4M3 value: then |x/s| <= qmax + 1 ulp(qmax)
+// (s = RN(amax/qmax) and |x| <= amax), and qmax + 1 ulp encodes like qmax
+// because the nearest E4M3 midpoint is 2^-4 of a binade away (448 + ulp
+// saturates to 448).
+template <bool kInt8, bool kClamp, bool kIeeeDiv>
+__device__ __forceinline__ uint2 quantize8(uint4 v, float sc, float rcp, float qmax) {
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
     uint32_t packed[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-        float a = __fdiv_rn(bf16_lo(w[j]), sc);
-        float b = __fdiv_rn(bf16_hi(w[j]), sc);
+        float a, b;
+        if constexpr (kIeeeDiv) {
+            a = __fdiv_rn(bf16_lo(w[j]), sc);
+            b = __fdiv_rn(bf16_hi(w[j]), sc);
+        } else {
+            a = div_rn_from_rcp(bf16_lo(w[j]), sc, rcp);
+            b = div_rn_from_rcp(bf16_hi(w[j]), sc, rcp);
+        }
         if constexpr (kInt8) {
             packed[j] = to_int8_byte(a) | (to_int8_byte(b) << 8);
         } else {
-            a = fminf(fmaxf(a, -qmax), qmax);
-            b = fminf(fmaxf(b, -qmax), qmax);
+            if constexpr (kClamp) {
+                a = fminf(fmaxf(a, -qmax), qmax);
+                b = fminf(fmaxf(b, -qmax), qmax);
+            }
             packed[j] = cvt_e4m3x2(a, b);
         }
     }
@@ -120,7 +172,7 @@ __device__ __forceinline__ void record_failure(volatile int* abort_flag, uint32_
     atomicOr(err, bit);
 }
 
-template <bool kInt8>
+template <bool kInt8, bool kClamp>
 __global__ void __launch_bounds__(kThreads) quant_rows_kernel(const uint16_t* __restrict__ x, int64_t M, int K,
                                                               float qmax, uint8_t* __restrict__ q,
                                                               float* __restrict__ s, QuantConfig cfg,
@@ -205,15 +257,16 @@ __global__ void __launch_bounds__(kThreads) quant_rows_kernel(const uint16_t* __
         for (int r = slot; r < rows; r += nslots) {
             const uint4* row = reinterpret_cast<const uint4*>(stage + static_cast<size_t>(r) * row_bytes);
             // pass 1: max |x| (bf16 magnitudes, packed)
-            uint32_t m2 = 0;
+            uint32_t m2 = 0, m3 = 0;
 #pragma unroll 4
             for (int u = tr; u < units; u += team) {
                 const uint4 v = row[u];
-                m2 = max_bf16x2(m2, v.x & 0x7FFF7FFFu);
-                m2 = max_bf16x2(m2, v.y & 0x7FFF7FFFu);
-                m2 = max_bf16x2(m2, v.z & 0x7FFF7FFFu);
-                m2 = max_bf16x2(m2, v.w & 0x7FFF7FFFu);
+                m2 = max_abs_bf16x2(m2, v.x);
+                m3 = max_abs_bf16x2(m3, v.y);
+                m2 = max_abs_bf16x2(m2, v.z);
+                m3 = max_abs_bf16x2(m3, v.w);
             }
+            m2 = max_abs_bf16x2(m2, m3) & 0x7FFF7FFFu;
             float amax = fmaxf(bf16_lo(m2), bf16_hi(m2));
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
@@ -234,16 +287,34 @@ __global__ void __launch_bounds__(kThreads) quant_rows_kernel(const uint16_t* __
                 ++team_uses;
             }
             const float sc = __fdiv_rn(fmaxf(amax, 1e-12f), qmax);
+            const float rcp = __frcp_rn(sc);
             const int64_t grow = r0 + r;
             if (tr == 0) s[grow] = sc;
             // pass 2: quantize and store (8 bytes per thread, 256 B per warp)
             uint2* qrow = reinterpret_cast<uint2*>(q + grow * K);
+            if (sc <= 0x1p125f) {
 #pragma unroll 2
-            for (int u = tr; u < units; u += team) qrow[u] = quantize8<kInt8>(row[u], sc, qmax);
+                for (int u = tr; u < units; u += team)
+                    qrow[u] = quantize8<kInt8, kClamp, false>(row[u], sc, rcp, qmax);
+            } else {  // reciprocal would be subnormal: IEEE division (row-uniform branch)
+                for (int u = tr; u < units; u += team)
+                    qrow[u] = quantize8<kInt8, kClamp, true>(row[u], sc, rcp, qmax);
+            }
         }
         if (!ok) break;
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[st]);
+    }
+}
+
+// Element-wise self-check of div_rn_from_rcp against the IEEE division.
+__global__ void div_selftest_kernel(const float* __restrict__ a, const float* __restrict__ b, int64_t n,
+                                    float* __restrict__ ours, float* __restrict__ ieee) {
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const float x = a[i], y = b[i];
+        ours[i] = div_rn_from_rcp(x, y, __frcp_rn(y));
+        ieee[i] = __fdiv_rn(x, y);
     }
 }
 
@@ -253,7 +324,25 @@ __global__ void empty_rows_scale_kernel(int64_t M, float qmax, float* s) {
     if (i < M) s[i] = __fdiv_rn(1e-12f, qmax);
 }
 
+// True when v is exactly representable in E4M3FN (at most 4 significant bits,
+// within the normal range used for qmax).
+bool is_e4m3_value(float v) {
+    int e = 0;
+    const float m = std::frexp(v, &e) * 16.0f;  // 4 significant bits -> integer
+    return v >= 0x1p-6f && v <= 448.0f && m == std::floor(m);
+}
+
 }  // namespace
+
+tfq_status launch_div_selftest(const float* a, const float* b, int64_t n, float* ours, float* ieee,
+                               cudaStream_t stream) {
+    if (n == 0) return TFQ_OK;
+    const int threads = 256;
+    const int64_t blocks = std::min<int64_t>((n + threads - 1) / threads, 65535);
+    div_selftest_kernel<<<static_cast<unsigned>(blocks), threads, 0, stream>>>(a, b, n, ours, ieee);
+    const cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? TFQ_OK : fail(TFQ_ECUDA, "self-test launch: %s", cudaGetErrorString(e));
+}
 
 tfq_status launch_quant_rows(const void* x, int64_t rows, int64_t K, float qmax, bool out_int8, void* q, float* s,
                              cudaStream_t stream, DeviceState* ds) {
@@ -266,8 +355,10 @@ tfq_status launch_quant_rows(const void* x, int64_t rows, int64_t K, float qmax,
         return e == cudaSuccess ? TFQ_OK : fail(TFQ_ECUDA, "quantizer launch: %s", cudaGetErrorString(e));
     }
     const QuantConfig cfg = choose_config(K);
-    auto kernel = out_int8 ? quant_rows_kernel<true> : quant_rows_kernel<false>;
-    const int kidx = out_int8 ? 1 : 0;
+    const bool clamp = !out_int8 && !is_e4m3_value(qmax);
+    auto kernel = out_int8 ? quant_rows_kernel<true, false>
+                           : (clamp ? quant_rows_kernel<false, true> : quant_rows_kernel<false, false>);
+    const int kidx = out_int8 ? 2 : (clamp ? 1 : 0);
     if (!ds->quant_attr_set[kidx]) {
         const cudaError_t e =
             cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
@@ -276,7 +367,7 @@ tfq_status launch_quant_rows(const void* x, int64_t rows, int64_t K, float qmax,
     }
     const int64_t n_groups = (rows + cfg.rows_per_stage - 1) / cfg.rows_per_stage;
     const int per_sm = std::max(1, static_cast<int>((228u * 1024u) / (cfg.smem_bytes + 1024u)));
-    const int64_t grid = std::min<int64_t>(n_groups, static_cast<int64_t>(ds->sm_count) * std::min(per_sm, 2));
+    const int64_t grid = std::min<int64_t>(n_groups, static_cast<int64_t>(ds->sm_count) * std::min(per_sm, TFQ_QUANT_CTAS_PER_SM));
     kernel<<<static_cast<unsigned>(grid), kThreads, cfg.smem_bytes, stream>>>(
         static_cast<const uint16_t*>(x), rows, static_cast<int>(K), qmax, static_cast<uint8_t*>(q), s, cfg,
         ds->err_word);

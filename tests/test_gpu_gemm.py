@@ -45,6 +45,16 @@ def test_ragged_full_compare(M, N, K, with_bias):
     _run_case(M, N, K, with_bias, seed=M + N + K)
 
 
+@pytest.mark.parametrize("M,N,K", [(512, 256, 128), (513, 264, 144), (777, 520, 1024), (1024, 136, 48),
+                                   (2128, 1032, 512), (3000, 3072, 256)])
+@pytest.mark.parametrize("with_bias", [True, False])
+def test_pair_kernel_full_compare(M, N, K, with_bias):
+    """M >= 512 runs the CTA-pair (cta_group::2) kernel: 256-row tiles split
+    over two SMs, ragged M (a CTA of the last pair may have no valid rows),
+    ragged N inside a 256-column tile, K tails."""
+    _run_case(M, N, K, with_bias, seed=7 * M + N + K)
+
+
 def test_many_tiles_persistent():
     """More tiles than SMs, several tiles per CTA, both accumulator buffers."""
     _run_case(1100, 2048, 512, True, seed=3)

@@ -32,10 +32,12 @@ def test_tiny_config_activation():
     _assert_fp8_equal(x, 448.0)
 
 
-@pytest.mark.parametrize("qmax", [448.0, 14.0, 7.0])
+@pytest.mark.parametrize("qmax", [448.0, 14.0, 7.0, 21.0, 100.0, 12.0])
 @pytest.mark.parametrize("M,K", [(1, 16), (3, 48), (37, 256), (129, 1024), (65, 3072), (33, 5120),
                                  (17, 12288), (9, 13824), (5, 32768), (300, 160)])
 def test_ragged_shapes(M, K, qmax):
+    """qmax 21 and 100 are not E4M3 numbers (21 is the midpoint of 20 and
+    22): the kernel clamps x/s there; for the others it needs no clamp."""
     x = workloads.activations(M, K, seed=M * 7 + K, nu=3, amplitude=4.0, outlier_cols=max(1, K // 100),
                               outlier_mult=30.0, zero_rows=1 if M > 2 else 0, device="cuda")
     _assert_fp8_equal(x, qmax)
@@ -88,8 +90,20 @@ def test_rounding_edges():
     x[4, :8] = torch.tensor([1e-13, -3e-13, 2e-13, 0, 0, 0, 0, -1e-14])   # below the floor
     x[5, :row.numel()] = row * 3.0                 # a non-power-of-two scale
     x = x.to(torch.bfloat16).cuda()
-    for qmax in (448.0, 14.0, 7.0):
+    for qmax in (448.0, 14.0, 7.0, 21.0, 100.0):
         _assert_fp8_equal(x, qmax)
+
+
+@pytest.mark.parametrize("qmax", [1.0, 2.0, 448.0])
+def test_huge_magnitude_rows(qmax):
+    """Rows near the bf16 maximum: with a small qmax the scale exceeds 2^125
+    and the kernel takes its IEEE-division branch for the row."""
+    x = workloads.activations(40, 256, seed=3, device="cuda").float()
+    x[:20] *= 3.0e38 / x[:20].abs().amax(dim=1, keepdim=True)
+    x[20:30] *= 1.0e30
+    x = x.to(torch.bfloat16)
+    assert torch.isfinite(x.float()).all()
+    _assert_fp8_equal(x, qmax)
 
 
 def test_empty_and_k0():
