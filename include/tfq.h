@@ -68,9 +68,9 @@ typedef enum tfq_status {
 /* Output element type of the per-row weight quantizer. */
 enum { TFQ_DTYPE_FP8_E4M3 = 0, TFQ_DTYPE_INT8 = 1 };
 
-/* Largest K (row length) the row quantizers accept: a row is staged whole
- * in shared memory.  Larger K returns TFQ_EUNSUPPORTED. */
-#define TFQ_QUANT_MAX_K 32768
+/* Largest K (row length) the row quantizers accept (keeps the kernels' index
+ * arithmetic in 32 bits).  Larger K returns TFQ_EUNSUPPORTED. */
+#define TFQ_QUANT_MAX_K (1 << 24)
 
 /*
  * Per-token FP8 activation quantization (step 1 above).
@@ -119,6 +119,34 @@ TFQ_API tfq_status tfq_quant_weight_per_channel(const void *w_bf16, int64_t N, i
 TFQ_API tfq_status tfq_scaled_fp8_linear(const void *A_q, const float *s_a, const void *W_q,
                                  const float *s_w, const void *bias_bf16, int64_t M, int64_t N,
                                  int64_t K, void *out_bf16, void *stream);
+
+/*
+ * INT8 W8A8 (the int8 modes of the LightX2V "模型量化技术" page, quantization-
+ * mode table: INT8 per-channel symmetric weights, dynamic per-token symmetric
+ * INT8 activations), with the integer formula of the TeleFuser
+ * "Quantization" page, section "Core ideas".
+ *
+ * tfq_quant_act_int8_per_token: x bf16 [M, K] -> q int8 [M, K],
+ *   s[m] = fl32(max(amax_m, 1e-12f) / qmax),
+ *   q = clamp(round_half_even(fl32(x / s)), -128, 127); qmax in [1, 127]
+ *   (the pages use 127).  Same preconditions and errors as
+ *   tfq_quant_act_fp8_per_token.
+ */
+TFQ_API tfq_status tfq_quant_act_int8_per_token(const void *x_bf16, int64_t M, int64_t K, float qmax,
+                                                void *q_int8, float *s, void *stream);
+
+/*
+ * tfq_scaled_int8_linear: as tfq_scaled_fp8_linear with int8 operands:
+ *   A_q int8 [M, K], W_q int8 [N, K] (both K-contiguous), s_a [M], s_w [N]
+ *   fp32, bias bf16 [N] or NULL, out bf16 [M, N]:
+ *   out[m,n] = bf16_rn(fp32(sum_k A_q[m,k] W_q[n,k]) * s_a[m] * s_w[n] + bias[n]),
+ * the integer sum exact in s32 on the tensor cores (|sum| <= 128^2 K < 2^31
+ * for K < 131072), converted to fp32 (round to nearest) in the epilogue.
+ * Same preconditions, tolerance and errors as tfq_scaled_fp8_linear.
+ */
+TFQ_API tfq_status tfq_scaled_int8_linear(const void *A_q, const float *s_a, const void *W_q,
+                                          const float *s_w, const void *bias_bf16, int64_t M, int64_t N,
+                                          int64_t K, void *out_bf16, void *stream);
 
 /*
  * Bytes of the static device array used by tfq_scaled_fp8_linear_noalloc.

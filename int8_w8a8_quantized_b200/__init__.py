@@ -24,8 +24,11 @@ from ._capi import (  # noqa: F401
     status_string,
     tfq_device_error,
     tfq_quant_act_fp8_per_token,
+    tfq_quant_act_int8_per_token,
     tfq_quant_weight_per_channel,
     tfq_scaled_fp8_linear,
+    tfq_scaled_int8_linear,
+    w8a8_int8_linear,
     w8a8_linear,
 )
 
@@ -33,6 +36,9 @@ __all__ = [
     "tfq_quant_act_fp8_per_token",
     "tfq_quant_weight_per_channel",
     "tfq_scaled_fp8_linear",
+    "tfq_quant_act_int8_per_token",
+    "tfq_scaled_int8_linear",
+    "w8a8_int8_linear",
     "tfq_device_error",
     "w8a8_linear",
     "TfqError",

@@ -24,7 +24,7 @@ LIB_PATH = os.path.join(PKG, "libtfq.so")
 
 TFQ_OK, TFQ_EINVAL, TFQ_EUNSUPPORTED, TFQ_ECUDA, TFQ_ETIMEOUT = range(5)
 TFQ_DTYPE_FP8_E4M3, TFQ_DTYPE_INT8 = 0, 1
-TFQ_QUANT_MAX_K = 32768
+TFQ_QUANT_MAX_K = 1 << 24
 
 # name -> (restype, argtypes), in the order include/tfq.h declares them
 _P, _I64, _F, _I = ctypes.c_void_p, ctypes.c_int64, ctypes.c_float, ctypes.c_int
@@ -32,6 +32,8 @@ SIGNATURES = {
     "tfq_quant_act_fp8_per_token": (_I, [_P, _I64, _I64, _F, _P, _P, _P]),
     "tfq_quant_weight_per_channel": (_I, [_P, _I64, _I64, _I, _F, _P, _P, _P]),
     "tfq_scaled_fp8_linear": (_I, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _P]),
+    "tfq_quant_act_int8_per_token": (_I, [_P, _I64, _I64, _F, _P, _P, _P]),
+    "tfq_scaled_int8_linear": (_I, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _P]),
     "tfq_scaled_fp8_linear_noalloc": (_I, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _P]),
     "tfq_selftest_div_rn": (_I, [_P, _P, _I64, _P, _P, _P]),
     "tfq_device_error": (_I, [_P]),
@@ -187,6 +189,61 @@ def tfq_scaled_fp8_linear(A_q, s_a, W_q, s_w, bias=None, out=None, stream=None):
                                        _stream_handle(stream))
     _check(st, "tfq_scaled_fp8_linear")
     return out
+
+
+def tfq_quant_act_int8_per_token(x, qmax: float = 127.0, q=None, s=None, stream=None):
+    """x bf16 [M, K] -> (q int8 [M, K], s fp32 [M]): dynamic per-token INT8."""
+    import torch
+    _require(x, torch.bfloat16, 2, "x")
+    M, K = x.shape
+    if q is None:
+        q = torch.empty((M, K), dtype=torch.int8, device=x.device)
+    if s is None:
+        s = torch.empty((M,), dtype=torch.float32, device=x.device)
+    _require(q, torch.int8, 2, "q")
+    _require(s, torch.float32, 1, "s")
+    if tuple(q.shape) != (M, K) or tuple(s.shape) != (M,):
+        raise ValueError("output shapes do not match x")
+    with torch.cuda.device(x.device):
+        st = raw.tfq_quant_act_int8_per_token(x.data_ptr(), M, K, float(qmax), q.data_ptr(), s.data_ptr(),
+                                              _stream_handle(stream))
+    _check(st, "tfq_quant_act_int8_per_token")
+    return q, s
+
+
+def tfq_scaled_int8_linear(A_q, s_a, W_q, s_w, bias=None, out=None, stream=None):
+    """A_q int8 [M, K], s_a fp32 [M], W_q int8 [N, K], s_w fp32 [N], bias bf16 [N] or None
+    -> out bf16 [M, N]."""
+    import torch
+    _require(A_q, torch.int8, 2, "A_q")
+    _require(W_q, torch.int8, 2, "W_q")
+    _require(s_a, torch.float32, 1, "s_a")
+    _require(s_w, torch.float32, 1, "s_w")
+    M, K = A_q.shape
+    N, K2 = W_q.shape
+    if K2 != K or s_a.shape[0] != M or s_w.shape[0] != N:
+        raise ValueError("shape mismatch")
+    if bias is not None:
+        _require(bias, torch.bfloat16, 1, "bias")
+        if bias.shape[0] != N:
+            raise ValueError("bias shape")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=A_q.device)
+    _require(out, torch.bfloat16, 2, "out")
+    if tuple(out.shape) != (M, N):
+        raise ValueError("out shape")
+    with torch.cuda.device(A_q.device):
+        st = raw.tfq_scaled_int8_linear(A_q.data_ptr(), s_a.data_ptr(), W_q.data_ptr(), s_w.data_ptr(),
+                                        None if bias is None else bias.data_ptr(), M, N, K, out.data_ptr(),
+                                        _stream_handle(stream))
+    _check(st, "tfq_scaled_int8_linear")
+    return out
+
+
+def w8a8_int8_linear(x, W_q, s_w, bias=None, qmax: float = 127.0, stream=None):
+    """The INT8 Linear: per-token INT8 quantization of x, then the scaled INT8 GEMM."""
+    A_q, s_a = tfq_quant_act_int8_per_token(x, qmax, stream=stream)
+    return tfq_scaled_int8_linear(A_q, s_a, W_q, s_w, bias, stream=stream)
 
 
 def tfq_device_error(stream=None) -> None:

@@ -59,10 +59,15 @@ constexpr size_t SMEM_BARS = (2 * STAGES + 4 + 1) * 8 + 16;
 constexpr size_t SMEM_BYTES = 1024 /* alignment slack */ + SMEM_RING + SMEM_EPI + SMEM_BARS;
 static_assert(SMEM_BYTES <= 232448, "shared memory budget exceeded");
 
-// Instruction descriptor of tcgen05.mma kind::f8f6f4: fp32 accumulator
-// (bits 4-5 = 1), A and B E4M3 (format 0 in bits 7-9 and 10-12), both
+// Instruction descriptor of tcgen05.mma: accumulator format in bits 4-5
+// (1 = F32 for kind::f8f6f4, 2 = S32 for kind::i8), A and B formats in bits
+// 7-9 and 10-12 (E4M3 = 0 for f8f6f4; signed 8-bit = 1 for i8), both
 // K-major (bits 15, 16 = 0), N >> 3 in bits 17-22, M >> 4 in bits 24-28.
-constexpr uint32_t IDESC = (1u << 4) | (static_cast<uint32_t>(BN >> 3) << 17) | (static_cast<uint32_t>(BM >> 4) << 24);
+template <bool kI8>
+constexpr uint32_t make_idesc(int m, int n) {
+    return (kI8 ? (2u << 4) | (1u << 7) | (1u << 10) : (1u << 4)) | (static_cast<uint32_t>(n >> 3) << 17) |
+           (static_cast<uint32_t>(m >> 4) << 24);
+}
 
 struct GemmArgs {
     const float* s_a;
@@ -89,6 +94,17 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return d;
 }
 
+// An accumulator word as fp32: the F32 accumulator as is, the S32 one
+// converted (round to nearest).
+template <bool kI8>
+__device__ __forceinline__ float acc_value(uint32_t w) {
+    if constexpr (kI8) {
+        return __int2float_rn(static_cast<int>(w));
+    } else {
+        return __uint_as_float(w);
+    }
+}
+
 __device__ __forceinline__ void give_up(volatile int* abort_flag, uint32_t* err, uint32_t bit) {
     *abort_flag = 1;
     atomicOr(err, bit);
@@ -99,7 +115,7 @@ __device__ __forceinline__ void give_up(volatile int* abort_flag, uint32_t* err,
 // staging buffer -> TMA store, EPI_COLS columns at a time.  `t_row` is the
 // TMEM address of this warp's 32 lanes at the tile's first column; `chunk`
 // counts stores of this warp (selects the staging buffer).
-template <int kBN>
+template <int kBN, bool kI8>
 __device__ __forceinline__ void store_tile_rows(const GemmArgs& p, const CUtensorMap& tmY, uint32_t t_row,
                                                 uint8_t* ebuf0, int& chunk, int n_tile0, int row0, float sa,
                                                 int lane) {
@@ -145,9 +161,9 @@ __device__ __forceinline__ void store_tile_rows(const GemmArgs& p, const CUtenso
                 uint32_t packed[4];
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
-                    const float y0 = fmaf(__uint_as_float(acc[h][g * 8 + 2 * j]) * sa, sw[2 * j], bb[2 * j]);
+                    const float y0 = fmaf(acc_value<kI8>(acc[h][g * 8 + 2 * j]) * sa, sw[2 * j], bb[2 * j]);
                     const float y1 =
-                        fmaf(__uint_as_float(acc[h][g * 8 + 2 * j + 1]) * sa, sw[2 * j + 1], bb[2 * j + 1]);
+                        fmaf(acc_value<kI8>(acc[h][g * 8 + 2 * j + 1]) * sa, sw[2 * j + 1], bb[2 * j + 1]);
                     packed[j] = pack_bf16x2(y0, y1);
                 }
                 // 128-byte swizzle: 16-byte unit u of row r lives at unit u ^ (r % 8).
@@ -166,8 +182,9 @@ __device__ __forceinline__ void store_tile_rows(const GemmArgs& p, const CUtenso
     }
 }
 
+template <bool kI8>
 __global__ void __launch_bounds__(THREADS, 1)
-    scaled_fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+    scaled_mm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                            const __grid_constant__ CUtensorMap tmY, GemmArgs p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -269,7 +286,8 @@ __global__ void __launch_bounds__(THREADS, 1)
                     for (int k = 0; k < BK / UMMA_K; ++k) {
                         // advance the start address by k * 32 bytes inside the swizzle atom
                         const uint64_t koff = static_cast<uint64_t>((k * UMMA_K) >> 4);
-                        mma_e4m3(d_tmem, a_desc + koff, b_desc + koff, IDESC, (kb | k) != 0 ? 1u : 0u);
+                        mma_e4m3<kI8>(d_tmem, a_desc + koff, b_desc + koff, make_idesc<kI8>(BM, BN),
+                                      (kb | k) != 0 ? 1u : 0u);
                     }
                     mma_commit(&empty[st]);
                 }
@@ -300,7 +318,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             const float sa = (m < p.M) ? __ldg(p.s_a + m) : 0.0f;
             const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
                                    static_cast<uint32_t>(buf * BN);
-            store_tile_rows<BN>(p, tmY, t_row, ebuf0, chunk, tn * BN, row0, sa, lane);
+            store_tile_rows<BN, kI8>(p, tmY, t_row, ebuf0, chunk, tn * BN, row0, sa, lane);
             // All of this warp's TMEM reads of `buf` are complete: hand it back.
             tc_fence_before();
             __syncwarp();
@@ -344,8 +362,6 @@ struct PairCfg {
     static constexpr int kTmemCols = 512;                       // two PBN-column accumulators, power of 2
     static constexpr size_t kRing = static_cast<size_t>(PAIR_STAGES) * (kAStage + kBStage);
     static constexpr size_t kSmem = 1024 + kRing + SMEM_EPI + (2 * PAIR_STAGES + 4 + 1) * 8 + 16;
-    static constexpr uint32_t kIdesc =
-        (1u << 4) | (static_cast<uint32_t>(PBN >> 3) << 17) | (static_cast<uint32_t>(256 >> 4) << 24);
     static_assert(kSmem <= 232448, "shared memory budget exceeded");
     static_assert(2 * PBN <= kTmemCols, "two accumulators must fit in TMEM");
     static_assert(PBN % 64 == 0 && PBN >= 64 && PBN <= 256, "N tile");
@@ -361,9 +377,9 @@ __device__ __forceinline__ void pair_tile_coords(int t, int m_tiles, int n_tiles
     tn = r / gsize;
 }
 
-template <int PBN>
+template <int PBN, bool kI8>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
-    scaled_fp8_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+    scaled_mm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                                 const __grid_constant__ CUtensorMap tmY, GemmArgs p) {
     using C = PairCfg<PBN>;
     extern __shared__ uint8_t smem_raw[];
@@ -477,7 +493,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
 #pragma unroll
                     for (int k = 0; k < BK / UMMA_K; ++k) {
                         const uint64_t koff = static_cast<uint64_t>((k * UMMA_K) >> 4);
-                        mma_e4m3_pair(d_tmem, a_desc + koff, b_desc + koff, C::kIdesc, (kb | k) != 0 ? 1u : 0u);
+                        mma_e4m3_pair<kI8>(d_tmem, a_desc + koff, b_desc + koff, make_idesc<kI8>(256, PBN),
+                                           (kb | k) != 0 ? 1u : 0u);
                     }
                     mma_commit_pair(&empty[st], 0x3);
                 }
@@ -509,7 +526,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             const float sa = (m < p.M) ? __ldg(p.s_a + m) : 0.0f;
             const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
                                    static_cast<uint32_t>(buf * PBN);
-            store_tile_rows<PBN>(p, tmY, t_row, ebuf0, chunk, tn * PBN, row0, sa, lane);
+            store_tile_rows<PBN, kI8>(p, tmY, t_row, ebuf0, chunk, tn * PBN, row0, sa, lane);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(buf == 0 ? tmem_empty_leader0 : tmem_empty_leader1);
@@ -536,27 +553,28 @@ bool use_pair_kernel(int64_t M, int sm_count) { return M >= TFQ_GEMM_PAIR_MIN_M 
 
 }  // namespace
 
-tfq_status launch_scaled_fp8_gemm(const void* A, const float* s_a, const void* W, const float* s_w,
-                                  const void* bias, int64_t M, int64_t N, int64_t K, void* out,
-                                  cudaStream_t stream, DeviceState* ds) {
+namespace {
+
+template <bool kI8>
+tfq_status launch_scaled_mm(const void* A, const float* s_a, const void* W, const float* s_w, const void* bias,
+                            int64_t M, int64_t N, int64_t K, void* out, cudaStream_t stream, DeviceState* ds) {
     if (M == 0 || N == 0) return TFQ_OK;
-    CUtensorMap tmA, tmB, tmY;
+    CUtensorMap tmA, tmY;
     tfq_status st = encode_tensor_map_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, A, K, M, K, BK, BM,
                                          CU_TENSOR_MAP_SWIZZLE_128B);
-    if (st != TFQ_OK) return st;
-    st = encode_tensor_map_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, W, K, N, K, BK, BN, CU_TENSOR_MAP_SWIZZLE_128B);
     if (st != TFQ_OK) return st;
     st = encode_tensor_map_2d(&tmY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, out, N, M, N * 2, EPI_COLS, 32,
                               CU_TENSOR_MAP_SWIZZLE_128B);
     if (st != TFQ_OK) return st;
-    if (!ds->gemm_attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(scaled_fp8_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    const int attr_idx = kI8 ? 1 : 0;
+    if (!ds->gemm_attr_set[attr_idx]) {
+        cudaError_t e = cudaFuncSetAttribute(scaled_mm_kernel<kI8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              static_cast<int>(SMEM_BYTES));
         if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(scaled_fp8_gemm_pair_kernel<256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+            e = cudaFuncSetAttribute(scaled_mm_pair_kernel<256, kI8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      static_cast<int>(PairCfg<256>::kSmem));
         if (e != cudaSuccess) return fail(TFQ_ECUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
-        ds->gemm_attr_set = true;
+        ds->gemm_attr_set[attr_idx] = true;
     }
     GemmArgs a;
     a.s_a = s_a;
@@ -578,14 +596,31 @@ tfq_status launch_scaled_fp8_gemm(const void* A, const float* s_a, const void* W
         if (st != TFQ_OK) return st;
         const int64_t pair_tiles = ((M + 255) / 256) * static_cast<int64_t>(a.n_tiles);
         const int clusters = static_cast<int>(std::min<int64_t>(pair_tiles, ds->sm_count / 2));
-        scaled_fp8_gemm_pair_kernel<256>
-            <<<2 * clusters, THREADS, PairCfg<256>::kSmem, stream>>>(tmA, tmBh, tmY, a);
+        scaled_mm_pair_kernel<256, kI8><<<2 * clusters, THREADS, PairCfg<256>::kSmem, stream>>>(tmA, tmBh, tmY, a);
     } else {
+        CUtensorMap tmB;
+        st = encode_tensor_map_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, W, K, N, K, BK, BN,
+                                  CU_TENSOR_MAP_SWIZZLE_128B);
+        if (st != TFQ_OK) return st;
         const int grid = static_cast<int>(std::min<int64_t>(tiles, ds->sm_count));
-        scaled_fp8_gemm_kernel<<<grid, THREADS, SMEM_BYTES, stream>>>(tmA, tmB, tmY, a);
+        scaled_mm_kernel<kI8><<<grid, THREADS, SMEM_BYTES, stream>>>(tmA, tmB, tmY, a);
     }
     const cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? TFQ_OK : fail(TFQ_ECUDA, "GEMM launch: %s", cudaGetErrorString(e));
+}
+
+}  // namespace
+
+tfq_status launch_scaled_fp8_gemm(const void* A, const float* s_a, const void* W, const float* s_w,
+                                  const void* bias, int64_t M, int64_t N, int64_t K, void* out,
+                                  cudaStream_t stream, DeviceState* ds) {
+    return launch_scaled_mm<false>(A, s_a, W, s_w, bias, M, N, K, out, stream, ds);
+}
+
+tfq_status launch_scaled_int8_gemm(const void* A, const float* s_a, const void* W, const float* s_w,
+                                   const void* bias, int64_t M, int64_t N, int64_t K, void* out,
+                                   cudaStream_t stream, DeviceState* ds) {
+    return launch_scaled_mm<true>(A, s_a, W, s_w, bias, M, N, K, out, stream, ds);
 }
 
 }  // namespace tfq

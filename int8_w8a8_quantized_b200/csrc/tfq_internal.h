@@ -12,8 +12,6 @@ namespace tfq {
 
 // Bits of the per-device error word (which role of which kernel gave up).
 enum : uint32_t {
-    kErrQuantProducer = 1u << 0,
-    kErrQuantConsumer = 1u << 1,
     kErrGemmProducer = 1u << 4,
     kErrGemmMma = 1u << 5,
     kErrGemmEpilogue = 1u << 6,
@@ -26,8 +24,7 @@ struct DeviceState {
     int cc_major = 0, cc_minor = 0;
     size_t smem_optin = 0;          // max dynamic shared memory per block
     uint32_t* err_word = nullptr;   // device memory, one 32-bit word
-    bool quant_attr_set[3] = {false, false, false};
-    bool gemm_attr_set = false;
+    bool gemm_attr_set[2] = {false, false};  // FP8, INT8
 };
 
 // Per-device state of the current device, created on first use.  Returns
@@ -60,5 +57,10 @@ tfq_status launch_div_selftest(const float* a, const float* b, int64_t n, float*
 tfq_status launch_scaled_fp8_gemm(const void* A, const float* s_a, const void* W, const float* s_w,
                                   const void* bias, int64_t M, int64_t N, int64_t K, void* out,
                                   cudaStream_t stream, DeviceState* ds);
+
+// Scaled INT8 GEMM (S8 x S8 -> S32 on the tensor cores) with the same epilogue.
+tfq_status launch_scaled_int8_gemm(const void* A, const float* s_a, const void* W, const float* s_w,
+                                   const void* bias, int64_t M, int64_t N, int64_t K, void* out,
+                                   cudaStream_t stream, DeviceState* ds);
 
 }  // namespace tfq

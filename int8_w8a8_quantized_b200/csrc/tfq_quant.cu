@@ -11,16 +11,17 @@
 // the symmetric INT8 formula of the TeleFuser page (section "Core ideas").
 // Rows are tokens (activations) or output channels (weights).
 //
-// Design (B200): each CTA is persistent over groups of consecutive rows.
-// One producer thread streams row groups HBM -> shared memory with 1-D bulk
-// copies (cp.async.bulk, completion on an mbarrier) into a ring of stages,
-// so tens of KB per SM are in flight with a single issuing thread.  Eight
-// consumer warps split each stage: a "team" of 1, 2, 4 or 8 warps owns one
-// row, reduces |x| with packed bf16x2 max + warp shuffles (and, for teams
-// larger than one warp, an mbarrier-synchronised exchange through shared
-// memory), then re-reads the row from shared memory, divides, converts two
-// values per cvt instruction and stores 8 output bytes per thread per step
-// (a warp writes 256 contiguous bytes).  Every wait is bounded.
+// Design (B200): one warp per row, rows strided over a grid of two CTAs of
+// eight warps per SM; no shared memory, no barriers, no waits.  Pass 1 loads
+// a whole segment of the row (16 x 16-byte loads per lane: 8 KiB per warp in
+// flight, a warp reads 512 contiguous bytes per load) and reduces |x| with
+// packed max.xorsign.abs.bf16x2 and shuffles.  Pass 2 quantizes: a row of
+// at most one segment (K <= 4096) is still in registers; a longer row is
+// read again, which hits L2 because pass 1 loaded it with an evict_last
+// cache policy (so HBM sees 2 bytes read and 1 written per element).  The
+// division is a branch-free correctly rounded one (Markstein's method from
+// the row's reciprocal); two values are converted per cvt instruction and a
+// lane stores 8 codes at a time (a warp writes 256 contiguous bytes).
 #include <cuda_bf16.h>
 
 #include <algorithm>
@@ -32,52 +33,7 @@
 namespace tfq {
 namespace {
 
-constexpr int kComputeWarps = 8;
-constexpr int kThreads = (kComputeWarps + 1) * 32;  // + one producer warp
-#ifndef TFQ_QUANT_STAGE_KB
-#define TFQ_QUANT_STAGE_KB 32   // bytes of x per stage (target), KiB
-#endif
-#ifndef TFQ_QUANT_RING_KB
-#define TFQ_QUANT_RING_KB 72    // ring size target per CTA, KiB (three CTAs per SM)
-#endif
-#ifndef TFQ_QUANT_CTAS_PER_SM
-#define TFQ_QUANT_CTAS_PER_SM 3
-#endif
-constexpr uint32_t kStageTarget = TFQ_QUANT_STAGE_KB * 1024;
-constexpr uint32_t kSmemTarget = TFQ_QUANT_RING_KB * 1024;
-constexpr uint32_t kBulkPiece = 32 * 1024;          // one cp.async.bulk moves at most this
-
-struct QuantConfig {
-    int rows_per_stage;
-    int warps_per_row;  // team size: 1, 2, 4 or 8
-    int stages;
-    uint32_t stage_bytes;
-    uint32_t smem_bytes;
-};
-
-__host__ QuantConfig choose_config(int64_t K) {
-    QuantConfig c{};
-    const uint32_t row_bytes = static_cast<uint32_t>(2 * K);
-    int r = static_cast<int>(std::max<uint32_t>(1u, kStageTarget / row_bytes));
-    if (r >= 8) {
-        c.warps_per_row = 1;
-        c.rows_per_stage = std::min(r, 64);
-    } else if (r >= 4) {
-        c.warps_per_row = 2;
-        c.rows_per_stage = 4;
-    } else if (r >= 2) {
-        c.warps_per_row = 4;
-        c.rows_per_stage = 2;
-    } else {
-        c.warps_per_row = 8;
-        c.rows_per_stage = 1;
-    }
-    c.stage_bytes = (static_cast<uint32_t>(c.rows_per_stage) * row_bytes + 127u) & ~127u;
-    c.stages = static_cast<int>(std::min<uint32_t>(8u, std::max<uint32_t>(2u, kSmemTarget / c.stage_bytes)));
-    // ring + full/empty barriers + team barriers + amax exchange + abort flag
-    c.smem_bytes = c.stages * c.stage_bytes + 2 * c.stages * 8 + kComputeWarps * 8 + 2 * kComputeWarps * 4 + 16;
-    return c;
-}
+constexpr int kCtasPerSm = 2;  // 8 warps per CTA; ~125 registers per thread allow two per SM
 
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
@@ -123,13 +79,15 @@ __device__ __forceinline__ uint32_t to_int8_byte(float t) {
 // the final copysign keeps it, also for a = +-0.  Five FMA-pipe
 // instructions, no branch.  Checked against the IEEE division __fdiv_rn by
 // tfq_selftest_div_rn.
-__device__ __forceinline__ float div_rn_from_rcp(float a, float b, float y) {
+__device__ __forceinline__ float div_rn_from_rcp_unsigned_zero(float a, float b, float y) {
     const float q0 = __fmul_rn(a, y);
     const float r0 = __fmaf_rn(-q0, b, a);
     const float q1 = __fmaf_rn(r0, y, q0);
     const float r1 = __fmaf_rn(-q1, b, a);
-    const float q2 = __fmaf_rn(r1, y, q1);
-    return copysignf(q2, a);
+    return __fmaf_rn(r1, y, q1);
+}
+__device__ __forceinline__ float div_rn_from_rcp(float a, float b, float y) {
+    return copysignf(div_rn_from_rcp_unsigned_zero(a, b, y), a);
 }
 
 namespace {
@@ -140,170 +98,157 @@ namespace {
 // (s = RN(amax/qmax) and |x| <= amax), and qmax + 1 ulp encodes like qmax
 // because the nearest E4M3 midpoint is 2^-4 of a binade away (448 + ulp
 // saturates to 448).
+// Two bf16 values (one 32-bit word) -> two codes in the low 16 bits.
+// (The Markstein quotient here may come out as +0 for a = -0; the caller
+// restores the sign of zero codes from the inputs' sign bits, which is
+// exact because every other quotient already carries the sign of a, and an
+// INT8 code has no negative zero.)
 template <bool kInt8, bool kClamp, bool kIeeeDiv>
-__device__ __forceinline__ uint2 quantize8(uint4 v, float sc, float rcp, float qmax) {
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-    uint32_t packed[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        float a, b;
-        if constexpr (kIeeeDiv) {
-            a = __fdiv_rn(bf16_lo(w[j]), sc);
-            b = __fdiv_rn(bf16_hi(w[j]), sc);
-        } else {
-            a = div_rn_from_rcp(bf16_lo(w[j]), sc, rcp);
-            b = div_rn_from_rcp(bf16_hi(w[j]), sc, rcp);
-        }
-        if constexpr (kInt8) {
-            packed[j] = to_int8_byte(a) | (to_int8_byte(b) << 8);
-        } else {
-            if constexpr (kClamp) {
-                a = fminf(fmaxf(a, -qmax), qmax);
-                b = fminf(fmaxf(b, -qmax), qmax);
-            }
-            packed[j] = cvt_e4m3x2(a, b);
-        }
+__device__ __forceinline__ uint32_t quantize2(uint32_t w, float sc, float rcp, float qmax) {
+    float a, b;
+    if constexpr (kIeeeDiv) {
+        a = __fdiv_rn(bf16_lo(w), sc);
+        b = __fdiv_rn(bf16_hi(w), sc);
+    } else {
+        a = div_rn_from_rcp_unsigned_zero(bf16_lo(w), sc, rcp);
+        b = div_rn_from_rcp_unsigned_zero(bf16_hi(w), sc, rcp);
     }
-    return make_uint2(packed[0] | (packed[1] << 16), packed[2] | (packed[3] << 16));
+    if constexpr (kInt8) {
+        return to_int8_byte(a) | (to_int8_byte(b) << 8);
+    } else {
+        if constexpr (kClamp) {
+            a = fminf(fmaxf(a, -qmax), qmax);
+            b = fminf(fmaxf(b, -qmax), qmax);
+        }
+        return cvt_e4m3x2(a, b);
+    }
 }
 
-__device__ __forceinline__ void record_failure(volatile int* abort_flag, uint32_t* err, uint32_t bit) {
-    *abort_flag = 1;
-    atomicOr(err, bit);
+// Sign bits of the four bf16 values in (w0, w1) moved to bit 7 of the four
+// bytes of the result (the high byte of every bf16 carries its sign in bit 7).
+__device__ __forceinline__ uint32_t sign_bytes(uint32_t w0, uint32_t w1) {
+    return __byte_perm(w0, w1, 0x7531) & 0x80808080u;
+}
+
+template <bool kInt8, bool kClamp, bool kIeeeDiv>
+__device__ __forceinline__ uint2 quantize8(uint4 v, float sc, float rcp, float qmax) {
+    const uint32_t p0 = quantize2<kInt8, kClamp, kIeeeDiv>(v.x, sc, rcp, qmax);
+    const uint32_t p1 = quantize2<kInt8, kClamp, kIeeeDiv>(v.y, sc, rcp, qmax);
+    const uint32_t p2 = quantize2<kInt8, kClamp, kIeeeDiv>(v.z, sc, rcp, qmax);
+    const uint32_t p3 = quantize2<kInt8, kClamp, kIeeeDiv>(v.w, sc, rcp, qmax);
+    uint32_t lo = p0 | (p1 << 16), hi = p2 | (p3 << 16);
+    if constexpr (!kInt8) {  // E4M3 codes keep the sign of (negative) zero
+        lo |= sign_bytes(v.x, v.y);
+        hi |= sign_bytes(v.z, v.w);
+    }
+    return make_uint2(lo, hi);
+}
+
+// Global loads: 16 bytes, not allocated in L1.
+__device__ __forceinline__ uint4 ldg_nc_v4(const uint4* p) {
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+#ifndef TFQ_QUANT_L2_KEEP
+#define TFQ_QUANT_L2_KEEP 1  // pass-1 loads ask L2 to keep the row for pass 2
+#endif
+// Load with an L2 cache policy (from createpolicy).
+__device__ __forceinline__ uint4 ldg_nc_v4_policy(const uint4* p, uint64_t policy) {
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.v4.u32 {%0, %1, %2, %3}, [%4], %5;"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p), "l"(policy));
+    return v;
+}
+__device__ __forceinline__ uint64_t l2_policy_evict_last() {
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+__device__ __forceinline__ uint64_t l2_policy_evict_first() {
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+
+__device__ __forceinline__ uint32_t max_abs4(uint32_t m, const uint4& v) {
+    return max_abs_bf16x2(max_abs_bf16x2(m, v.x), max_abs_bf16x2(v.y, max_abs_bf16x2(v.z, v.w)));
+}
+
+#ifndef TFQ_QUANT_SEG
+#define TFQ_QUANT_SEG 16  // 16-byte units per lane per segment (a warp moves 32 * 16 * 16 B = 8 KiB)
+#endif
+
+template <bool kInt8, bool kClamp, bool kIeeeDiv, int SEG>
+__device__ __forceinline__ void quantize_segment(const uint4 (&v)[SEG], uint2* qrow, int base, int lane, int units,
+                                                 float sc, float rcp, float qmax) {
+#pragma unroll
+    for (int j = 0; j < SEG; ++j) {
+        const int idx = base + lane + 32 * j;
+        if (idx < units) qrow[idx] = quantize8<kInt8, kClamp, kIeeeDiv>(v[j], sc, rcp, qmax);
+    }
+}
+
+template <int SEG>
+__device__ __forceinline__ void load_segment(uint4 (&v)[SEG], const uint4* row, int base, int lane, int units,
+                                             uint64_t policy) {
+#pragma unroll
+    for (int j = 0; j < SEG; ++j) {
+        const int idx = base + lane + 32 * j;
+#if TFQ_QUANT_L2_KEEP
+        v[j] = idx < units ? ldg_nc_v4_policy(row + idx, policy) : make_uint4(0u, 0u, 0u, 0u);
+#else
+        v[j] = idx < units ? ldg_nc_v4(row + idx) : make_uint4(0u, 0u, 0u, 0u);
+#endif
+    }
 }
 
 template <bool kInt8, bool kClamp>
-__global__ void __launch_bounds__(kThreads) quant_rows_kernel(const uint16_t* __restrict__ x, int64_t M, int K,
-                                                              float qmax, uint8_t* __restrict__ q,
-                                                              float* __restrict__ s, QuantConfig cfg,
-                                                              uint32_t* err) {
-    extern __shared__ __align__(128) uint8_t smem[];
-    const int S = cfg.stages;
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + static_cast<size_t>(S) * cfg.stage_bytes);
-    uint64_t* empty = full + S;
-    uint64_t* team_bar = empty + S;                               // one per row slot
-    float* red = reinterpret_cast<float*>(team_bar + kComputeWarps);  // [2][8]
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(red + 2 * kComputeWarps);
-
-    const int warp = threadIdx.x >> 5;
+__global__ void __launch_bounds__(256) quant_rows_kernel(const uint4* __restrict__ x, int64_t M, int K,
+                                                                float qmax, uint8_t* __restrict__ q,
+                                                                float* __restrict__ s) {
+    constexpr int SEG = TFQ_QUANT_SEG;
     const int lane = threadIdx.x & 31;
-    const int R = cfg.rows_per_stage;
-    const int G = cfg.warps_per_row;
-    const int64_t n_groups = (M + R - 1) / R;
-    const uint32_t row_bytes = 2u * static_cast<uint32_t>(K);
-
-    if (threadIdx.x == 0) {
-        for (int i = 0; i < S; ++i) {
-            mbar_init(&full[i], 1);
-            mbar_init(&empty[i], kComputeWarps);
-        }
-        for (int i = 0; i < kComputeWarps; ++i) mbar_init(&team_bar[i], G);
-        *abort_flag = 0;
-        fence_mbar_init();
-    }
-    __syncthreads();
-
-    if (warp == kComputeWarps) {
-        // ------------------------------------------------------- producer
-        if (lane != 0) return;
-        int issued_phase[8];
-        for (int i = 0; i < 8; ++i) issued_phase[i] = -1;
-        int it = 0;
-        for (int64_t g = blockIdx.x; g < n_groups; g += gridDim.x, ++it) {
-            const int st = it % S;
-            const uint32_t ph = static_cast<uint32_t>(it / S) & 1u;
-            if (!mbar_wait(&empty[st], ph ^ 1u, abort_flag)) {
-                record_failure(abort_flag, err, kErrQuantProducer);
-                break;
-            }
-            const int64_t r0 = g * R;
-            const uint32_t rows = static_cast<uint32_t>(min(static_cast<int64_t>(R), M - r0));
-            const uint32_t bytes = rows * row_bytes;
-            mbar_arrive_expect_tx(&full[st], bytes);
-            const uint8_t* src = reinterpret_cast<const uint8_t*>(x + r0 * K);
-            uint8_t* dst = smem + static_cast<size_t>(st) * cfg.stage_bytes;
-            for (uint32_t off = 0; off < bytes; off += kBulkPiece)
-                bulk_g2s(dst + off, src + off, min(kBulkPiece, bytes - off), &full[st]);
-            issued_phase[st] = static_cast<int>(ph);
-        }
-        // Every copy this thread issued must land before the CTA may exit
-        // (on the normal path they already have, or soon will).
-        for (int i = 0; i < S; ++i) {
-            if (issued_phase[i] >= 0 && !mbar_wait(&full[i], static_cast<uint32_t>(issued_phase[i]), nullptr))
-                atomicOr(err, kErrQuantProducer);
-        }
-        return;
-    }
-
-    // ------------------------------------------------------------ consumers
-    const int slot = warp / G;
-    const int nslots = kComputeWarps / G;
-    const int tr = (warp % G) * 32 + lane;  // index within the row team
-    const int team = G * 32;
-    const int units = K / 8;                // 16-byte units of 8 bf16
-    uint32_t team_uses = 0;
-    int it = 0;
-    for (int64_t g = blockIdx.x; g < n_groups; g += gridDim.x, ++it) {
-        const int st = it % S;
-        const uint32_t ph = static_cast<uint32_t>(it / S) & 1u;
-        if (!mbar_wait_warp(&full[st], ph, abort_flag)) {
-            if (lane == 0) record_failure(abort_flag, err, kErrQuantConsumer);
-            break;
-        }
-        const int64_t r0 = g * R;
-        const int rows = static_cast<int>(min(static_cast<int64_t>(R), M - r0));
-        const uint8_t* stage = smem + static_cast<size_t>(st) * cfg.stage_bytes;
-        bool ok = true;
-        for (int r = slot; r < rows; r += nslots) {
-            const uint4* row = reinterpret_cast<const uint4*>(stage + static_cast<size_t>(r) * row_bytes);
-            // pass 1: max |x| (bf16 magnitudes, packed)
-            uint32_t m2 = 0, m3 = 0;
-#pragma unroll 4
-            for (int u = tr; u < units; u += team) {
-                const uint4 v = row[u];
-                m2 = max_abs_bf16x2(m2, v.x);
-                m3 = max_abs_bf16x2(m3, v.y);
-                m2 = max_abs_bf16x2(m2, v.z);
-                m3 = max_abs_bf16x2(m3, v.w);
-            }
-            m2 = max_abs_bf16x2(m2, m3) & 0x7FFF7FFFu;
-            float amax = fmaxf(bf16_lo(m2), bf16_hi(m2));
+    const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+    const int units = K >> 3;  // 16-byte units of 8 bf16 per row
+    const bool one_segment = units <= 32 * SEG;
+    const uint64_t keep = l2_policy_evict_last(), drop = l2_policy_evict_first();
+    for (int64_t r = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; r < M; r += nwarps) {
+        const uint4* row = x + r * units;
+        uint4 v[SEG];
+        // pass 1: max |x|, a whole segment of loads in flight per warp
+        uint32_t m = 0;
+        for (int base = 0; base < units; base += 32 * SEG) {
+            load_segment<SEG>(v, row, base, lane, units, one_segment ? drop : keep);
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
-            if (G > 1) {
-                float* red_buf = red + (team_uses & 1u) * kComputeWarps;
-                if (lane == 0) {
-                    red_buf[warp] = amax;
-                    mbar_arrive(&team_bar[slot]);
-                }
-                __syncwarp();
-                if (!mbar_wait_warp(&team_bar[slot], team_uses & 1u, abort_flag)) {
-                    if (lane == 0) record_failure(abort_flag, err, kErrQuantConsumer);
-                    ok = false;
-                    break;
-                }
-                amax = red_buf[slot * G];
-                for (int j = 1; j < G; ++j) amax = fmaxf(amax, red_buf[slot * G + j]);
-                ++team_uses;
-            }
-            const float sc = __fdiv_rn(fmaxf(amax, 1e-12f), qmax);
-            const float rcp = __frcp_rn(sc);
-            const int64_t grow = r0 + r;
-            if (tr == 0) s[grow] = sc;
-            // pass 2: quantize and store (8 bytes per thread, 256 B per warp)
-            uint2* qrow = reinterpret_cast<uint2*>(q + grow * K);
-            if (sc <= 0x1p125f) {
-#pragma unroll 2
-                for (int u = tr; u < units; u += team)
-                    qrow[u] = quantize8<kInt8, kClamp, false>(row[u], sc, rcp, qmax);
-            } else {  // reciprocal would be subnormal: IEEE division (row-uniform branch)
-                for (int u = tr; u < units; u += team)
-                    qrow[u] = quantize8<kInt8, kClamp, true>(row[u], sc, rcp, qmax);
-            }
+            for (int j = 0; j < SEG; ++j) m = max_abs4(m, v[j]);
         }
-        if (!ok) break;
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[st]);
+        m &= 0x7FFF7FFFu;
+        float amax = fmaxf(bf16_lo(m), bf16_hi(m));
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+        const float sc = __fdiv_rn(fmaxf(amax, 1e-12f), qmax);
+        const float rcp = __frcp_rn(sc);
+        if (lane == 0) s[r] = sc;
+        uint2* qrow = reinterpret_cast<uint2*>(q + r * K);
+        // pass 2: a row of one segment is still in registers; longer rows are
+        // read again (from L2: the same row was read microseconds earlier)
+        if (sc <= 0x1p125f) {
+            if (one_segment) {
+                quantize_segment<kInt8, kClamp, false, SEG>(v, qrow, 0, lane, units, sc, rcp, qmax);
+            } else {
+                for (int base = 0; base < units; base += 32 * SEG) {
+                    load_segment<SEG>(v, row, base, lane, units, drop);
+                    quantize_segment<kInt8, kClamp, false, SEG>(v, qrow, base, lane, units, sc, rcp, qmax);
+                }
+            }
+        } else {  // reciprocal would be subnormal: IEEE division (warp-uniform branch)
+            for (int u = lane; u < units; u += 32)
+                qrow[u] = quantize8<kInt8, kClamp, true>(ldg_nc_v4(row + u), sc, rcp, qmax);
+        }
     }
 }
 
@@ -354,23 +299,14 @@ tfq_status launch_quant_rows(const void* x, int64_t rows, int64_t K, float qmax,
         const cudaError_t e = cudaGetLastError();
         return e == cudaSuccess ? TFQ_OK : fail(TFQ_ECUDA, "quantizer launch: %s", cudaGetErrorString(e));
     }
-    const QuantConfig cfg = choose_config(K);
     const bool clamp = !out_int8 && !is_e4m3_value(qmax);
     auto kernel = out_int8 ? quant_rows_kernel<true, false>
                            : (clamp ? quant_rows_kernel<false, true> : quant_rows_kernel<false, false>);
-    const int kidx = out_int8 ? 2 : (clamp ? 1 : 0);
-    if (!ds->quant_attr_set[kidx]) {
-        const cudaError_t e =
-            cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
-        if (e != cudaSuccess) return fail(TFQ_ECUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
-        ds->quant_attr_set[kidx] = true;
-    }
-    const int64_t n_groups = (rows + cfg.rows_per_stage - 1) / cfg.rows_per_stage;
-    const int per_sm = std::max(1, static_cast<int>((228u * 1024u) / (cfg.smem_bytes + 1024u)));
-    const int64_t grid = std::min<int64_t>(n_groups, static_cast<int64_t>(ds->sm_count) * std::min(per_sm, TFQ_QUANT_CTAS_PER_SM));
-    kernel<<<static_cast<unsigned>(grid), kThreads, cfg.smem_bytes, stream>>>(
-        static_cast<const uint16_t*>(x), rows, static_cast<int>(K), qmax, static_cast<uint8_t*>(q), s, cfg,
-        ds->err_word);
+    const int threads = 256;  // 8 warps, one row per warp at a time
+    const int64_t blocks = std::min<int64_t>((rows + 7) / 8, static_cast<int64_t>(ds->sm_count) * kCtasPerSm);
+    kernel<<<static_cast<unsigned>(blocks), threads, 0, stream>>>(static_cast<const uint4*>(x), rows,
+                                                                 static_cast<int>(K), qmax,
+                                                                 static_cast<uint8_t*>(q), s);
     const cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? TFQ_OK : fail(TFQ_ECUDA, "quantizer launch: %s", cudaGetErrorString(e));
 }

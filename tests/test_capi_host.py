@@ -65,7 +65,7 @@ ALIGNED = 0x10000  # a fake, 16-byte aligned address: never dereferenced by a re
     ((ALIGNED, 4, 32, 448.0, ALIGNED, None, None), _capi.TFQ_EINVAL),           # null s
     ((ALIGNED + 8, 4, 32, 448.0, ALIGNED, ALIGNED, None), _capi.TFQ_EINVAL),    # misaligned
     ((ALIGNED, -1, 32, 448.0, ALIGNED, ALIGNED, None), _capi.TFQ_EINVAL),
-    ((ALIGNED, 4, 32768 + 16, 448.0, ALIGNED, ALIGNED, None), _capi.TFQ_EUNSUPPORTED),
+    ((ALIGNED, 4, (1 << 24) + 16, 448.0, ALIGNED, ALIGNED, None), _capi.TFQ_EUNSUPPORTED),
     ((ALIGNED, 0, 32, 448.0, None, None, None), _capi.TFQ_OK),                  # M == 0: no-op
 ])
 def test_quant_act_validation(lib, args, status):

@@ -34,7 +34,7 @@ def test_tiny_config_activation():
 
 @pytest.mark.parametrize("qmax", [448.0, 14.0, 7.0, 21.0, 100.0, 12.0])
 @pytest.mark.parametrize("M,K", [(1, 16), (3, 48), (37, 256), (129, 1024), (65, 3072), (33, 5120),
-                                 (17, 12288), (9, 13824), (5, 32768), (300, 160)])
+                                 (17, 12288), (9, 13824), (5, 32768), (300, 160), (3, 65536), (2, 100000)])
 def test_ragged_shapes(M, K, qmax):
     """qmax 21 and 100 are not E4M3 numbers (21 is the midpoint of 20 and
     22): the kernel clamps x/s there; for the others it needs no clamp."""
