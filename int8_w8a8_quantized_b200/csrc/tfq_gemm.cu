@@ -54,7 +54,10 @@ constexpr int TMEM_COLS = 2 * BN;                    // double-buffered accumula
 constexpr int GROUP_M = 16;
 
 constexpr size_t SMEM_RING = static_cast<size_t>(STAGES) * (A_STAGE_BYTES + B_STAGE_BYTES);
-constexpr size_t SMEM_EPI = static_cast<size_t>(EPI_WARPS) * 2 * EPI_BUF_BYTES;
+// Per epilogue warp: one output staging buffer and a copy of the tile's
+// column scales and bias (fp32, 2 x BN floats).
+constexpr size_t COLP_BYTES = 2 * BN * sizeof(float);
+constexpr size_t SMEM_EPI = static_cast<size_t>(EPI_WARPS) * (EPI_BUF_BYTES + COLP_BYTES);
 constexpr size_t SMEM_BARS = (2 * STAGES + 4 + 1) * 8 + 16;
 constexpr size_t SMEM_BYTES = 1024 /* alignment slack */ + SMEM_RING + SMEM_EPI + SMEM_BARS;
 static_assert(SMEM_BYTES <= 232448, "shared memory budget exceeded");
@@ -110,15 +113,47 @@ __device__ __forceinline__ void give_up(volatile int* abort_flag, uint32_t* err,
     atomicOr(err, bit);
 }
 
+// Copies s_w[n] and bias[n] (as fp32; 0 past N or without bias) for the
+// tile's kBN columns starting at n_tile0 into this warp's buffer colp
+// (s_w at colp[0..kBN), bias at colp[kBN..2 kBN)).  Called while the MMA of
+// the tile is still running, so the global-load latency is off the path.
+template <int kBN>
+__device__ __forceinline__ void stage_col_params(const GemmArgs& p, float* colp, int n_tile0, int lane) {
+    __syncwarp();  // the previous tile's reads of colp are done
+    for (int g = lane; g < kBN / 8; g += 32) {
+        const int n = n_tile0 + g * 8;
+        float4 w0 = make_float4(0.f, 0.f, 0.f, 0.f), w1 = w0, b0 = w0, b1 = w0;
+        if (n < p.N) {  // N % 8 == 0: a group of 8 columns is all valid or all out
+            w0 = __ldg(reinterpret_cast<const float4*>(p.s_w + n));
+            w1 = __ldg(reinterpret_cast<const float4*>(p.s_w + n + 4));
+            if (p.bias != nullptr) {
+                const uint4 bv = __ldg(reinterpret_cast<const uint4*>(p.bias + n));
+                b0 = make_float4(__uint_as_float(bv.x << 16), __uint_as_float(bv.x & 0xFFFF0000u),
+                                 __uint_as_float(bv.y << 16), __uint_as_float(bv.y & 0xFFFF0000u));
+                b1 = make_float4(__uint_as_float(bv.z << 16), __uint_as_float(bv.z & 0xFFFF0000u),
+                                 __uint_as_float(bv.w << 16), __uint_as_float(bv.w & 0xFFFF0000u));
+            }
+        }
+        float4* cw = reinterpret_cast<float4*>(colp + g * 8);
+        float4* cb = reinterpret_cast<float4*>(colp + kBN + g * 8);
+        cw[0] = w0;
+        cw[1] = w1;
+        cb[0] = b0;
+        cb[1] = b1;
+    }
+    __syncwarp();
+}
+
 // Epilogue of one 32-row slice of a finished tile: TMEM -> registers ->
-// y = acc * s_a[m] * s_w[n] + bias[n] in fp32 -> bf16 -> 128-byte swizzled
-// staging buffer -> TMA store, EPI_COLS columns at a time.  `t_row` is the
-// TMEM address of this warp's 32 lanes at the tile's first column; `chunk`
-// counts stores of this warp (selects the staging buffer).
+// y = acc * s_a[m] * s_w[n] + bias[n] in fp32 (packed fp32x2 operations) ->
+// bf16 -> 128-byte swizzled staging buffer -> TMA store, EPI_COLS columns
+// at a time.  `t_row` is the TMEM address of this warp's 32 lanes at the
+// tile's first column; colp holds the tile's column scales and bias.
 template <int kBN, bool kI8>
 __device__ __forceinline__ void store_tile_rows(const GemmArgs& p, const CUtensorMap& tmY, uint32_t t_row,
-                                                uint8_t* ebuf0, int& chunk, int n_tile0, int row0, float sa,
+                                                uint8_t* ebuf, const float* colp, int n_tile0, int row0, float sa,
                                                 int lane) {
+    const float2 sa2 = make_float2(sa, sa);
 #pragma unroll 1
     for (int c = 0; c < kBN / EPI_COLS; ++c) {
         const int n0 = n_tile0 + c * EPI_COLS;
@@ -127,50 +162,37 @@ __device__ __forceinline__ void store_tile_rows(const GemmArgs& p, const CUtenso
         tmem_ld_32x32b_x32(t_row + c * EPI_COLS, acc[0]);
         tmem_ld_32x32b_x32(t_row + c * EPI_COLS + 32, acc[1]);
         tmem_ld_wait();
-        uint8_t* ebuf = ebuf0 + (chunk & 1) * EPI_BUF_BYTES;
-        // The staging buffer written two chunks ago must have been read by its TMA store.
-        if (lane == 0) bulk_wait_read<1>();
-        __syncwarp();
+        uint32_t packed[2][16];
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
 #pragma unroll
-            for (int g = 0; g < 4; ++g) {  // 8 columns -> one 16-byte unit
-                const int nl = h * 32 + g * 8;
-                float sw[8], bb[8];
-                if (n0 + nl < p.N) {  // N % 8 == 0: a group is all valid or all out
-                    const float4 w0 = __ldg(reinterpret_cast<const float4*>(p.s_w + n0 + nl));
-                    const float4 w1 = __ldg(reinterpret_cast<const float4*>(p.s_w + n0 + nl + 4));
-                    sw[0] = w0.x; sw[1] = w0.y; sw[2] = w0.z; sw[3] = w0.w;
-                    sw[4] = w1.x; sw[5] = w1.y; sw[6] = w1.z; sw[7] = w1.w;
-                    if (p.bias != nullptr) {
-                        const uint4 bv = __ldg(reinterpret_cast<const uint4*>(p.bias + n0 + nl));
-                        const uint32_t bw[4] = {bv.x, bv.y, bv.z, bv.w};
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            bb[2 * j] = __uint_as_float(bw[j] << 16);
-                            bb[2 * j + 1] = __uint_as_float(bw[j] & 0xFFFF0000u);
-                        }
-                    } else {
-#pragma unroll
-                        for (int j = 0; j < 8; ++j) bb[j] = 0.0f;
-                    }
-                } else {
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) sw[j] = bb[j] = 0.0f;
-                }
-                uint32_t packed[4];
+            for (int g = 0; g < 4; ++g) {  // 8 columns
+                const int nl = c * EPI_COLS + h * 32 + g * 8;
+                const float4 w0 = *reinterpret_cast<const float4*>(colp + nl);
+                const float4 w1 = *reinterpret_cast<const float4*>(colp + nl + 4);
+                const float4 b0 = *reinterpret_cast<const float4*>(colp + kBN + nl);
+                const float4 b1 = *reinterpret_cast<const float4*>(colp + kBN + nl + 4);
+                const float2 sw[4] = {make_float2(w0.x, w0.y), make_float2(w0.z, w0.w), make_float2(w1.x, w1.y),
+                                      make_float2(w1.z, w1.w)};
+                const float2 bb[4] = {make_float2(b0.x, b0.y), make_float2(b0.z, b0.w), make_float2(b1.x, b1.y),
+                                      make_float2(b1.z, b1.w)};
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
-                    const float y0 = fmaf(acc_value<kI8>(acc[h][g * 8 + 2 * j]) * sa, sw[2 * j], bb[2 * j]);
-                    const float y1 =
-                        fmaf(acc_value<kI8>(acc[h][g * 8 + 2 * j + 1]) * sa, sw[2 * j + 1], bb[2 * j + 1]);
-                    packed[j] = pack_bf16x2(y0, y1);
+                    const float2 a2 = make_float2(acc_value<kI8>(acc[h][g * 8 + 2 * j]),
+                                                  acc_value<kI8>(acc[h][g * 8 + 2 * j + 1]));
+                    const float2 y = __ffma2_rn(__fmul2_rn(a2, sa2), sw[j], bb[j]);
+                    packed[h][g * 4 + j] = pack_bf16x2(y.x, y.y);
                 }
-                // 128-byte swizzle: 16-byte unit u of row r lives at unit u ^ (r % 8).
-                const int unit = h * 4 + g;
-                uint4* dst = reinterpret_cast<uint4*>(ebuf + lane * 128 + ((unit ^ (lane & 7)) << 4));
-                *dst = make_uint4(packed[0], packed[1], packed[2], packed[3]);
             }
+        }
+        // The staging buffer's previous TMA store must have finished reading it.
+        if (lane == 0) bulk_wait_read<0>();
+        __syncwarp();
+#pragma unroll
+        for (int unit = 0; unit < 8; ++unit) {  // 128-byte swizzle: unit u of row r at u ^ (r % 8)
+            uint4* dst = reinterpret_cast<uint4*>(ebuf + lane * 128 + ((unit ^ (lane & 7)) << 4));
+            const uint32_t* w = &packed[unit >> 2][(unit & 3) * 4];
+            *dst = make_uint4(w[0], w[1], w[2], w[3]);
         }
         fence_proxy_async_smem();
         __syncwarp();
@@ -178,7 +200,6 @@ __device__ __forceinline__ void store_tile_rows(const GemmArgs& p, const CUtenso
             tma_store_2d(&tmY, ebuf, n0, row0);
             bulk_commit();
         }
-        ++chunk;
     }
 }
 
@@ -301,11 +322,13 @@ __global__ void __launch_bounds__(THREADS, 1)
         // -------------------------------------------------------- epilogue
         const int ew = warp - 2;         // 0..3: staging buffers
         const int quarter = warp & 3;    // TMEM lanes this warp may read
-        uint8_t* ebuf0 = sE + static_cast<size_t>(ew) * 2 * EPI_BUF_BYTES;
-        int tcount = 0, chunk = 0;
+        uint8_t* ebuf = sE + static_cast<size_t>(ew) * EPI_BUF_BYTES;
+        float* colp = reinterpret_cast<float*>(sE + EPI_WARPS * EPI_BUF_BYTES + ew * COLP_BYTES);
+        int tcount = 0;
         for (int t = blockIdx.x; t < total_tiles; t += gridDim.x, ++tcount) {
             int tm, tn;
             tile_coords(t, p, tm, tn);
+            stage_col_params<BN>(p, colp, tn * BN, lane);
             const int buf = tcount & 1;
             const uint32_t use = static_cast<uint32_t>(tcount >> 1);
             if (!mbar_wait_warp(&tmem_full[buf], use & 1u, abort_flag)) {
@@ -318,7 +341,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             const float sa = (m < p.M) ? __ldg(p.s_a + m) : 0.0f;
             const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
                                    static_cast<uint32_t>(buf * BN);
-            store_tile_rows<BN, kI8>(p, tmY, t_row, ebuf0, chunk, tn * BN, row0, sa, lane);
+            store_tile_rows<BN, kI8>(p, tmY, t_row, ebuf, colp, tn * BN, row0, sa, lane);
             // All of this warp's TMEM reads of `buf` are complete: hand it back.
             tc_fence_before();
             __syncwarp();
@@ -507,13 +530,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         // ------------------------------------------- epilogue (both CTAs)
         const int ew = warp - 2;
         const int quarter = warp & 3;
-        uint8_t* ebuf0 = sE + static_cast<size_t>(ew) * 2 * EPI_BUF_BYTES;
+        uint8_t* ebuf = sE + static_cast<size_t>(ew) * EPI_BUF_BYTES;
+        float* colp = reinterpret_cast<float*>(sE + EPI_WARPS * EPI_BUF_BYTES + ew * COLP_BYTES);
         const uint32_t tmem_empty_leader0 = mapa_shared(smem_u32(&tmem_empty[0]), 0);
         const uint32_t tmem_empty_leader1 = mapa_shared(smem_u32(&tmem_empty[1]), 0);
-        int tcount = 0, chunk = 0;
+        int tcount = 0;
         for (int t = cluster; t < total_tiles; t += n_clusters, ++tcount) {
             int tm, tn;
             pair_tile_coords(t, m_tiles, p.n_tiles, tm, tn);
+            stage_col_params<PBN>(p, colp, tn * PBN, lane);
             const int buf = tcount & 1;
             const uint32_t use = static_cast<uint32_t>(tcount >> 1);
             if (!mbar_wait_warp(&tmem_full[buf], use & 1u, abort_flag)) {
@@ -526,7 +551,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             const float sa = (m < p.M) ? __ldg(p.s_a + m) : 0.0f;
             const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
                                    static_cast<uint32_t>(buf * PBN);
-            store_tile_rows<PBN, kI8>(p, tmY, t_row, ebuf0, chunk, tn * PBN, row0, sa, lane);
+            store_tile_rows<PBN, kI8>(p, tmY, t_row, ebuf, colp, tn * PBN, row0, sa, lane);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(buf == 0 ? tmem_empty_leader0 : tmem_empty_leader1);

@@ -75,19 +75,18 @@ __device__ __forceinline__ uint32_t to_int8_byte(float t) {
 // to be normal numbers, which holds for |a| >= 2^-102 and
 // 2^-49 <= b <= 2^125 (every row scale is >= 1e-12 / 448 > 2^-49; rows with
 // a larger scale take the IEEE division instead).  For |a| < 2^-102 the
-// quotient is below 2^-53 in magnitude, so only its sign reaches the codes;
-// the final copysign keeps it, also for a = +-0.  Five FMA-pipe
-// instructions, no branch.  Checked against the IEEE division __fdiv_rn by
+// quotient is below 2^-53 in magnitude, so only its sign reaches the codes
+// (a = -0 may give +0 here; the caller restores the sign, see quantize8).
+// Five packed fp32x2 instructions (sm_100: two IEEE round-to-nearest
+// operations each, exactly the scalar ones) per pair of elements, no
+// branch; nb = -b.  Checked against the IEEE division __fdiv_rn by
 // tfq_selftest_div_rn.
-__device__ __forceinline__ float div_rn_from_rcp_unsigned_zero(float a, float b, float y) {
-    const float q0 = __fmul_rn(a, y);
-    const float r0 = __fmaf_rn(-q0, b, a);
-    const float q1 = __fmaf_rn(r0, y, q0);
-    const float r1 = __fmaf_rn(-q1, b, a);
-    return __fmaf_rn(r1, y, q1);
-}
-__device__ __forceinline__ float div_rn_from_rcp(float a, float b, float y) {
-    return copysignf(div_rn_from_rcp_unsigned_zero(a, b, y), a);
+__device__ __forceinline__ float2 div2_rn_from_rcp_unsigned_zero(float2 a, float2 nb, float2 y) {
+    const float2 q0 = __fmul2_rn(a, y);
+    const float2 r0 = __ffma2_rn(q0, nb, a);
+    const float2 q1 = __ffma2_rn(r0, y, q0);
+    const float2 r1 = __ffma2_rn(q1, nb, a);
+    return __ffma2_rn(r1, y, q1);
 }
 
 namespace {
@@ -110,8 +109,10 @@ __device__ __forceinline__ uint32_t quantize2(uint32_t w, float sc, float rcp, f
         a = __fdiv_rn(bf16_lo(w), sc);
         b = __fdiv_rn(bf16_hi(w), sc);
     } else {
-        a = div_rn_from_rcp_unsigned_zero(bf16_lo(w), sc, rcp);
-        b = div_rn_from_rcp_unsigned_zero(bf16_hi(w), sc, rcp);
+        const float2 t = div2_rn_from_rcp_unsigned_zero(make_float2(bf16_lo(w), bf16_hi(w)), make_float2(-sc, -sc),
+                                                       make_float2(rcp, rcp));
+        a = t.x;
+        b = t.y;
     }
     if constexpr (kInt8) {
         return to_int8_byte(a) | (to_int8_byte(b) << 8);
@@ -258,7 +259,11 @@ __global__ void div_selftest_kernel(const float* __restrict__ a, const float* __
     for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
          i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
         const float x = a[i], y = b[i];
-        ours[i] = div_rn_from_rcp(x, y, __frcp_rn(y));
+        const float r = __frcp_rn(y);
+        // the packed form the quantizers use; both lanes carry the same
+        // quotient, the sign of a zero result is restored as the quantizers do
+        const float2 t = div2_rn_from_rcp_unsigned_zero(make_float2(x, x), make_float2(-y, -y), make_float2(r, r));
+        ours[i] = copysignf(t.y, x);
         ieee[i] = __fdiv_rn(x, y);
     }
 }
