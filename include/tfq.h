@@ -202,6 +202,17 @@ TFQ_API tfq_status tfq_selftest_div_rn(const float *a, const float *b, int64_t n
                                        void *stream);
 
 /*
+ * Self-check of the failure path: launches one tiny kernel whose only wait
+ * is on a barrier that never completes, with the bounded-wait helper every
+ * kernel here uses but a limit of limit_us microseconds (1 <= limit_us <=
+ * 10^7) instead of the kernels' seconds.  The wait runs out, the kernel
+ * records it in the device error word and returns; the next
+ * tfq_device_error() then reports TFQ_ETIMEOUT and clears the word, and
+ * the CUDA context stays usable.  Errors: TFQ_EINVAL (limit out of range).
+ */
+TFQ_API tfq_status tfq_selftest_wait_timeout(uint32_t limit_us, void *stream);
+
+/*
  * Synchronizes `stream`, then reads and clears the current device's error
  * word.  Returns TFQ_ETIMEOUT if a bounded wait inside a kernel ran out
  * since the last call (the outputs of that launch are then incomplete),

@@ -36,6 +36,7 @@ SIGNATURES = {
     "tfq_scaled_int8_linear": (_I, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _P]),
     "tfq_scaled_fp8_linear_noalloc": (_I, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _P]),
     "tfq_selftest_div_rn": (_I, [_P, _P, _I64, _P, _P, _P]),
+    "tfq_selftest_wait_timeout": (_I, [ctypes.c_uint32, _P]),
     "tfq_device_error": (_I, [_P]),
     "tfq_status_string": (ctypes.c_char_p, [_I]),
     "tfq_last_error_message": (ctypes.c_char_p, []),

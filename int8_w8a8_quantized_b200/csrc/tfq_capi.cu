@@ -229,6 +229,14 @@ tfq_status tfq_selftest_div_rn(const float* a, const float* b, int64_t n, float*
     return launch_div_selftest(a, b, n, ours, ieee, static_cast<cudaStream_t>(stream));
 }
 
+tfq_status tfq_selftest_wait_timeout(uint32_t limit_us, void* stream) {
+    if (limit_us < 1 || limit_us > 10000000u) return fail(TFQ_EINVAL, "limit_us=%u outside [1, 1e7]", limit_us);
+    tfq_status st;
+    DeviceState* ds = current_device_state(&st);
+    if (ds == nullptr) return st;
+    return launch_wait_selftest(static_cast<uint64_t>(limit_us) * 1000u, static_cast<cudaStream_t>(stream), ds);
+}
+
 tfq_status tfq_device_error(void* stream) {
     tfq_status st;
     DeviceState* ds = current_device_state(&st);

@@ -51,7 +51,6 @@ constexpr int EPI_COLS = 64;                         // bf16 columns per TMA sto
 constexpr int EPI_BUF_BYTES = 32 * EPI_COLS * 2;     // 4 KiB per staging buffer
 constexpr int THREADS = 64 + EPI_WARPS * 32;         // producer warp, MMA warp, epilogue warps
 constexpr int TMEM_COLS = 2 * BN;                    // double-buffered accumulator
-constexpr int GROUP_M = 16;
 
 constexpr size_t SMEM_RING = static_cast<size_t>(STAGES) * (A_STAGE_BYTES + B_STAGE_BYTES);
 // Per epilogue warp: one output staging buffer and a copy of the tile's
@@ -78,14 +77,32 @@ struct GemmArgs {
     const uint16_t* bias;  // may be null
     int M, N, K;
     int m_tiles, n_tiles, k_blocks;
+    // Tile order.  band_n > 0: bands of band_n consecutive N tiles; each band
+    // sweeps every M tile (N fastest inside the band), so the band's weight
+    // panels are reused by the whole sweep (kept in L2: evict_last) and the
+    // activation panels stream (evict_first), re-read once per band.
+    // band_n == 0: groups of group_m consecutive M tiles, each sweeping every
+    // N tile (M fastest inside the group): activations kept, weights stream.
+    int band_n;
+    int group_m;
     uint32_t* err;
 };
 
 __device__ __forceinline__ void tile_coords(int t, const GemmArgs& p, int& tm, int& tn) {
-    const int per_group = GROUP_M * p.n_tiles;
+    if (p.band_n > 0) {
+        const int per_band = p.band_n * p.m_tiles;
+        const int bid = t / per_band;
+        const int first_n = bid * p.band_n;
+        const int gsize = min(p.n_tiles - first_n, p.band_n);
+        const int r = t - bid * per_band;
+        tn = first_n + r % gsize;
+        tm = r / gsize;
+        return;
+    }
+    const int per_group = p.group_m * p.n_tiles;
     const int gid = t / per_group;
-    const int first_m = gid * GROUP_M;
-    const int gsize = min(p.m_tiles - first_m, GROUP_M);
+    const int first_m = gid * p.group_m;
+    const int gsize = min(p.m_tiles - first_m, p.group_m);
     const int r = t - gid * per_group;
     tm = first_m + r % gsize;
     tn = r / gsize;
@@ -144,6 +161,32 @@ __device__ __forceinline__ void stage_col_params(const GemmArgs& p, float* colp,
     __syncwarp();
 }
 
+#ifndef TFQ_GEMM_POLICY_A
+#define TFQ_GEMM_POLICY_A 0  // L2 policy of activation loads in N bands: 0 first, 1 normal, 2 last
+#endif
+#ifndef TFQ_GEMM_POLICY_B
+#define TFQ_GEMM_POLICY_B 2  // L2 policy of weight loads in N bands: 0 first, 1 normal, 2 last
+#endif
+
+__device__ __forceinline__ uint64_t l2_policy(int kind) {
+    return kind == 2 ? make_l2_policy_evict_last()
+                     : (kind == 1 ? make_l2_policy_evict_normal() : make_l2_policy_evict_first());
+}
+
+// L2 policies of the operand loads: in N bands the band's weight panels are
+// reused by the whole M sweep and are kept; the activation panels are reused
+// only by the band's N tiles running at about the same time.  In M groups
+// the roles swap.
+__device__ __forceinline__ void l2_policies(const GemmArgs& p, uint64_t& pol_a, uint64_t& pol_b) {
+    if (p.band_n > 0) {
+        pol_a = l2_policy(TFQ_GEMM_POLICY_A);
+        pol_b = l2_policy(TFQ_GEMM_POLICY_B);
+    } else {
+        pol_a = make_l2_policy_evict_last();
+        pol_b = make_l2_policy_evict_normal();
+    }
+}
+
 // Epilogue of one 32-row slice of a finished tile: TMEM -> registers ->
 // y = acc * s_a[m] * s_w[n] + bias[n] in fp32 (packed fp32x2 operations) ->
 // bf16 -> 128-byte swizzled staging buffer -> TMA store, EPI_COLS columns
@@ -154,6 +197,7 @@ __device__ __forceinline__ void store_tile_rows(const GemmArgs& p, const CUtenso
                                                 uint8_t* ebuf, const float* colp, int n_tile0, int row0, float sa,
                                                 int lane) {
     const float2 sa2 = make_float2(sa, sa);
+    const uint64_t y_policy = make_l2_policy_evict_first();
 #pragma unroll 1
     for (int c = 0; c < kBN / EPI_COLS; ++c) {
         const int n0 = n_tile0 + c * EPI_COLS;
@@ -197,7 +241,7 @@ __device__ __forceinline__ void store_tile_rows(const GemmArgs& p, const CUtenso
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
-            tma_store_2d(&tmY, ebuf, n0, row0);
+            tma_store_2d_hint(&tmY, ebuf, n0, row0, y_policy);  // the output streams out of L2
             bulk_commit();
         }
     }
@@ -252,6 +296,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (warp == 0) {
         // ---------------------------------------------------- TMA producer
         if (lane == 0) {
+            uint64_t pol_a, pol_b;
+            l2_policies(p, pol_a, pol_b);
             int it = 0;
             int issued_phase[STAGES];
             for (int i = 0; i < STAGES; ++i) issued_phase[i] = -1;
@@ -268,8 +314,8 @@ __global__ void __launch_bounds__(THREADS, 1)
                         break;
                     }
                     mbar_arrive_expect_tx(&full[st], A_STAGE_BYTES + B_STAGE_BYTES);
-                    tma_load_2d(sA + st * A_STAGE_BYTES, &tmA, kb * BK, tm * BM, &full[st]);
-                    tma_load_2d(sB + st * B_STAGE_BYTES, &tmB, kb * BK, tn * BN, &full[st]);
+                    tma_load_2d_hint(sA + st * A_STAGE_BYTES, &tmA, kb * BK, tm * BM, &full[st], pol_a);
+                    tma_load_2d_hint(sB + st * B_STAGE_BYTES, &tmB, kb * BK, tn * BN, &full[st], pol_b);
                     issued_phase[st] = static_cast<int>(ph);
                 }
             }
@@ -375,7 +421,6 @@ __global__ void __launch_bounds__(THREADS, 1)
 // commit; both CTAs' epilogue warps hand the accumulator back on the even
 // CTA's "tmem_empty" barrier.  The epilogue is the same as above.
 constexpr int PAIR_STAGES = 6;
-constexpr int PAIR_GROUP_M = 8;  // pair tiles per M group (2048 rows)
 
 template <int PBN>
 struct PairCfg {
@@ -390,11 +435,22 @@ struct PairCfg {
     static_assert(PBN % 64 == 0 && PBN >= 64 && PBN <= 256, "N tile");
 };
 
-__device__ __forceinline__ void pair_tile_coords(int t, int m_tiles, int n_tiles, int& tm, int& tn) {
-    const int per_group = PAIR_GROUP_M * n_tiles;
+__device__ __forceinline__ void pair_tile_coords(int t, int m_tiles, int n_tiles, int group_m, int band_n, int& tm,
+                                                 int& tn) {
+    if (band_n > 0) {
+        const int per_band = band_n * m_tiles;
+        const int bid = t / per_band;
+        const int first_n = bid * band_n;
+        const int gsize = min(n_tiles - first_n, band_n);
+        const int r = t - bid * per_band;
+        tn = first_n + r % gsize;
+        tm = r / gsize;
+        return;
+    }
+    const int per_group = group_m * n_tiles;
     const int gid = t / per_group;
-    const int first_m = gid * PAIR_GROUP_M;
-    const int gsize = min(m_tiles - first_m, PAIR_GROUP_M);
+    const int first_m = gid * group_m;
+    const int gsize = min(m_tiles - first_m, group_m);
     const int r = t - gid * per_group;
     tm = first_m + r % gsize;
     tn = r / gsize;
@@ -454,13 +510,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     if (warp == 0) {
         // ---------------------------------------------------- TMA producer
         if (lane == 0) {
+            uint64_t pol_a, pol_b;
+            l2_policies(p, pol_a, pol_b);
             int it = 0;
             int issued_phase[PAIR_STAGES];
             for (int i = 0; i < PAIR_STAGES; ++i) issued_phase[i] = -1;
             bool ok = true;
             for (int t = cluster; t < total_tiles && ok; t += n_clusters) {
                 int tm, tn;
-                pair_tile_coords(t, m_tiles, p.n_tiles, tm, tn);
+                pair_tile_coords(t, m_tiles, p.n_tiles, p.group_m, p.band_n, tm, tn);
                 const int a_row = tm * 256 + static_cast<int>(rank) * 128;
                 const int b_row = tn * PBN + static_cast<int>(rank) * C::kBHalf;
                 for (int kb = 0; kb < p.k_blocks; ++kb, ++it) {
@@ -473,8 +531,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                     }
                     const uint32_t full_leader = mapa_shared(smem_u32(&full[st]), 0);
                     if (rank == 0) mbar_arrive_expect_tx(&full[st], 2 * (C::kAStage + C::kBStage));
-                    tma_load_2d_pair(sA + st * C::kAStage, &tmA, kb * BK, a_row, full_leader);
-                    tma_load_2d_pair(sB + st * C::kBStage, &tmB, kb * BK, b_row, full_leader);
+                    tma_load_2d_pair(sA + st * C::kAStage, &tmA, kb * BK, a_row, full_leader, pol_a);
+                    tma_load_2d_pair(sB + st * C::kBStage, &tmB, kb * BK, b_row, full_leader, pol_b);
                     issued_phase[st] = static_cast<int>(ph);
                 }
             }
@@ -537,7 +595,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         int tcount = 0;
         for (int t = cluster; t < total_tiles; t += n_clusters, ++tcount) {
             int tm, tn;
-            pair_tile_coords(t, m_tiles, p.n_tiles, tm, tn);
+            pair_tile_coords(t, m_tiles, p.n_tiles, p.group_m, p.band_n, tm, tn);
             stage_col_params<PBN>(p, colp, tn * PBN, lane);
             const int buf = tcount & 1;
             const uint32_t use = static_cast<uint32_t>(tcount >> 1);
@@ -576,9 +634,42 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
 
 bool use_pair_kernel(int64_t M, int sm_count) { return M >= TFQ_GEMM_PAIR_MIN_M && sm_count >= 2; }
 
+#ifndef TFQ_GEMM_BAND_MB
+#define TFQ_GEMM_BAND_MB 40     // > 0: N bands holding about this many MB of weight; 0: M groups
+#endif
+#ifndef TFQ_GEMM_GROUP_M
+#define TFQ_GEMM_GROUP_M 8
+#endif
+
+// Raster order (see GemmArgs): N bands whose weight panels total about
+// TFQ_GEMM_BAND_MB, or M groups of TFQ_GEMM_GROUP_M tiles.
+void choose_raster(int64_t K, int bn, int& band_n, int& group_m) {
+    group_m = TFQ_GEMM_GROUP_M;
+    band_n = 0;
+    if (TFQ_GEMM_BAND_MB > 0) {
+        const int64_t panel = static_cast<int64_t>(bn) * K;  // bytes of one N tile's weight panel
+        band_n = static_cast<int>(std::max<int64_t>(1, static_cast<int64_t>(TFQ_GEMM_BAND_MB) * 1000000 / panel));
+    }
+}
+
 }  // namespace
 
 namespace {
+
+// A wait that can only end by running out: the barrier expects one arrival
+// that nothing makes.  Exercises the bounded wait the GEMM roles use (same
+// helper, a shorter limit) and the error word that reports it.
+__global__ void wait_selftest_kernel(uint64_t limit_ns, uint32_t* err) {
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0 && !mbar_wait(&bar, 0, &abort_flag, limit_ns)) atomicOr(err, kErrSelfTest);
+}
 
 template <bool kI8>
 tfq_status launch_scaled_mm(const void* A, const float* s_a, const void* W, const float* s_w, const void* bias,
@@ -611,6 +702,7 @@ tfq_status launch_scaled_mm(const void* A, const float* s_a, const void* W, cons
     a.m_tiles = static_cast<int>((M + BM - 1) / BM);
     a.n_tiles = static_cast<int>((N + BN - 1) / BN);
     a.k_blocks = static_cast<int>((K + BK - 1) / BK);
+    choose_raster(K, use_pair_kernel(M, ds->sm_count) ? 256 : BN, a.band_n, a.group_m);
     a.err = ds->err_word;
     const int64_t tiles = static_cast<int64_t>(a.m_tiles) * a.n_tiles;
     if (tiles > INT32_MAX) return fail(TFQ_EUNSUPPORTED, "too many output tiles");
@@ -635,6 +727,12 @@ tfq_status launch_scaled_mm(const void* A, const float* s_a, const void* W, cons
 }
 
 }  // namespace
+
+tfq_status launch_wait_selftest(uint64_t limit_ns, cudaStream_t stream, DeviceState* ds) {
+    wait_selftest_kernel<<<1, 32, 0, stream>>>(limit_ns, ds->err_word);
+    const cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? TFQ_OK : fail(TFQ_ECUDA, "self-test launch: %s", cudaGetErrorString(e));
+}
 
 tfq_status launch_scaled_fp8_gemm(const void* A, const float* s_a, const void* W, const float* s_w,
                                   const void* bias, int64_t M, int64_t N, int64_t K, void* out,

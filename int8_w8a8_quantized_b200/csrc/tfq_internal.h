@@ -16,6 +16,7 @@ enum : uint32_t {
     kErrGemmMma = 1u << 5,
     kErrGemmEpilogue = 1u << 6,
     kErrGemmDrain = 1u << 7,
+    kErrSelfTest = 1u << 8,
 };
 
 struct DeviceState {
@@ -52,6 +53,9 @@ tfq_status launch_quant_rows(const void* x, int64_t rows, int64_t K, float qmax,
 // Self-check: the quantizer's division next to the IEEE division.
 tfq_status launch_div_selftest(const float* a, const float* b, int64_t n, float* ours, float* ieee,
                                cudaStream_t stream);
+
+// Self-check of the bounded wait: a wait on a barrier that never completes.
+tfq_status launch_wait_selftest(uint64_t limit_ns, cudaStream_t stream, DeviceState* ds);
 
 // Scaled FP8 GEMM with the fused scale/bias/BF16 epilogue.
 tfq_status launch_scaled_fp8_gemm(const void* A, const float* s_a, const void* W, const float* s_w,

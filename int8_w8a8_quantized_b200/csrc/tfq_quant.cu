@@ -193,6 +193,16 @@ __device__ __forceinline__ void quantize_segment(const uint4 (&v)[SEG], uint2* q
     }
 }
 
+// Returns the row's L2 lines to normal eviction priority once pass 2 is done
+// with them, so that the evict_last marks of pass 1 do not outlive the row
+// and crowd the next kernel's working set out of L2.
+__device__ __forceinline__ void release_row_l2(const uint4* row, int units, int lane) {
+    const char* base = reinterpret_cast<const char*>(row);
+    const int lines = (units * 16 + 127) / 128;
+    for (int l = lane; l < lines; l += 32)
+        asm volatile("applypriority.global.L2::evict_normal [%0], 128;" ::"l"(base + 128 * l) : "memory");
+}
+
 template <int SEG>
 __device__ __forceinline__ void load_segment(uint4 (&v)[SEG], const uint4* row, int base, int lane, int units,
                                              uint64_t policy) {
@@ -250,6 +260,9 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(const uint4* __restrict
             for (int u = lane; u < units; u += 32)
                 qrow[u] = quantize8<kInt8, kClamp, true>(ldg_nc_v4(row + u), sc, rcp, qmax);
         }
+#if TFQ_QUANT_L2_KEEP
+        if (!one_segment) release_row_l2(row, units, lane);
+#endif
     }
 }
 

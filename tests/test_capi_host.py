@@ -108,3 +108,8 @@ def test_valid_call_without_gpu_fails_loudly(lib):
     assert st in (_capi.TFQ_ECUDA, _capi.TFQ_EUNSUPPORTED)
     assert lib.tfq_scaled_fp8_linear(ALIGNED, ALIGNED, ALIGNED, ALIGNED, None, 4, 16, 32, ALIGNED, None) \
         in (_capi.TFQ_ECUDA, _capi.TFQ_EUNSUPPORTED)
+
+
+def test_wait_selftest_rejects_bad_limits_before_any_launch(lib):
+    assert lib.tfq_selftest_wait_timeout(0, None) == _capi.TFQ_EINVAL
+    assert lib.tfq_selftest_wait_timeout(10_000_001, None) == _capi.TFQ_EINVAL
