@@ -64,6 +64,36 @@ def parse_args():
     return ap.parse_args()
 
 
+KERNEL_SOURCES = {
+    "gemm": ("int8_w8a8_quantized_b200/csrc/tfq_gemm.cu", "int8_w8a8_quantized_b200/csrc/tfq_ptx.cuh"),
+    "quant": ("int8_w8a8_quantized_b200/csrc/tfq_quant.cu", "int8_w8a8_quantized_b200/csrc/tfq_ptx.cuh"),
+}
+TRAFFIC_RECORD = os.path.join(ROOT, "profiles", "roofline_traffic_video_dit_block.md")
+
+
+def recorded_traffic(kind: str, workload: str, dtype: str):
+    """DRAM bytes per launch from the committed ncu capture, or None when the
+    capture is for another workload or the kernel sources changed since."""
+    import hashlib
+    try:
+        kv = {}
+        for line in open(TRAFFIC_RECORD, encoding="utf-8"):
+            if " = " in line:
+                k, v = line.strip().split(" = ", 1)
+                kv[k] = v
+        if kv.get("workload") != workload or kv.get("dtype") != dtype:
+            return None
+        m = hashlib.sha256()
+        for f in KERNEL_SOURCES[kind]:
+            with open(os.path.join(ROOT, f), "rb") as fh:
+                m.update(fh.read())
+        if m.hexdigest() != kv.get(f"{kind}.sources_sha256"):
+            return None
+        return float(kv[f"{kind}.traffic_bytes_per_launch"])
+    except (OSError, KeyError, ValueError):
+        return None
+
+
 def measured_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -255,10 +285,11 @@ def gpu_arm(args, wl, rank, world, local_rank):
     gemm_ms = [a.elapsed_time(b) for a, b, _ in ev["gemm"]]
     quant_ms = [a.elapsed_time(b) for a, b, _ in ev["quant"]]
     gemm_flops = [2 * m * n * k for _, _, (m, n, k) in ev["gemm"]]
+    gemm_bytes = [m * k + n * k + 2 * m * n + 4 * m + 6 * n for _, _, (m, n, k) in ev["gemm"]]
     quant_bytes = [nbytes for _, _, nbytes in ev["quant"]]
     out = {
         "ms_per_step": ms_per_step,
-        "gemm_ms_total": sum(gemm_ms), "gemm_flops_total": sum(gemm_flops),
+        "gemm_ms_total": sum(gemm_ms), "gemm_flops_total": sum(gemm_flops), "gemm_bytes_total": sum(gemm_bytes),
         "quant_ms_total": sum(quant_ms), "quant_bytes_total": sum(quant_bytes),
         "gemm_launches": len(gemm_ms), "quant_launches": len(quant_ms),
         "gpu_launches": launches[0], "clocks": clk,
@@ -452,7 +483,8 @@ def main():
             "peak": round(fp8_peak, 1),
             "unit": "TFLOP/s" if args.dtype == "fp8" else "TOPS",
             "frac": round(gemm_tflops / fp8_peak, 4),
-            "traffic": None,
+            "traffic": recorded_traffic("gemm", wl.name, args.dtype),
+            "algorithmic_bytes_per_launch": round(res["gemm_bytes_total"] / max(1, res["gemm_launches"])),
             "peak_source": f"{peak_src} bf16 sustained x {FP8_OVER_BF16} (nominal fp8|int8 / bf16 dense ratio)",
             "frac_of_burst_peak": round(gemm_tflops / (bf16_burst * FP8_OVER_BF16), 4),
             "avg_launch_ms": round(gemm_avg_ms, 4),
@@ -466,6 +498,8 @@ def main():
             "unit": "GB/s",
             "frac": None if quant_gbs is None else round(quant_gbs / peaks.get("hbm_gbs", FALLBACK_HBM_GBS), 4),
             "share_of_step": round(res["quant_ms_total"] / (res["ms_per_step"] * args.steps), 4),
+            "traffic": recorded_traffic("quant", wl.name, args.dtype),
+            "algorithmic_bytes_per_launch": round(res["quant_bytes_total"] / max(1, res["quant_launches"])),
         },
         "per_linear_ms": {k: round(statistics.median(v), 4) for k, v in res["per_linear"].items()},
         "gpu_launches": res["gpu_launches"],
