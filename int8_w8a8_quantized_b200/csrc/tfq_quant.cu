@@ -266,6 +266,39 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(const uint4* __restrict
     }
 }
 
+// Short rows (K <= 128, e.g. one head_dim vector of a KV cache): a warp
+// holds 32 / LPR rows, LPR lanes per row and one 16-byte unit per lane, so
+// no lane idles; the max reduction stays inside each LPR-lane group.
+template <bool kInt8, bool kClamp, int LPR>
+__global__ void __launch_bounds__(256) quant_short_rows_kernel(const uint4* __restrict__ x, int64_t M, int K,
+                                                               float qmax, uint8_t* __restrict__ q,
+                                                               float* __restrict__ s) {
+    constexpr int RPW = 32 / LPR;  // rows per warp
+    const int lane = threadIdx.x & 31;
+    const int sub = lane % LPR;
+    const int units = K >> 3;      // <= LPR
+    const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+    for (int64_t base = warp * RPW; base < M; base += nwarps * RPW) {
+        const int64_t r = base + lane / LPR;
+        const bool active = r < M && sub < units;
+        const uint4 v = active ? ldg_nc_v4(x + r * units + sub) : make_uint4(0u, 0u, 0u, 0u);
+        uint32_t m = max_abs4(0u, v) & 0x7FFF7FFFu;
+        float amax = fmaxf(bf16_lo(m), bf16_hi(m));
+#pragma unroll
+        for (int o = LPR / 2; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+        const float sc = __fdiv_rn(fmaxf(amax, 1e-12f), qmax);
+        if (r < M) {
+            if (sub == 0) s[r] = sc;
+            if (active) {
+                uint2* qrow = reinterpret_cast<uint2*>(q + r * K);
+                qrow[sub] = sc <= 0x1p125f ? quantize8<kInt8, kClamp, false>(v, sc, __frcp_rn(sc), qmax)
+                                           : quantize8<kInt8, kClamp, true>(v, sc, 0.0f, qmax);
+            }
+        }
+    }
+}
+
 // Element-wise self-check of div_rn_from_rcp against the IEEE division.
 __global__ void div_selftest_kernel(const float* __restrict__ a, const float* __restrict__ b, int64_t n,
                                     float* __restrict__ ours, float* __restrict__ ieee) {
@@ -295,6 +328,30 @@ bool is_e4m3_value(float v) {
     return v >= 0x1p-6f && v <= 448.0f && m == std::floor(m);
 }
 
+template <int LPR>
+void launch_short_rows_lpr(const void* x, int64_t rows, int64_t K, float qmax, bool out_int8, bool clamp, void* q,
+                           float* s, cudaStream_t stream, int64_t blocks) {
+    auto kernel = out_int8 ? quant_short_rows_kernel<true, false, LPR>
+                           : (clamp ? quant_short_rows_kernel<false, true, LPR> : quant_short_rows_kernel<false, false, LPR>);
+    kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(static_cast<const uint4*>(x), rows, static_cast<int>(K),
+                                                               qmax, static_cast<uint8_t*>(q), s);
+}
+
+tfq_status launch_short_rows(const void* x, int64_t rows, int64_t K, float qmax, bool out_int8, bool clamp, int lpr,
+                             void* q, float* s, cudaStream_t stream, DeviceState* ds) {
+    const int64_t rows_per_block = 8 * (32 / lpr);
+    const int64_t blocks = std::min<int64_t>((rows + rows_per_block - 1) / rows_per_block,
+                                             static_cast<int64_t>(ds->sm_count) * 8);
+    switch (lpr) {
+        case 2: launch_short_rows_lpr<2>(x, rows, K, qmax, out_int8, clamp, q, s, stream, blocks); break;
+        case 4: launch_short_rows_lpr<4>(x, rows, K, qmax, out_int8, clamp, q, s, stream, blocks); break;
+        case 8: launch_short_rows_lpr<8>(x, rows, K, qmax, out_int8, clamp, q, s, stream, blocks); break;
+        default: launch_short_rows_lpr<16>(x, rows, K, qmax, out_int8, clamp, q, s, stream, blocks); break;
+    }
+    const cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? TFQ_OK : fail(TFQ_ECUDA, "quantizer launch: %s", cudaGetErrorString(e));
+}
+
 }  // namespace
 
 tfq_status launch_div_selftest(const float* a, const float* b, int64_t n, float* ours, float* ieee,
@@ -318,6 +375,11 @@ tfq_status launch_quant_rows(const void* x, int64_t rows, int64_t K, float qmax,
         return e == cudaSuccess ? TFQ_OK : fail(TFQ_ECUDA, "quantizer launch: %s", cudaGetErrorString(e));
     }
     const bool clamp = !out_int8 && !is_e4m3_value(qmax);
+    if (K <= 128) {
+        const int units = static_cast<int>(K / 8);
+        const int lpr = units <= 2 ? 2 : units <= 4 ? 4 : units <= 8 ? 8 : 16;
+        return launch_short_rows(x, rows, K, qmax, out_int8, clamp, lpr, q, s, stream, ds);
+    }
     auto kernel = out_int8 ? quant_rows_kernel<true, false>
                            : (clamp ? quant_rows_kernel<false, true> : quant_rows_kernel<false, false>);
     const int threads = 256;  // 8 warps, one row per warp at a time

@@ -141,3 +141,27 @@ def test_tensor_wrappers_match_raw():
     q2, s2 = tfq_quant_act_fp8_per_token(x, 14.0)
     torch.cuda.synchronize()
     assert torch.equal(q1, q2) and torch.equal(s1, s2)
+
+
+@pytest.mark.parametrize("K", [16, 32, 48, 64, 96, 112, 128])
+@pytest.mark.parametrize("M", [1, 3, 37, 1000, 4097])
+def test_short_rows_sub_warp(M, K):
+    """K <= 128 runs the sub-warp kernel (2..16 lanes per row, several rows per
+    warp): ragged M, lanes beyond the row's units, FP8 with and without the
+    clamp, INT8."""
+    x = workloads.activations(M, K, seed=M + K, nu=3, outlier_cols=1, outlier_mult=25.0,
+                              zero_rows=1 if M > 2 else 0, device="cuda")
+    for qmax in (448.0, 21.0):
+        _assert_fp8_equal(x, qmax)
+    q, s = _gpu.quant_weight(x, _capi.TFQ_DTYPE_INT8, 127.0)
+    q_ref, s_ref = _gpu.oracle_quant_int8(x, 127.0)
+    np.testing.assert_array_equal(s.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
+    np.testing.assert_array_equal(q.cpu().numpy().view(np.int8), q_ref)
+
+
+def test_kv_cache_per_vector_full_size():
+    """Per-vector FP8 KV cache: one fp32 scale per head_dim vector -- the video
+    DiT's K projection viewed as [75600 tokens x 40 heads, 128]; sampled rows."""
+    x = workloads.activations(75600 * 40, 128, seed=77, nu=4, device="cuda")
+    rows = _gpu.sample_rows(x.shape[0], 4096, seed=78)
+    _assert_fp8_equal(x, 448.0, rows)
