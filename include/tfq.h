@@ -149,6 +149,21 @@ TFQ_API tfq_status tfq_scaled_int8_linear(const void *A_q, const float *s_a, con
                                           int64_t K, void *out_bf16, void *stream);
 
 /*
+ * tfq_scaled_fp8_linear_f16acc: tfq_scaled_fp8_linear with the products
+ * accumulated in FP16 on the tensor cores instead of FP32 (the fp8-f16-accum
+ * mode of the LightX2V "模型量化技术" page, quantization-mode table and
+ * section "MiniMax-H3 FP8 FP16 累加"); the accumulator is widened to fp32 for
+ * the epilogue.  A partial sum beyond +-65504 becomes +-inf and the output
+ * element is then non-finite: that page lowers the activation qmax (14 or 7)
+ * to keep the accumulator in range.  The result carries FP16 rounding of the
+ * partial sums, so it is not held to tfq_scaled_fp8_linear's tolerance.
+ * Same arguments, preconditions and errors as tfq_scaled_fp8_linear.
+ */
+TFQ_API tfq_status tfq_scaled_fp8_linear_f16acc(const void *A_q, const float *s_a, const void *W_q,
+                                                const float *s_w, const void *bias_bf16, int64_t M, int64_t N,
+                                                int64_t K, void *out_bf16, void *stream);
+
+/*
  * Bytes of the static device array used by tfq_scaled_fp8_linear_noalloc.
  * Every GPU that loads the library holds this array until the process exits.
  */

@@ -34,6 +34,7 @@ SIGNATURES = {
     "tfq_scaled_fp8_linear": (_I, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _P]),
     "tfq_quant_act_int8_per_token": (_I, [_P, _I64, _I64, _F, _P, _P, _P]),
     "tfq_scaled_int8_linear": (_I, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _P]),
+    "tfq_scaled_fp8_linear_f16acc": (_I, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _P]),
     "tfq_scaled_fp8_linear_noalloc": (_I, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _P]),
     "tfq_selftest_div_rn": (_I, [_P, _P, _I64, _P, _P, _P]),
     "tfq_selftest_wait_timeout": (_I, [ctypes.c_uint32, _P]),

@@ -197,6 +197,17 @@ tfq_status tfq_scaled_int8_linear(const void* A_q, const float* s_a, const void*
                                    static_cast<cudaStream_t>(stream), ds);
 }
 
+tfq_status tfq_scaled_fp8_linear_f16acc(const void* A_q, const float* s_a, const void* W_q, const float* s_w,
+                                        const void* bias_bf16, int64_t M, int64_t N, int64_t K, void* out_bf16,
+                                        void* stream) {
+    tfq_status st = check_gemm_args(A_q, s_a, W_q, s_w, bias_bf16, M, N, K, out_bf16);
+    if (st != TFQ_OK || M == 0 || N == 0) return st;
+    DeviceState* ds = current_device_state(&st);
+    if (ds == nullptr) return st;
+    return launch_scaled_fp8_gemm_f16acc(A_q, s_a, W_q, s_w, bias_bf16, M, N, K, out_bf16,
+                                         static_cast<cudaStream_t>(stream), ds);
+}
+
 tfq_status tfq_scaled_fp8_linear(const void* A_q, const float* s_a, const void* W_q, const float* s_w,
                                  const void* bias_bf16, int64_t M, int64_t N, int64_t K, void* out_bf16,
                                  void* stream) {

@@ -30,6 +30,7 @@
 // the error word, drains its own outstanding copies and MMAs, frees TMEM and
 // returns.
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include <algorithm>
 
@@ -65,10 +66,15 @@ static_assert(SMEM_BYTES <= 232448, "shared memory budget exceeded");
 // (1 = F32 for kind::f8f6f4, 2 = S32 for kind::i8), A and B formats in bits
 // 7-9 and 10-12 (E4M3 = 0 for f8f6f4; signed 8-bit = 1 for i8), both
 // K-major (bits 15, 16 = 0), N >> 3 in bits 17-22, M >> 4 in bits 24-28.
-template <bool kI8>
+// Accumulator kinds: F32 (E4M3 x E4M3, kind::f8f6f4), S32 (S8 x S8,
+// kind::i8), F16 (E4M3 x E4M3 with a half-precision accumulator).
+enum : int { kAccF32 = 0, kAccS32 = 1, kAccF16 = 2 };
+
+template <int kAcc>
 constexpr uint32_t make_idesc(int m, int n) {
-    return (kI8 ? (2u << 4) | (1u << 7) | (1u << 10) : (1u << 4)) | (static_cast<uint32_t>(n >> 3) << 17) |
-           (static_cast<uint32_t>(m >> 4) << 24);
+    const uint32_t fmt = kAcc == kAccS32 ? (2u << 4) | (1u << 7) | (1u << 10)
+                                         : (kAcc == kAccF16 ? 0u : (1u << 4));
+    return fmt | (static_cast<uint32_t>(n >> 3) << 17) | (static_cast<uint32_t>(m >> 4) << 24);
 }
 
 struct GemmArgs {
@@ -114,12 +120,15 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return d;
 }
 
-// An accumulator word as fp32: the F32 accumulator as is, the S32 one
-// converted (round to nearest).
-template <bool kI8>
+// An accumulator word (one 32-bit TMEM column) as fp32: the F32 accumulator
+// as is, the S32 one converted (round to nearest), the F16 one from the low
+// half of its column.
+template <int kAcc>
 __device__ __forceinline__ float acc_value(uint32_t w) {
-    if constexpr (kI8) {
+    if constexpr (kAcc == kAccS32) {
         return __int2float_rn(static_cast<int>(w));
+    } else if constexpr (kAcc == kAccF16) {
+        return __half2float(__ushort_as_half(static_cast<unsigned short>(w & 0xFFFFu)));
     } else {
         return __uint_as_float(w);
     }
@@ -192,7 +201,7 @@ __device__ __forceinline__ void l2_policies(const GemmArgs& p, uint64_t& pol_a, 
 // bf16 -> 128-byte swizzled staging buffer -> TMA store, EPI_COLS columns
 // at a time.  `t_row` is the TMEM address of this warp's 32 lanes at the
 // tile's first column; colp holds the tile's column scales and bias.
-template <int kBN, bool kI8>
+template <int kBN, int kAcc>
 __device__ __forceinline__ void store_tile_rows(const GemmArgs& p, const CUtensorMap& tmY, uint32_t t_row,
                                                 uint8_t* ebuf, const float* colp, int n_tile0, int row0, float sa,
                                                 int lane) {
@@ -222,8 +231,8 @@ __device__ __forceinline__ void store_tile_rows(const GemmArgs& p, const CUtenso
                                       make_float2(b1.z, b1.w)};
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
-                    const float2 a2 = make_float2(acc_value<kI8>(acc[h][g * 8 + 2 * j]),
-                                                  acc_value<kI8>(acc[h][g * 8 + 2 * j + 1]));
+                    const float2 a2 = make_float2(acc_value<kAcc>(acc[h][g * 8 + 2 * j]),
+                                                  acc_value<kAcc>(acc[h][g * 8 + 2 * j + 1]));
                     const float2 y = __ffma2_rn(__fmul2_rn(a2, sa2), sw[j], bb[j]);
                     packed[h][g * 4 + j] = pack_bf16x2(y.x, y.y);
                 }
@@ -247,7 +256,7 @@ __device__ __forceinline__ void store_tile_rows(const GemmArgs& p, const CUtenso
     }
 }
 
-template <bool kI8>
+template <int kAcc>
 __global__ void __launch_bounds__(THREADS, 1)
     scaled_mm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                            const __grid_constant__ CUtensorMap tmY, GemmArgs p) {
@@ -353,7 +362,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                     for (int k = 0; k < BK / UMMA_K; ++k) {
                         // advance the start address by k * 32 bytes inside the swizzle atom
                         const uint64_t koff = static_cast<uint64_t>((k * UMMA_K) >> 4);
-                        mma_e4m3<kI8>(d_tmem, a_desc + koff, b_desc + koff, make_idesc<kI8>(BM, BN),
+                        mma_e4m3<kAcc == kAccS32>(d_tmem, a_desc + koff, b_desc + koff, make_idesc<kAcc>(BM, BN),
                                       (kb | k) != 0 ? 1u : 0u);
                     }
                     mma_commit(&empty[st]);
@@ -387,7 +396,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             const float sa = (m < p.M) ? __ldg(p.s_a + m) : 0.0f;
             const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
                                    static_cast<uint32_t>(buf * BN);
-            store_tile_rows<BN, kI8>(p, tmY, t_row, ebuf, colp, tn * BN, row0, sa, lane);
+            store_tile_rows<BN, kAcc>(p, tmY, t_row, ebuf, colp, tn * BN, row0, sa, lane);
             // All of this warp's TMEM reads of `buf` are complete: hand it back.
             tc_fence_before();
             __syncwarp();
@@ -456,7 +465,7 @@ __device__ __forceinline__ void pair_tile_coords(int t, int m_tiles, int n_tiles
     tn = r / gsize;
 }
 
-template <int PBN, bool kI8>
+template <int PBN, int kAcc>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     scaled_mm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                                 const __grid_constant__ CUtensorMap tmY, GemmArgs p) {
@@ -574,7 +583,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
 #pragma unroll
                     for (int k = 0; k < BK / UMMA_K; ++k) {
                         const uint64_t koff = static_cast<uint64_t>((k * UMMA_K) >> 4);
-                        mma_e4m3_pair<kI8>(d_tmem, a_desc + koff, b_desc + koff, make_idesc<kI8>(256, PBN),
+                        mma_e4m3_pair<kAcc == kAccS32>(d_tmem, a_desc + koff, b_desc + koff, make_idesc<kAcc>(256, PBN),
                                            (kb | k) != 0 ? 1u : 0u);
                     }
                     mma_commit_pair(&empty[st], 0x3);
@@ -609,7 +618,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             const float sa = (m < p.M) ? __ldg(p.s_a + m) : 0.0f;
             const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
                                    static_cast<uint32_t>(buf * PBN);
-            store_tile_rows<PBN, kI8>(p, tmY, t_row, ebuf, colp, tn * PBN, row0, sa, lane);
+            store_tile_rows<PBN, kAcc>(p, tmY, t_row, ebuf, colp, tn * PBN, row0, sa, lane);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(buf == 0 ? tmem_empty_leader0 : tmem_empty_leader1);
@@ -671,7 +680,7 @@ __global__ void wait_selftest_kernel(uint64_t limit_ns, uint32_t* err) {
     if (threadIdx.x == 0 && !mbar_wait(&bar, 0, &abort_flag, limit_ns)) atomicOr(err, kErrSelfTest);
 }
 
-template <bool kI8>
+template <int kAcc>
 tfq_status launch_scaled_mm(const void* A, const float* s_a, const void* W, const float* s_w, const void* bias,
                             int64_t M, int64_t N, int64_t K, void* out, cudaStream_t stream, DeviceState* ds) {
     if (M == 0 || N == 0) return TFQ_OK;
@@ -682,12 +691,12 @@ tfq_status launch_scaled_mm(const void* A, const float* s_a, const void* W, cons
     st = encode_tensor_map_2d(&tmY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, out, N, M, N * 2, EPI_COLS, 32,
                               CU_TENSOR_MAP_SWIZZLE_128B);
     if (st != TFQ_OK) return st;
-    const int attr_idx = kI8 ? 1 : 0;
+    const int attr_idx = kAcc;
     if (!ds->gemm_attr_set[attr_idx]) {
-        cudaError_t e = cudaFuncSetAttribute(scaled_mm_kernel<kI8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaError_t e = cudaFuncSetAttribute(scaled_mm_kernel<kAcc>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              static_cast<int>(SMEM_BYTES));
         if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(scaled_mm_pair_kernel<256, kI8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+            e = cudaFuncSetAttribute(scaled_mm_pair_kernel<256, kAcc>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      static_cast<int>(PairCfg<256>::kSmem));
         if (e != cudaSuccess) return fail(TFQ_ECUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
         ds->gemm_attr_set[attr_idx] = true;
@@ -713,14 +722,14 @@ tfq_status launch_scaled_mm(const void* A, const float* s_a, const void* W, cons
         if (st != TFQ_OK) return st;
         const int64_t pair_tiles = ((M + 255) / 256) * static_cast<int64_t>(a.n_tiles);
         const int clusters = static_cast<int>(std::min<int64_t>(pair_tiles, ds->sm_count / 2));
-        scaled_mm_pair_kernel<256, kI8><<<2 * clusters, THREADS, PairCfg<256>::kSmem, stream>>>(tmA, tmBh, tmY, a);
+        scaled_mm_pair_kernel<256, kAcc><<<2 * clusters, THREADS, PairCfg<256>::kSmem, stream>>>(tmA, tmBh, tmY, a);
     } else {
         CUtensorMap tmB;
         st = encode_tensor_map_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, W, K, N, K, BK, BN,
                                   CU_TENSOR_MAP_SWIZZLE_128B);
         if (st != TFQ_OK) return st;
         const int grid = static_cast<int>(std::min<int64_t>(tiles, ds->sm_count));
-        scaled_mm_kernel<kI8><<<grid, THREADS, SMEM_BYTES, stream>>>(tmA, tmB, tmY, a);
+        scaled_mm_kernel<kAcc><<<grid, THREADS, SMEM_BYTES, stream>>>(tmA, tmB, tmY, a);
     }
     const cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? TFQ_OK : fail(TFQ_ECUDA, "GEMM launch: %s", cudaGetErrorString(e));
@@ -737,13 +746,19 @@ tfq_status launch_wait_selftest(uint64_t limit_ns, cudaStream_t stream, DeviceSt
 tfq_status launch_scaled_fp8_gemm(const void* A, const float* s_a, const void* W, const float* s_w,
                                   const void* bias, int64_t M, int64_t N, int64_t K, void* out,
                                   cudaStream_t stream, DeviceState* ds) {
-    return launch_scaled_mm<false>(A, s_a, W, s_w, bias, M, N, K, out, stream, ds);
+    return launch_scaled_mm<kAccF32>(A, s_a, W, s_w, bias, M, N, K, out, stream, ds);
+}
+
+tfq_status launch_scaled_fp8_gemm_f16acc(const void* A, const float* s_a, const void* W, const float* s_w,
+                                         const void* bias, int64_t M, int64_t N, int64_t K, void* out,
+                                         cudaStream_t stream, DeviceState* ds) {
+    return launch_scaled_mm<kAccF16>(A, s_a, W, s_w, bias, M, N, K, out, stream, ds);
 }
 
 tfq_status launch_scaled_int8_gemm(const void* A, const float* s_a, const void* W, const float* s_w,
                                    const void* bias, int64_t M, int64_t N, int64_t K, void* out,
                                    cudaStream_t stream, DeviceState* ds) {
-    return launch_scaled_mm<true>(A, s_a, W, s_w, bias, M, N, K, out, stream, ds);
+    return launch_scaled_mm<kAccS32>(A, s_a, W, s_w, bias, M, N, K, out, stream, ds);
 }
 
 }  // namespace tfq

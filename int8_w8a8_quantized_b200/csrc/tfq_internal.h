@@ -25,7 +25,7 @@ struct DeviceState {
     int cc_major = 0, cc_minor = 0;
     size_t smem_optin = 0;          // max dynamic shared memory per block
     uint32_t* err_word = nullptr;   // device memory, one 32-bit word
-    bool gemm_attr_set[2] = {false, false};  // FP8, INT8
+    bool gemm_attr_set[3] = {false, false, false};  // FP8, INT8, FP8 with FP16 accumulator
 };
 
 // Per-device state of the current device, created on first use.  Returns
@@ -61,6 +61,11 @@ tfq_status launch_wait_selftest(uint64_t limit_ns, cudaStream_t stream, DeviceSt
 tfq_status launch_scaled_fp8_gemm(const void* A, const float* s_a, const void* W, const float* s_w,
                                   const void* bias, int64_t M, int64_t N, int64_t K, void* out,
                                   cudaStream_t stream, DeviceState* ds);
+
+// Scaled FP8 GEMM with a half-precision (FP16) accumulator.
+tfq_status launch_scaled_fp8_gemm_f16acc(const void* A, const float* s_a, const void* W, const float* s_w,
+                                         const void* bias, int64_t M, int64_t N, int64_t K, void* out,
+                                         cudaStream_t stream, DeviceState* ds);
 
 // Scaled INT8 GEMM (S8 x S8 -> S32 on the tensor cores) with the same epilogue.
 tfq_status launch_scaled_int8_gemm(const void* A, const float* s_a, const void* W, const float* s_w,
