@@ -40,11 +40,15 @@ L2_BYTES = 126 * 1024 * 1024
 
 
 def metric_name(dtype: str) -> str:
-    return METRIC if dtype == "fp8" else METRIC.replace("FP8", "INT8").replace("TFLOP/s", "TOPS")
+    if dtype == "int8":
+        return METRIC.replace("FP8", "INT8").replace("TFLOP/s", "TOPS")
+    if dtype == "fp8_f16acc":
+        return METRIC.replace("scaled-FP8 Linear", "scaled-FP8 Linear (FP16 accumulator)")
+    return METRIC
 
 
 def unit_name(dtype: str) -> str:
-    return "TFLOP/s" if dtype == "fp8" else "TOPS"
+    return "TOPS" if dtype == "int8" else "TFLOP/s"
 
 
 def parse_args():
@@ -55,8 +59,9 @@ def parse_args():
     ap.add_argument("--workload", default="video_dit_block",
                     choices=["video_dit_block", "image_dit_block", "reduced_qmax_ffn_out", "tiny_w8a8_linear"])
     ap.add_argument("--impl", default="tfq", choices=["tfq", "reference"])
-    ap.add_argument("--dtype", default="fp8", choices=["fp8", "int8"],
-                    help="fp8: E4M3 W8A8 (the headline); int8: the INT8 W8A8 path")
+    ap.add_argument("--dtype", default="fp8", choices=["fp8", "int8", "fp8_f16acc"],
+                    help="fp8: E4M3 W8A8 (the headline); int8: the INT8 W8A8 path; "
+                         "fp8_f16acc: E4M3 with an FP16 accumulator")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -185,7 +190,7 @@ def aggregate_throughput(world: int, flops_per_step: int, ms_per_step_max: float
 
 # ------------------------------------------------------------ GPU arm
 def act_qmaxes(wl, dtype):
-    return wl.act_qmax if dtype == "fp8" else (127.0,)
+    return (127.0,) if dtype == "int8" else wl.act_qmax
 
 
 def build_block(wl, dev, dtype="fp8"):
@@ -197,7 +202,8 @@ def build_block(wl, dev, dtype="fp8"):
     lins = []
     for lin in wl.linears:
         w = wl.make_w(lin, device=dev)
-        Wq, sw = tfq_quant_weight_per_channel(w, dtype, 448.0 if dtype == "fp8" else 127.0)
+        wdt = "int8" if dtype == "int8" else "fp8"
+        Wq, sw = tfq_quant_weight_per_channel(w, wdt, 127.0 if dtype == "int8" else 448.0)
         del w
         b = wl.make_bias(lin, device=dev)
         lins.append((lin, Wq, sw, b))
@@ -221,8 +227,9 @@ def gpu_arm(args, wl, rank, world, local_rank):
     sh = int(stream.cuda_stream)
     xs, lins, aq, ys = build_block(wl, dev, args.dtype)
     qmaxes = act_qmaxes(wl, args.dtype)
-    quant_fn = lib.tfq_quant_act_fp8_per_token if args.dtype == "fp8" else lib.tfq_quant_act_int8_per_token
-    gemm_fn = lib.tfq_scaled_fp8_linear if args.dtype == "fp8" else lib.tfq_scaled_int8_linear
+    quant_fn = lib.tfq_quant_act_int8_per_token if args.dtype == "int8" else lib.tfq_quant_act_fp8_per_token
+    gemm_fn = {"fp8": lib.tfq_scaled_fp8_linear, "int8": lib.tfq_scaled_int8_linear,
+               "fp8_f16acc": lib.tfq_scaled_fp8_linear_f16acc}[args.dtype]
 
     # per-kernel events, recorded on the launching stream
     ev = {"quant": [], "gemm": []}
@@ -408,15 +415,15 @@ def oracle_sample(wl, seconds: float, seed: int = 0, dtype: str = "fp8"):
             if key not in cache:
                 w = wl.make_w(lin)
                 wbits = w.contiguous().view(torch.int16).numpy().view(np.uint16)
-                Wq, sw = oracle.quant_rows_fp8(wbits, 448.0) if dtype == "fp8" else oracle.quant_rows_int8(wbits)
+                Wq, sw = oracle.quant_rows_int8(wbits) if dtype == "int8" else oracle.quant_rows_fp8(wbits, 448.0)
                 b = wl.make_bias(lin)
                 bbits = None if b is None else b.contiguous().view(torch.int16).numpy().view(np.uint16)
                 cache[key] = (Wq, sw, bbits)
             Wq, sw, bbits = cache[key]
             x = _x_rows(wl, lin, rows_per_linear, int(rng.integers(1 << 30)))
-            for q in (wl.act_qmax if dtype == "fp8" else (127.0,)):
+            for q in ((127.0,) if dtype == "int8" else wl.act_qmax):
                 t0 = time.perf_counter()
-                if dtype == "fp8":
+                if dtype != "int8":  # the oracle's GEMM accumulates exactly for both FP8 variants
                     A, sa = oracle.quant_rows_fp8(x, q)
                     oracle.scaled_fp8_linear(A, sa, Wq, sw, bbits)
                 else:
@@ -508,7 +515,7 @@ def main():
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "e4m3" if args.dtype == "fp8" else "s8",
+        "dtype": {"fp8": "e4m3", "int8": "s8", "fp8_f16acc": "e4m3 (f16 accumulate)"}[args.dtype],
         "data": "synthetic",
         "config": cfg,
         "roofline": {
@@ -516,7 +523,7 @@ def main():
             "bound": "tensor",
             "achieved": round(gemm_tflops, 1),
             "peak": round(fp8_peak, 1),
-            "unit": "TFLOP/s" if args.dtype == "fp8" else "TOPS",
+            "unit": unit_name(args.dtype),
             "frac": round(gemm_tflops / fp8_peak, 4),
             "traffic": recorded_traffic("gemm", wl.name, args.dtype),
             "algorithmic_bytes_per_launch": round(res["gemm_bytes_total"] / max(1, res["gemm_launches"])),

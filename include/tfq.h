@@ -183,15 +183,18 @@ TFQ_API tfq_status tfq_scaled_fp8_linear_f16acc(const void *A_q, const float *s_
  * of TFQ_NOALLOC_SCRATCH_BYTES bytes, and no call allocates (no cudaMalloc,
  * cudaFree or allocating library routine).
  *  - The caller still owns and passes every input and output.
- *  - A call needs 4 bytes of the array whatever M, N and K; a call needing
- *    more than the array holds is rejected with TFQ_EUNSUPPORTED.
+ *  - A call needs 132 bytes of the array whatever M, N and K (the error
+ *    word and, one 128-byte line further, a counter the kernel's clusters use
+ *    to keep pace); a call needing more than the array holds is rejected with
+ *    TFQ_EUNSUPPORTED.
  *  - The first call on a device does a one-time set-up with that device
  *    current (device checks, cudaGetSymbolAddress of the array, which may
  *    load the library's device code into the context); make that first call
  *    before any stream capture.
  *  - Every call on a device shares the array, which keeps the last call's
- *    contents; each call clears the word on `stream` before its kernel.
- *    Calls that overlap on the GPU (on different streams) race on the word.
+ *    contents; each call clears the error word and the counter on `stream`
+ *    before its kernel.  Calls that overlap on the GPU (on different
+ *    streams) race on both (the counter only paces; results stay correct).
  *  - A bounded wait that runs out is recorded in the array's word only:
  *    this entry point does not read it back (that would need a host
  *    synchronization), and tfq_device_error() does not see it.

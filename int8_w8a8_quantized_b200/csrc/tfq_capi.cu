@@ -71,13 +71,18 @@ DeviceState* current_device_state(tfq_status* st) {
                        prop.minor);
             return nullptr;
         }
+        // One allocation: the error word in the first 128-byte line, then
+        // kRoundSlots round counters, one line each.
+        constexpr int kRoundSlots = 64;
         uint32_t* err_word = nullptr;
-        e = cudaMalloc(&err_word, sizeof(uint32_t));
-        if (e == cudaSuccess) e = cudaMemset(err_word, 0, sizeof(uint32_t));
+        e = cudaMalloc(&err_word, 128 * (1 + kRoundSlots));
+        if (e == cudaSuccess) e = cudaMemset(err_word, 0, 128 * (1 + kRoundSlots));
         if (e != cudaSuccess) {
             *st = fail(TFQ_ECUDA, "allocating the device error word: %s", cudaGetErrorString(e));
             return nullptr;
         }
+        ds->round_ctrs = err_word + 32;
+        ds->round_slots = kRoundSlots;
         tfq_status rs = resolve_encode();
         if (rs != TFQ_OK) {
             *st = rs;
@@ -92,6 +97,14 @@ DeviceState* current_device_state(tfq_status* st) {
     }
     *st = TFQ_OK;
     return ds;
+}
+
+unsigned* take_round_counter(DeviceState* ds) {
+    if (ds->round_ctrs == nullptr || ds->round_slots <= 0) return nullptr;
+    std::lock_guard<std::mutex> lock(g_mutex);
+    const int slot = ds->next_round_slot;
+    ds->next_round_slot = (slot + 1) % ds->round_slots;
+    return ds->round_ctrs + 32 * slot;
 }
 
 tfq_status encode_tensor_map_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, uint64_t inner,

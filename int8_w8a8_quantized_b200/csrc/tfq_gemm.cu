@@ -92,7 +92,31 @@ struct GemmArgs {
     int band_n;
     int group_m;
     uint32_t* err;
+    // Cluster pacing (CTA-pair kernel): zeroed before the launch; the even
+    // CTA's producer adds 1 after issuing each tile's loads and, before its
+    // round r, waits (up to TFQ_PACING_WAIT_NS, then goes on: a performance
+    // hint, not a dependency) until every cluster has issued its rounds
+    // before r.  Keeps the clusters within one tile of each other, so the N
+    // tiles of a band that share an activation panel read it from L2 together
+    // instead of drifting apart and re-reading it from DRAM.  Null: no pacing.
+    unsigned* round_ctr;
 };
+
+#ifndef TFQ_PACING_WAIT_NS
+#define TFQ_PACING_WAIT_NS 200000ull
+#endif
+
+__device__ __forceinline__ void pace_round(const unsigned* ctr, int round, int total_tiles, int n_clusters) {
+    if (ctr == nullptr || round < 1) return;
+    const long long need = min(static_cast<long long>(total_tiles), static_cast<long long>(round) * n_clusters);
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t i = 0; i < TFQ_WAIT_LIMIT_POLLS; ++i) {
+        unsigned v;
+        asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ctr) : "memory");
+        if (static_cast<long long>(v) >= need) return;
+        if (globaltimer_ns() - t0 > TFQ_PACING_WAIT_NS) return;
+    }
+}
 
 __device__ __forceinline__ void tile_coords(int t, const GemmArgs& p, int& tm, int& tn) {
     if (p.band_n > 0) {
@@ -525,7 +549,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             int issued_phase[PAIR_STAGES];
             for (int i = 0; i < PAIR_STAGES; ++i) issued_phase[i] = -1;
             bool ok = true;
-            for (int t = cluster; t < total_tiles && ok; t += n_clusters) {
+            int round = 0;
+            for (int t = cluster; t < total_tiles && ok; t += n_clusters, ++round) {
+                if (rank == 0) pace_round(p.round_ctr, round, total_tiles, n_clusters);
                 int tm, tn;
                 pair_tile_coords(t, m_tiles, p.n_tiles, p.group_m, p.band_n, tm, tn);
                 const int a_row = tm * 256 + static_cast<int>(rank) * 128;
@@ -544,6 +570,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                     tma_load_2d_pair(sB + st * C::kBStage, &tmB, kb * BK, b_row, full_leader, pol_b);
                     issued_phase[st] = static_cast<int>(ph);
                 }
+                if (ok && rank == 0 && p.round_ctr != nullptr) atomicAdd(p.round_ctr, 1u);
             }
             // The even CTA's "full" barriers count both CTAs' loads: the even
             // producer waits for everything in flight before the final
@@ -713,6 +740,7 @@ tfq_status launch_scaled_mm(const void* A, const float* s_a, const void* W, cons
     a.k_blocks = static_cast<int>((K + BK - 1) / BK);
     choose_raster(K, use_pair_kernel(M, ds->sm_count) ? 256 : BN, a.band_n, a.group_m);
     a.err = ds->err_word;
+    a.round_ctr = nullptr;
     const int64_t tiles = static_cast<int64_t>(a.m_tiles) * a.n_tiles;
     if (tiles > INT32_MAX) return fail(TFQ_EUNSUPPORTED, "too many output tiles");
     if (use_pair_kernel(M, ds->sm_count)) {
@@ -722,6 +750,11 @@ tfq_status launch_scaled_mm(const void* A, const float* s_a, const void* W, cons
         if (st != TFQ_OK) return st;
         const int64_t pair_tiles = ((M + 255) / 256) * static_cast<int64_t>(a.n_tiles);
         const int clusters = static_cast<int>(std::min<int64_t>(pair_tiles, ds->sm_count / 2));
+        a.round_ctr = take_round_counter(ds);
+        if (a.round_ctr != nullptr) {
+            const cudaError_t e = cudaMemsetAsync(a.round_ctr, 0, sizeof(unsigned), stream);
+            if (e != cudaSuccess) return fail(TFQ_ECUDA, "clearing the round counter: %s", cudaGetErrorString(e));
+        }
         scaled_mm_pair_kernel<256, kAcc><<<2 * clusters, THREADS, PairCfg<256>::kSmem, stream>>>(tmA, tmBh, tmY, a);
     } else {
         CUtensorMap tmB;

@@ -25,6 +25,12 @@ struct DeviceState {
     int cc_major = 0, cc_minor = 0;
     size_t smem_optin = 0;          // max dynamic shared memory per block
     uint32_t* err_word = nullptr;   // device memory, one 32-bit word
+    // Round counters of the GEMM's cluster pacing (one 128-byte line each);
+    // launches take slots round-robin so that launches in flight at the same
+    // time on different streams do not share one.
+    unsigned* round_ctrs = nullptr;
+    int round_slots = 0;
+    int next_round_slot = 0;
     bool gemm_attr_set[3] = {false, false, false};  // FP8, INT8, FP8 with FP16 accumulator
 };
 
@@ -56,6 +62,9 @@ tfq_status launch_div_selftest(const float* a, const float* b, int64_t n, float*
 
 // Self-check of the bounded wait: a wait on a barrier that never completes.
 tfq_status launch_wait_selftest(uint64_t limit_ns, cudaStream_t stream, DeviceState* ds);
+
+// Round-counter slot for the next GEMM launch on this device (thread safe).
+unsigned* take_round_counter(DeviceState* ds);
 
 // Scaled FP8 GEMM with the fused scale/bias/BF16 epilogue.
 tfq_status launch_scaled_fp8_gemm(const void* A, const float* s_a, const void* W, const float* s_w,

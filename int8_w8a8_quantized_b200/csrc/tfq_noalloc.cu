@@ -3,14 +3,15 @@
 //
 // Who needs it: the regular entry points allocate one small device buffer
 // (the per-device word in which a kernel records that a bounded wait ran
-// out) with cudaMalloc on their first call on a device.  Some callers cannot
-// allow that: a host framework that owns every byte of device memory through
-// its own pool and forbids libraries from calling cudaMalloc, a serving
-// process that reserved nearly all of HBM up front, or code running where a
-// CUDA API call that may synchronize the device is not allowed (for example
-// inside a host callback enqueued on a stream).  This entry point runs the
-// same GEMM kernel, but the word the kernel may write lives in a file-scope
-// __device__ array, so no call allocates anything.
+// out, and the counters the GEMM's clusters use to keep pace) with
+// cudaMalloc on their first call on a device.  Some callers cannot allow
+// that: a host framework that owns every byte of device memory through its
+// own pool and forbids libraries from calling cudaMalloc, a serving process
+// that reserved nearly all of HBM up front, or code running where a CUDA API
+// call that may synchronize the device is not allowed (for example inside a
+// host callback enqueued on a stream).  This entry point runs the same GEMM
+// kernel, but the words the kernel writes live in a file-scope __device__
+// array, so no call allocates anything.
 //
 // The array is part of the library image: every GPU that loads the library
 // holds it until the process exits.
@@ -30,8 +31,9 @@ static_assert(TFQ_NOALLOC_SCRATCH_BYTES % 256 == 0, "scratch size must keep 256-
 // obtained with cudaGetSymbolAddress at set-up.
 static __device__ __align__(256) uint32_t g_noalloc_scratch[TFQ_NOALLOC_SCRATCH_BYTES / sizeof(uint32_t)];
 
-// Scratch the GEMM needs per call: its error word.
-constexpr size_t kGemmScratchBytes = sizeof(uint32_t);
+// Scratch the GEMM needs per call: its error word (first 128-byte line) and
+// the round counter of its cluster pacing (second line).
+constexpr size_t kGemmScratchBytes = 128 + sizeof(unsigned);
 
 constexpr int kMaxDevices = 64;
 std::mutex g_noalloc_mutex;
@@ -81,6 +83,8 @@ DeviceState* noalloc_state(tfq_status* st) {
         ds->cc_major = major;
         ds->cc_minor = minor;
         ds->err_word = ptr;
+        ds->round_ctrs = ptr + 32;  // one slot: calls overlapping on the GPU share it
+        ds->round_slots = 1;
         ds->device = dev;
     }
     *st = TFQ_OK;
@@ -113,8 +117,9 @@ extern "C" tfq_status tfq_scaled_fp8_linear_noalloc(const void* A_q, const float
     DeviceState* ds = noalloc_state(&st);
     if (ds == nullptr) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    // The array keeps the previous call's contents: the error word must start at zero.
-    const cudaError_t e = cudaMemsetAsync(ds->err_word, 0, kGemmScratchBytes, s);
+    // The array keeps the previous call's contents: the error word must start
+    // at zero (the launcher clears the round counter itself).
+    const cudaError_t e = cudaMemsetAsync(ds->err_word, 0, sizeof(uint32_t), s);
     if (e != cudaSuccess) return fail(TFQ_ECUDA, "clearing the scratch word: %s", cudaGetErrorString(e));
     return launch_scaled_fp8_gemm(A_q, s_a, W_q, s_w, bias_bf16, M, N, K, out_bf16, s, ds);
 }
