@@ -11,8 +11,12 @@
 // the symmetric INT8 formula of the TeleFuser page (section "Core ideas").
 // Rows are tokens (activations) or output channels (weights).
 //
-// Design (B200): one warp per row, rows strided over a grid of two CTAs of
-// eight warps per SM; no shared memory, no barriers, no waits.  Pass 1 loads
+// Design (B200): no shared memory, no barriers, no waits.  Rows of
+// K <= 2048 go to a grouped kernel: a power-of-two group of lanes per row,
+// several rows per warp, each lane holding 1, 4 or 8 of the row's 16-byte
+// units, so that a warp keeps kilobytes in flight however short the row.
+// Longer rows: one warp per row, rows strided over a grid of two CTAs of
+// eight warps per SM.  Pass 1 loads
 // a whole segment of the row (16 x 16-byte loads per lane: 8 KiB per warp in
 // flight, a warp reads 512 contiguous bytes per load) and reduces |x| with
 // packed max.xorsign.abs.bf16x2 and shuffles.  Pass 2 quantizes: a row of
@@ -266,34 +270,72 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(const uint4* __restrict
     }
 }
 
-// Short rows (K <= 128, e.g. one head_dim vector of a KV cache): a warp
-// holds 32 / LPR rows, LPR lanes per row and one 16-byte unit per lane, so
-// no lane idles; the max reduction stays inside each LPR-lane group.
-template <bool kInt8, bool kClamp, int LPR>
-__global__ void __launch_bounds__(256) quant_short_rows_kernel(const uint4* __restrict__ x, int64_t M, int K,
-                                                               float qmax, uint8_t* __restrict__ q,
-                                                               float* __restrict__ s) {
+#ifndef TFQ_QUANT_J4_CTAS
+#define TFQ_QUANT_J4_CTAS 4  // resident CTAs of 8 warps per SM for the grouped kernel with 4 units per lane
+#endif
+#ifndef TFQ_QUANT_J8_CTAS
+#define TFQ_QUANT_J8_CTAS 3  // ... with 8 units per lane (~70 registers)
+#endif
+#ifndef TFQ_QUANT_FORCE_J
+#define TFQ_QUANT_FORCE_J 0  // 0: choose units per lane from the row length (1, 4 or 8 to force one)
+#endif
+constexpr int kGroupMaxUnits = 256;  // rows of K <= 2048 take the grouped kernel
+
+template <int J>
+constexpr int grouped_ctas_per_sm() {
+    return J == 1 ? 8 : J == 4 ? TFQ_QUANT_J4_CTAS : TFQ_QUANT_J8_CTAS;
+}
+
+// Short and mid-length rows (K <= 2048: a head_dim vector of a KV cache, the
+// hidden size of a small DiT): LPR lanes share a row, so a warp holds 32 / LPR
+// rows at a time; lane `sub` of a row holds its 16-byte units sub, sub + LPR,
+// sub + 2 LPR, ... (at most J of them).  Each load instruction then reads LPR
+// consecutive units of every row in the warp, all of a row's loads are in
+// flight together, and the max reduction stays inside each LPR-lane group.
+// A one-row-per-warp loop would keep only K * 2 bytes per warp in flight,
+// too little to cover HBM latency for K of a few hundred.
+template <bool kInt8, bool kClamp, int LPR, int J>
+__global__ void __launch_bounds__(256, grouped_ctas_per_sm<J>()) quant_grouped_rows_kernel(const uint4* __restrict__ x, int64_t M, int K,
+                                                                 float qmax, uint8_t* __restrict__ q,
+                                                                 float* __restrict__ s) {
     constexpr int RPW = 32 / LPR;  // rows per warp
     const int lane = threadIdx.x & 31;
     const int sub = lane % LPR;
-    const int units = K >> 3;      // <= LPR
+    const int units = K >> 3;      // <= LPR * J
     const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
     const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
     for (int64_t base = warp * RPW; base < M; base += nwarps * RPW) {
         const int64_t r = base + lane / LPR;
-        const bool active = r < M && sub < units;
-        const uint4 v = active ? ldg_nc_v4(x + r * units + sub) : make_uint4(0u, 0u, 0u, 0u);
-        uint32_t m = max_abs4(0u, v) & 0x7FFF7FFFu;
+        const bool row_ok = r < M;
+        uint4 v[J];
+        uint32_t m = 0;
+#pragma unroll
+        for (int j = 0; j < J; ++j) {
+            const int u = sub + LPR * j;
+            v[j] = (row_ok && u < units) ? ldg_nc_v4(x + r * units + u) : make_uint4(0u, 0u, 0u, 0u);
+            m = max_abs4(m, v[j]);
+        }
+        m &= 0x7FFF7FFFu;
         float amax = fmaxf(bf16_lo(m), bf16_hi(m));
 #pragma unroll
         for (int o = LPR / 2; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
         const float sc = __fdiv_rn(fmaxf(amax, 1e-12f), qmax);
-        if (r < M) {
+        if (row_ok) {
             if (sub == 0) s[r] = sc;
-            if (active) {
-                uint2* qrow = reinterpret_cast<uint2*>(q + r * K);
-                qrow[sub] = sc <= 0x1p125f ? quantize8<kInt8, kClamp, false>(v, sc, __frcp_rn(sc), qmax)
-                                           : quantize8<kInt8, kClamp, true>(v, sc, 0.0f, qmax);
+            uint2* qrow = reinterpret_cast<uint2*>(q + r * K);
+            if (sc <= 0x1p125f) {
+                const float rcp = __frcp_rn(sc);
+#pragma unroll
+                for (int j = 0; j < J; ++j) {
+                    const int u = sub + LPR * j;
+                    if (u < units) qrow[u] = quantize8<kInt8, kClamp, false>(v[j], sc, rcp, qmax);
+                }
+            } else {  // reciprocal would be subnormal: IEEE division for this row
+#pragma unroll
+                for (int j = 0; j < J; ++j) {
+                    const int u = sub + LPR * j;
+                    if (u < units) qrow[u] = quantize8<kInt8, kClamp, true>(v[j], sc, 0.0f, qmax);
+                }
             }
         }
     }
@@ -328,25 +370,67 @@ bool is_e4m3_value(float v) {
     return v >= 0x1p-6f && v <= 448.0f && m == std::floor(m);
 }
 
-template <int LPR>
-void launch_short_rows_lpr(const void* x, int64_t rows, int64_t K, float qmax, bool out_int8, bool clamp, void* q,
-                           float* s, cudaStream_t stream, int64_t blocks) {
-    auto kernel = out_int8 ? quant_short_rows_kernel<true, false, LPR>
-                           : (clamp ? quant_short_rows_kernel<false, true, LPR> : quant_short_rows_kernel<false, false, LPR>);
+template <int LPR, int J>
+void launch_grouped_lpr(const void* x, int64_t rows, int64_t K, float qmax, bool out_int8, bool clamp, void* q,
+                        float* s, cudaStream_t stream, int64_t blocks) {
+    auto kernel = out_int8 ? quant_grouped_rows_kernel<true, false, LPR, J>
+                           : (clamp ? quant_grouped_rows_kernel<false, true, LPR, J>
+                                    : quant_grouped_rows_kernel<false, false, LPR, J>);
     kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(static_cast<const uint4*>(x), rows, static_cast<int>(K),
                                                                qmax, static_cast<uint8_t*>(q), s);
 }
 
-tfq_status launch_short_rows(const void* x, int64_t rows, int64_t K, float qmax, bool out_int8, bool clamp, int lpr,
-                             void* q, float* s, cudaStream_t stream, DeviceState* ds) {
+template <int J>
+void launch_grouped_j(int lpr, const void* x, int64_t rows, int64_t K, float qmax, bool out_int8, bool clamp,
+                      void* q, float* s, cudaStream_t stream, int sm_count) {
     const int64_t rows_per_block = 8 * (32 / lpr);
     const int64_t blocks = std::min<int64_t>((rows + rows_per_block - 1) / rows_per_block,
-                                             static_cast<int64_t>(ds->sm_count) * 8);
+                                             static_cast<int64_t>(sm_count) * grouped_ctas_per_sm<J>());
     switch (lpr) {
-        case 2: launch_short_rows_lpr<2>(x, rows, K, qmax, out_int8, clamp, q, s, stream, blocks); break;
-        case 4: launch_short_rows_lpr<4>(x, rows, K, qmax, out_int8, clamp, q, s, stream, blocks); break;
-        case 8: launch_short_rows_lpr<8>(x, rows, K, qmax, out_int8, clamp, q, s, stream, blocks); break;
-        default: launch_short_rows_lpr<16>(x, rows, K, qmax, out_int8, clamp, q, s, stream, blocks); break;
+        case 2: launch_grouped_lpr<2, J>(x, rows, K, qmax, out_int8, clamp, q, s, stream, blocks); break;
+        case 4: launch_grouped_lpr<4, J>(x, rows, K, qmax, out_int8, clamp, q, s, stream, blocks); break;
+        case 8: launch_grouped_lpr<8, J>(x, rows, K, qmax, out_int8, clamp, q, s, stream, blocks); break;
+        case 16: launch_grouped_lpr<16, J>(x, rows, K, qmax, out_int8, clamp, q, s, stream, blocks); break;
+        default: launch_grouped_lpr<32, J>(x, rows, K, qmax, out_int8, clamp, q, s, stream, blocks); break;
+    }
+}
+
+struct GroupShape {
+    int lpr;    // lanes per row (a power of two, 2..32)
+    int j;      // units per lane (1, 4 or 8)
+    int waste;  // lane slots left empty per row: lpr * j - units
+};
+
+GroupShape group_shape(int units, int j) {
+    int lpr = 2;
+    while (lpr * j < units) lpr *= 2;
+    return {lpr, j, lpr * j - units};
+}
+
+// Lanes per row and units per lane for a row of `units` 16-byte units
+// (units <= kGroupMaxUnits), from a sweep of K = 16..2048 on B200 (1 GiB of
+// input per call): 4 units per lane wins where it fills every lane slot
+// (K = 64, 128, 256, 512, 1024) and where 8 units per lane would leave only
+// two lanes per row; otherwise the shape with fewer empty slots, 8 units per
+// lane on a tie; one unit per lane for rows of K <= 16.
+GroupShape pick_group_shape(int units) {
+    if (TFQ_QUANT_FORCE_J != 0) return group_shape(units, TFQ_QUANT_FORCE_J);
+    if (units <= 2) return group_shape(units, 1);
+    const GroupShape g8 = group_shape(units, 8);
+    if (units > 128) return g8;
+    const GroupShape g4 = group_shape(units, 4);
+    if (g4.waste == 0 || g8.lpr == 2) return g4;
+    return g4.waste < g8.waste ? g4 : g8;
+}
+
+tfq_status launch_grouped_rows(const void* x, int64_t rows, int64_t K, float qmax, bool out_int8, bool clamp,
+                               void* q, float* s, cudaStream_t stream, DeviceState* ds) {
+    const GroupShape g = pick_group_shape(static_cast<int>(K / 8));
+    if (g.lpr > 32) return fail(TFQ_EUNSUPPORTED, "row of K=%lld does not fit one warp", (long long)K);
+    switch (g.j) {
+        case 1: launch_grouped_j<1>(g.lpr, x, rows, K, qmax, out_int8, clamp, q, s, stream, ds->sm_count); break;
+        case 4: launch_grouped_j<4>(g.lpr, x, rows, K, qmax, out_int8, clamp, q, s, stream, ds->sm_count); break;
+        default: launch_grouped_j<8>(g.lpr, x, rows, K, qmax, out_int8, clamp, q, s, stream, ds->sm_count); break;
     }
     const cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? TFQ_OK : fail(TFQ_ECUDA, "quantizer launch: %s", cudaGetErrorString(e));
@@ -375,11 +459,7 @@ tfq_status launch_quant_rows(const void* x, int64_t rows, int64_t K, float qmax,
         return e == cudaSuccess ? TFQ_OK : fail(TFQ_ECUDA, "quantizer launch: %s", cudaGetErrorString(e));
     }
     const bool clamp = !out_int8 && !is_e4m3_value(qmax);
-    if (K <= 128) {
-        const int units = static_cast<int>(K / 8);
-        const int lpr = units <= 2 ? 2 : units <= 4 ? 4 : units <= 8 ? 8 : 16;
-        return launch_short_rows(x, rows, K, qmax, out_int8, clamp, lpr, q, s, stream, ds);
-    }
+    if (K / 8 <= kGroupMaxUnits) return launch_grouped_rows(x, rows, K, qmax, out_int8, clamp, q, s, stream, ds);
     auto kernel = out_int8 ? quant_rows_kernel<true, false>
                            : (clamp ? quant_rows_kernel<false, true> : quant_rows_kernel<false, false>);
     const int threads = 256;  // 8 warps, one row per warp at a time

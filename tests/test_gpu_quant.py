@@ -146,9 +146,9 @@ def test_tensor_wrappers_match_raw():
 @pytest.mark.parametrize("K", [16, 32, 48, 64, 96, 112, 128])
 @pytest.mark.parametrize("M", [1, 3, 37, 1000, 4097])
 def test_short_rows_sub_warp(M, K):
-    """K <= 128 runs the sub-warp kernel (2..16 lanes per row, several rows per
-    warp): ragged M, lanes beyond the row's units, FP8 with and without the
-    clamp, INT8."""
+    """K <= 128 runs the grouped kernel with 2..4 lanes per row and 1 or 4
+    units per lane (8..16 rows per warp): ragged M, lane slots beyond the
+    row's units, FP8 with and without the clamp, INT8."""
     x = workloads.activations(M, K, seed=M + K, nu=3, outlier_cols=1, outlier_mult=25.0,
                               zero_rows=1 if M > 2 else 0, device="cuda")
     for qmax in (448.0, 21.0):
@@ -165,3 +165,20 @@ def test_kv_cache_per_vector_full_size():
     x = workloads.activations(75600 * 40, 128, seed=77, nu=4, device="cuda")
     rows = _gpu.sample_rows(x.shape[0], 4096, seed=78)
     _assert_fp8_equal(x, 448.0, rows)
+
+
+@pytest.mark.parametrize("K", [144, 256, 272, 384, 512, 528, 1024, 1152, 1536, 2048, 2064])
+@pytest.mark.parametrize("M", [1, 5, 130, 2049])
+def test_mid_rows_grouped(M, K):
+    """128 < K <= 2048 runs the grouped kernel (several rows per warp, up to 8
+    units per lane, a row's lanes reduce among themselves); K = 2064 is the
+    first size past it.  Ragged M (a warp's last rows missing), units that do
+    not fill the row's lanes, FP8 with and without the clamp, INT8."""
+    x = workloads.activations(M, K, seed=3 * M + K, nu=3, outlier_cols=2, outlier_mult=25.0,
+                              zero_rows=1 if M > 2 else 0, device="cuda")
+    for qmax in (448.0, 21.0, 7.0):
+        _assert_fp8_equal(x, qmax)
+    q, s = _gpu.quant_weight(x, _capi.TFQ_DTYPE_INT8, 127.0)
+    q_ref, s_ref = _gpu.oracle_quant_int8(x, 127.0)
+    np.testing.assert_array_equal(s.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
+    np.testing.assert_array_equal(q.cpu().numpy().view(np.int8), q_ref)

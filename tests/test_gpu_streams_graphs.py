@@ -1,0 +1,97 @@
+"""Concurrency and graph capture of the C-ABI calls:
+* GEMMs launched concurrently on two streams (each launch takes its own
+  pacing-counter slot) give exactly the results of the same calls run one
+  after the other -- every output element is computed by one CTA in a fixed
+  order, so the kernels are deterministic;
+* the quantizer and the GEMM calls captured into a CUDA graph (after the
+  device's one-time set-up) replay to the eager results on new inputs."""
+import pytest
+import torch
+
+from int8_w8a8_quantized_b200 import _capi, workloads
+from tests import _gpu
+
+pytestmark = pytest.mark.gpu
+
+
+def _codes(g, shape):
+    mag = torch.randint(0, 0x70, shape, generator=g, dtype=torch.int32)
+    return (mag | (torch.randint(0, 2, shape, generator=g, dtype=torch.int32) << 7)).to(torch.uint8).cuda()
+
+
+def _gemm(lib, A, sa, W, sw, b, y, stream):
+    M, K = A.shape
+    N = W.shape[0]
+    st = lib.tfq_scaled_fp8_linear(A.data_ptr(), sa.data_ptr(), W.data_ptr(), sw.data_ptr(),
+                                   None if b is None else b.data_ptr(), M, N, K, y.data_ptr(),
+                                   int(stream.cuda_stream))
+    assert st == _capi.TFQ_OK, _capi.last_error_message()
+
+
+def test_concurrent_streams_match_serial():
+    lib = _gpu.lib()
+    g = torch.Generator().manual_seed(11)
+    cases = []
+    for (M, N, K) in [(3000, 3072, 1024), (2048, 1032, 2048), (700, 520, 512)]:
+        A, W = _codes(g, (M, K)), _codes(g, (N, K))
+        sa = (torch.rand(M, generator=g) * 1e-2).cuda()
+        sw = (torch.rand(N, generator=g) * 1e-2).cuda()
+        b = torch.randn(N, generator=g).to(torch.bfloat16).cuda()
+        cases.append((A, sa, W, sw, b))
+    main = torch.cuda.current_stream()
+    serial = []
+    for c in cases:
+        y = torch.empty((c[0].shape[0], c[2].shape[0]), dtype=torch.bfloat16, device="cuda")
+        _gemm(lib, *c, y, main)
+        serial.append(y)
+    torch.cuda.synchronize()
+    streams = [torch.cuda.Stream() for _ in cases]
+    conc = [torch.empty_like(y) for y in serial]
+    for _ in range(3):
+        for c, y, s in zip(cases, conc, streams):
+            s.wait_stream(main)
+            _gemm(lib, *c, y, s)
+        for s in streams:
+            main.wait_stream(s)
+        torch.cuda.synchronize()
+        for a, b in zip(serial, conc):
+            assert torch.equal(a, b)
+    _gpu.check_device_error()
+
+
+def test_cuda_graph_capture_and_replay():
+    lib = _gpu.lib()
+    M, K, N = 1500, 1024, 776
+    x = workloads.activations(M, K, seed=5, outlier_cols=4, outlier_mult=20.0, device="cuda")
+    w = workloads.weights(N, K, seed=6, std=0.02, device="cuda")
+    b = workloads.bias(N, seed=7, device="cuda")
+    Wq, sw = _gpu.quant_weight(w, _capi.TFQ_DTYPE_FP8_E4M3, 448.0)
+    A = torch.empty((M, K), dtype=torch.uint8, device="cuda")
+    sa = torch.empty(M, device="cuda")
+    y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+
+    def linear(stream):
+        sh = int(stream.cuda_stream)
+        assert lib.tfq_quant_act_fp8_per_token(x.data_ptr(), M, K, 448.0, A.data_ptr(), sa.data_ptr(), sh) == 0
+        assert lib.tfq_scaled_fp8_linear(A.data_ptr(), sa.data_ptr(), Wq.data_ptr(), sw.data_ptr(), b.data_ptr(),
+                                         M, N, K, y.data_ptr(), sh) == 0
+
+    linear(torch.cuda.current_stream())          # one-time set-up happens outside the capture
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        with torch.cuda.graph(graph, stream=side):
+            linear(side)
+    torch.cuda.current_stream().wait_stream(side)
+    for seed in (8, 9):
+        x.copy_(workloads.activations(M, K, seed=seed, nu=4, device="cuda"))
+        graph.replay()
+        torch.cuda.synchronize()
+        y_graph = y.clone()
+        linear(torch.cuda.current_stream())
+        torch.cuda.synchronize()
+        assert torch.equal(y_graph, y)
+    del graph
+    _gpu.check_device_error()
