@@ -24,6 +24,10 @@ What each function follows (page titles and sections of the source pages):
 * ``scaled_int8_linear``: the INT8 W8A8 modes of LightX2V "模型量化技术",
   quantization-mode table (INT8 per-channel weights, dynamic per-token INT8
   activations), exact int64 sums.
+* ``quant_mxfp8`` / ``mxfp8_linear``: MXFP8 as named on the TeleFuser
+  "Quantization" page, "Offline conversion" (32-value blocks, E8M0 scales),
+  with the conversion of the OCP Microscaling (MX) v1.0 specification; the
+  GEMM applies both block scales per 32-element block of K, in double.
 
 Every function is pinned by the ``-m "not gpu"`` tests against values fixed
 by the format definition, brute force and invariants (see ``tests/``).
@@ -78,6 +82,10 @@ def _load():
                 fn = getattr(lib, name)
                 fn.restype = None
                 fn.argtypes = [P, P, P, P, P, I64, I64, I64, P, I64, P]
+            lib.tfq_oracle_quant_mxfp8.restype = None
+            lib.tfq_oracle_quant_mxfp8.argtypes = [P, I64, I64, P, P]
+            lib.tfq_oracle_mxfp8_linear.restype = None
+            lib.tfq_oracle_mxfp8_linear.argtypes = [P, P, P, P, P, I64, I64, I64, P, I64, P]
             lib.tfq_oracle_num_threads.restype = ctypes.c_int
             lib.tfq_oracle_num_threads.argtypes = []
             lib.tfq_oracle_set_num_threads.restype = None
@@ -185,3 +193,45 @@ def scaled_int8_linear(A, s_a, W, s_w, bias_bits=None, rows=None) -> np.ndarray:
     """y[i,n] = sum_k A[m,k] W[n,k] * s_a[m] * s_w[n] + bias[n] (double)."""
     return _linear(_load().tfq_oracle_scaled_int8_linear, A, s_a, W, s_w,
                    bias_bits, rows, np.int8)
+
+
+def quant_mxfp8(x_bits):
+    """MXFP8 quantization of bf16 bits [R, K] (K % 32 == 0) ->
+    (codes u8 [R, K], E8M0 scale codes u8 [R, K // 32], row-major)."""
+    x = _bf16_bits(x_bits)
+    R, K = x.shape
+    if K % 32:
+        raise ValueError("K must be a multiple of 32")
+    q = np.empty((R, K), dtype=np.uint8)
+    sf = np.empty((R, K // 32), dtype=np.uint8)
+    _load().tfq_oracle_quant_mxfp8(_ptr(x), R, K, _ptr(q), _ptr(sf))
+    return q, sf
+
+
+def mxfp8_linear(A, sf_a, W, sf_w, bias_bits=None, rows=None) -> np.ndarray:
+    """y[i,n] = sum_b 2^(sf_a[m,b]-127) 2^(sf_w[n,b]-127) sum_{k in b} dec(A) dec(W)
+    + bias[n] (double); sf_* are row-major [rows, K // 32] E8M0 codes."""
+    A = np.ascontiguousarray(A, dtype=np.uint8)
+    W = np.ascontiguousarray(W, dtype=np.uint8)
+    sf_a = np.ascontiguousarray(sf_a, dtype=np.uint8)
+    sf_w = np.ascontiguousarray(sf_w, dtype=np.uint8)
+    M, K = A.shape
+    N, K2 = W.shape
+    if K2 != K or K % 32 or sf_a.shape != (M, K // 32) or sf_w.shape != (N, K // 32):
+        raise ValueError("shape mismatch")
+    b = None
+    if bias_bits is not None:
+        b = _bf16_bits(bias_bits)
+        if b.shape != (N,):
+            raise ValueError("bias shape")
+    r = None
+    nrows = M
+    if rows is not None:
+        r = np.ascontiguousarray(rows, dtype=np.int64)
+        if r.size and (r.min() < 0 or r.max() >= M):
+            raise ValueError("row index out of range")
+        nrows = r.size
+    y = np.empty((nrows, N), dtype=np.float64)
+    _load().tfq_oracle_mxfp8_linear(_ptr(A), _ptr(sf_a), _ptr(W), _ptr(sf_w), _ptr(b), M, N, K, _ptr(r),
+                                    nrows, _ptr(y))
+    return y

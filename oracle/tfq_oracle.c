@@ -18,6 +18,9 @@
  *  - The INT8 variant  s = max|x| / 127,  q = clamp(round(x / s), -128, 127)
  *    TeleFuser "Quantization" page, section "Core ideas" (integer formula),
  *    one scale per output row as in section "Offline conversion".
+ *  - MXFP8 (32-value blocks, E8M0 power-of-two scales) and its block-scaled
+ *    GEMM: TeleFuser "Quantization" page, section "Offline conversion" names
+ *    the format; the conversion is the OCP MX v1.0 one (see below).
  *  - The scaled GEMM  y[m,n] = s_a[m] s_w[n] sum_k q_a[m,k] q_w[n,k] (+ b[n])
  *    TeleFuser "Quantization" page, sections "Scaled FP8 checkpoints" and
  *    "tf-kernel FP8: online W8A8" (per-token activations, per-output-channel
@@ -270,6 +273,120 @@ void tfq_oracle_scaled_int8_linear(const int8_t *A, const float *s_a,
             if (bias)
                 v += (double)bf16_bits_to_float(bias[n]);
             y[i * N + n] = v;
+        }
+    }
+}
+
+/* ------------------------------------------------------------------ */
+/* MXFP8: E4M3 elements with one E8M0 (power-of-two) scale per block of */
+/* 32 consecutive values of a row.                                     */
+/* ------------------------------------------------------------------ */
+/*
+ * The TeleFuser "Quantization" page (section "Offline conversion") names the
+ * format -- 32-value blocks with E8M0 scales -- but not the conversion.  The
+ * reading taken is the conversion of the OCP Microscaling Formats (MX) v1.0
+ * specification (section "Conversion from vectors of scalars to MX"):
+ *   shared exponent  E = floor(log2(max_k |x_k|)) - emax,  emax = 8 for E4M3
+ *                    (its largest normal is 1.75 * 2^8 = 448);
+ *   E is clamped to the E8M0 range [-127, 127] and stored as code E + 127;
+ *   element          q_k = E4M3_RNE(clamp(x_k / 2^E, -448, 448)).
+ * A block whose values are all zero has no exponent; it takes the smallest
+ * scale, code 0 (its elements are zeros whatever the scale).
+ * Dividing by 2^E is exact in double, so no fp32 rounding step is involved.
+ */
+static uint8_t e8m0_block_code(float amax)
+{
+    int E, e;
+    if (amax == 0.0f)
+        return 0;
+    (void)frexp((double)amax, &E); /* amax = f * 2^E, f in [0.5, 1) */
+    e = (E - 1) - 8;               /* floor(log2(amax)) - emax(E4M3) */
+    if (e < -127)
+        e = -127;
+    if (e > 127)
+        e = 127;
+    return (uint8_t)(e + 127);
+}
+
+/*
+ * MXFP8 quantization of a row-major bf16 matrix x[rows, K] (K % 32 == 0):
+ * codes q[rows, K] and scale codes sf[rows, K / 32], both row-major.  Used
+ * for activations (rows = tokens) and weights (rows = output channels).
+ */
+void tfq_oracle_quant_mxfp8(const uint16_t *x, int64_t rows, int64_t K,
+                            uint8_t *q, uint8_t *sf)
+{
+    const int64_t nb = K / 32;
+    int64_t r;
+#pragma omp parallel for schedule(static)
+    for (r = 0; r < rows; ++r) {
+        int64_t b;
+        for (b = 0; b < nb; ++b) {
+            const uint16_t *blk = x + r * K + b * 32;
+            float amax = 0.0f;
+            uint8_t code;
+            double scale;
+            int k;
+            for (k = 0; k < 32; ++k) {
+                float v = fabsf(bf16_bits_to_float(blk[k]));
+                if (v > amax)
+                    amax = v;
+            }
+            code = e8m0_block_code(amax);
+            sf[r * nb + b] = code;
+            scale = ldexp(1.0, (int)code - 127);
+            for (k = 0; k < 32; ++k) {
+                double t = (double)bf16_bits_to_float(blk[k]) / scale;
+                if (t > 448.0)
+                    t = 448.0;
+                if (t < -448.0)
+                    t = -448.0;
+                q[r * K + b * 32 + k] = tfq_oracle_e4m3_encode((float)t);
+            }
+        }
+    }
+}
+
+/*
+ * MXFP8 GEMM, "TN" layout, both operands block-scaled along K:
+ *   y[i, n] = sum_b 2^(sfa[m,b] - 127) * 2^(sfw[n,b] - 127)
+ *                   * sum_{k in block b} dec(A[m,k]) * dec(W[n,k])   (+ bias[n])
+ * for m = rows[i] (or m = i when rows is NULL).  Each block sum is exact in
+ * double (32 products, each a multiple of 2^-18 below 2^18); the power-of-two
+ * scaling is exact; only the sum over blocks rounds (to 53 bits).
+ */
+void tfq_oracle_mxfp8_linear(const uint8_t *A, const uint8_t *sfa,
+                             const uint8_t *W, const uint8_t *sfw,
+                             const uint16_t *bias, int64_t M, int64_t N,
+                             int64_t K, const int64_t *rows, int64_t nrows,
+                             double *y)
+{
+    const int64_t nb = K / 32;
+    double dec[256];
+    int64_t i;
+    int c;
+    (void)M;
+    for (c = 0; c < 256; ++c)
+        dec[c] = tfq_oracle_e4m3_decode((uint8_t)c);
+#pragma omp parallel for schedule(dynamic, 1)
+    for (i = 0; i < nrows; ++i) {
+        int64_t m = rows ? rows[i] : i;
+        int64_t n;
+        for (n = 0; n < N; ++n) {
+            double acc = 0.0;
+            int64_t b;
+            for (b = 0; b < nb; ++b) {
+                const uint8_t *a = A + m * K + b * 32;
+                const uint8_t *w = W + n * K + b * 32;
+                double part = 0.0;
+                int k;
+                for (k = 0; k < 32; ++k)
+                    part += dec[a[k]] * dec[w[k]];
+                acc += ldexp(part, (int)sfa[m * nb + b] + (int)sfw[n * nb + b] - 254);
+            }
+            if (bias)
+                acc += (double)bf16_bits_to_float(bias[n]);
+            y[i * N + n] = acc;
         }
     }
 }
