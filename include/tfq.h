@@ -164,6 +164,54 @@ TFQ_API tfq_status tfq_scaled_fp8_linear_f16acc(const void *A_q, const float *s_
                                                 int64_t K, void *out_bf16, void *stream);
 
 /*
+ * MXFP8: E4M3FN codes with one E8M0 scale (a power of two 2^(c - 127), code
+ * c in 0..254) per block of 32 consecutive elements of a row -- the format
+ * the TeleFuser "Quantization" page names in section "Offline conversion"
+ * (32-value blocks, E8M0 scales).  The page gives no conversion rule; the one
+ * implemented is that of the OCP Microscaling (MX) v1.0 specification:
+ *   E = floor(log2(max |x| over the block)) - 8, clamped to [-127, 127]
+ *       (8 = exponent of 448, the largest E4M3 normal), code E + 127;
+ *   q = E4M3FN_rn(clamp(x / 2^E, -448, 448))   (x / 2^E is exact);
+ *   a block of zeros gets code 0.
+ *
+ * Scale-factor layout (the one the sm_100 block-scaled tensor-core MMA reads
+ * from shared memory), for an operand of `rows` rows and K columns: with
+ * RA = ceil(rows / 128) and KA = ceil(K / 128), the buffer holds RA * KA
+ * atoms of 512 bytes; the atom of rows 128 ra.. and K blocks 4 ka.. is atom
+ * number ka * RA + ra, and inside it the code of row r, K block b (b = k / 32)
+ * is at byte 16 (r % 32) + 4 ((r % 128) / 32) + (b % 4).  Entries of rows >=
+ * rows or blocks >= K / 32 are padding, written as 127 (scale 1) by
+ * tfq_quant_mxfp8.  tfq_mxfp8_scale_bytes gives the buffer size.
+ */
+#define TFQ_MX_BLOCK 32
+TFQ_API int64_t tfq_mxfp8_scale_bytes(int64_t rows, int64_t K);
+
+/*
+ * tfq_quant_mxfp8: x bf16 [rows, K] (row-major) -> q [rows, K] E4M3FN codes
+ * and sf (tfq_mxfp8_scale_bytes(rows, K) bytes, layout above).  Activations
+ * (rows = tokens) and weights (rows = output channels) alike.
+ * Preconditions: K % 32 == 0, K <= TFQ_QUANT_MAX_K; 16-byte aligned pointers.
+ * rows == 0 is a no-op.  Errors as tfq_quant_act_fp8_per_token.
+ */
+TFQ_API tfq_status tfq_quant_mxfp8(const void *x_bf16, int64_t rows, int64_t K, void *q_e4m3, void *sf_e8m0,
+                                   void *stream);
+
+/*
+ * tfq_mxfp8_linear: the block-scaled GEMM, "TN":
+ *   out[m,n] = bf16_rn(sum_b 2^(sfa[m,b]-127) 2^(sfw[n,b]-127)
+ *                        sum_{k in block b} A_q[m,k] W_q[n,k] + bias[n])
+ * with A_q [M, K], W_q [N, K] E4M3FN codes and sf_a, sf_w their scale
+ * buffers from tfq_quant_mxfp8 (or any buffer in that layout with finite
+ * codes <= 254).  The tensor cores apply both scales per 32-element block and
+ * accumulate in fp32; tolerance as tfq_scaled_fp8_linear.
+ * Preconditions: K % 32 == 0, N % 8 == 0, 16-byte aligned pointers.
+ * Errors as tfq_scaled_fp8_linear.
+ */
+TFQ_API tfq_status tfq_mxfp8_linear(const void *A_q, const void *sf_a, const void *W_q, const void *sf_w,
+                                    const void *bias_bf16, int64_t M, int64_t N, int64_t K, void *out_bf16,
+                                    void *stream);
+
+/*
  * Bytes of the static device array used by tfq_scaled_fp8_linear_noalloc.
  * Every GPU that loads the library holds this array until the process exits.
  */

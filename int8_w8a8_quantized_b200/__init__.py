@@ -20,11 +20,15 @@ from ._capi import (  # noqa: F401
     TfqError,
     last_error_message,
     load_library,
+    mxfp8_linear,
     raw,
     status_string,
     tfq_device_error,
+    tfq_mxfp8_linear,
+    tfq_mxfp8_scale_bytes,
     tfq_quant_act_fp8_per_token,
     tfq_quant_act_int8_per_token,
+    tfq_quant_mxfp8,
     tfq_quant_weight_per_channel,
     tfq_scaled_fp8_linear,
     tfq_scaled_int8_linear,
@@ -41,6 +45,10 @@ __all__ = [
     "w8a8_int8_linear",
     "tfq_device_error",
     "w8a8_linear",
+    "tfq_quant_mxfp8",
+    "tfq_mxfp8_linear",
+    "tfq_mxfp8_scale_bytes",
+    "mxfp8_linear",
     "TfqError",
     "raw",
 ]

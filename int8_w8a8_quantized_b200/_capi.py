@@ -35,6 +35,9 @@ SIGNATURES = {
     "tfq_quant_act_int8_per_token": (_I, [_P, _I64, _I64, _F, _P, _P, _P]),
     "tfq_scaled_int8_linear": (_I, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _P]),
     "tfq_scaled_fp8_linear_f16acc": (_I, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _P]),
+    "tfq_mxfp8_scale_bytes": (_I64, [_I64, _I64]),
+    "tfq_quant_mxfp8": (_I, [_P, _I64, _I64, _P, _P, _P]),
+    "tfq_mxfp8_linear": (_I, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _P]),
     "tfq_scaled_fp8_linear_noalloc": (_I, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _P]),
     "tfq_selftest_div_rn": (_I, [_P, _P, _I64, _P, _P, _P]),
     "tfq_selftest_wait_timeout": (_I, [ctypes.c_uint32, _P]),
@@ -246,6 +249,69 @@ def w8a8_int8_linear(x, W_q, s_w, bias=None, qmax: float = 127.0, stream=None):
     """The INT8 Linear: per-token INT8 quantization of x, then the scaled INT8 GEMM."""
     A_q, s_a = tfq_quant_act_int8_per_token(x, qmax, stream=stream)
     return tfq_scaled_int8_linear(A_q, s_a, W_q, s_w, bias, stream=stream)
+
+
+def tfq_mxfp8_scale_bytes(rows: int, K: int) -> int:
+    """Bytes of the E8M0 scale buffer of a [rows, K] MXFP8 operand."""
+    n = int(load_library().tfq_mxfp8_scale_bytes(int(rows), int(K)))
+    if n < 0:
+        raise ValueError("negative size")
+    return n
+
+
+def tfq_quant_mxfp8(x, q=None, sf=None, stream=None):
+    """x bf16 [R, K] (K % 32 == 0) -> (q uint8 [R, K] E4M3FN codes,
+    sf uint8 [tfq_mxfp8_scale_bytes(R, K)] E8M0 codes in the tensor-core layout)."""
+    import torch
+    _require(x, torch.bfloat16, 2, "x")
+    R, K = x.shape
+    if q is None:
+        q = torch.empty((R, K), dtype=torch.uint8, device=x.device)
+    if sf is None:
+        sf = torch.empty((tfq_mxfp8_scale_bytes(R, K),), dtype=torch.uint8, device=x.device)
+    _require(q, torch.uint8, 2, "q")
+    _require(sf, torch.uint8, 1, "sf")
+    if tuple(q.shape) != (R, K) or sf.numel() < tfq_mxfp8_scale_bytes(R, K):
+        raise ValueError("output shapes do not match x")
+    with torch.cuda.device(x.device):
+        st = raw.tfq_quant_mxfp8(x.data_ptr(), R, K, q.data_ptr(), sf.data_ptr(), _stream_handle(stream))
+    _check(st, "tfq_quant_mxfp8")
+    return q, sf
+
+
+def tfq_mxfp8_linear(A_q, sf_a, W_q, sf_w, bias=None, out=None, stream=None):
+    """A_q uint8 [M, K], W_q uint8 [N, K] E4M3FN codes with their scale buffers
+    from tfq_quant_mxfp8, bias bf16 [N] or None -> out bf16 [M, N]."""
+    import torch
+    _require(A_q, torch.uint8, 2, "A_q")
+    _require(W_q, torch.uint8, 2, "W_q")
+    _require(sf_a, torch.uint8, 1, "sf_a")
+    _require(sf_w, torch.uint8, 1, "sf_w")
+    M, K = A_q.shape
+    N, K2 = W_q.shape
+    if K2 != K or sf_a.numel() < tfq_mxfp8_scale_bytes(M, K) or sf_w.numel() < tfq_mxfp8_scale_bytes(N, K):
+        raise ValueError("shape mismatch")
+    if bias is not None:
+        _require(bias, torch.bfloat16, 1, "bias")
+        if bias.shape[0] != N:
+            raise ValueError("bias shape")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=A_q.device)
+    _require(out, torch.bfloat16, 2, "out")
+    if tuple(out.shape) != (M, N):
+        raise ValueError("out shape")
+    with torch.cuda.device(A_q.device):
+        st = raw.tfq_mxfp8_linear(A_q.data_ptr(), sf_a.data_ptr(), W_q.data_ptr(), sf_w.data_ptr(),
+                                  None if bias is None else bias.data_ptr(), M, N, K, out.data_ptr(),
+                                  _stream_handle(stream))
+    _check(st, "tfq_mxfp8_linear")
+    return out
+
+
+def mxfp8_linear(x, W_q, sf_w, bias=None, stream=None):
+    """The MXFP8 Linear: block quantization of x, then the block-scaled GEMM."""
+    A_q, sf_a = tfq_quant_mxfp8(x, stream=stream)
+    return tfq_mxfp8_linear(A_q, sf_a, W_q, sf_w, bias, stream=stream)
 
 
 def tfq_device_error(stream=None) -> None:

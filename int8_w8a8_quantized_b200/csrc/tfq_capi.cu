@@ -221,6 +221,48 @@ tfq_status tfq_scaled_fp8_linear_f16acc(const void* A_q, const float* s_a, const
                                          static_cast<cudaStream_t>(stream), ds);
 }
 
+int64_t tfq_mxfp8_scale_bytes(int64_t rows, int64_t K) {
+    if (rows < 0 || K < 0) return -1;
+    return ((rows + 127) / 128) * ((K + 127) / 128) * 512;
+}
+
+tfq_status tfq_quant_mxfp8(const void* x_bf16, int64_t rows, int64_t K, void* q_e4m3, void* sf_e8m0,
+                           void* stream) {
+    if (rows < 0 || K < 0) return fail(TFQ_EINVAL, "negative size (rows=%lld, K=%lld)", (long long)rows, (long long)K);
+    if (K % TFQ_MX_BLOCK != 0) return fail(TFQ_EINVAL, "K=%lld is not a multiple of %d", (long long)K, TFQ_MX_BLOCK);
+    if (K > TFQ_QUANT_MAX_K) return fail(TFQ_EUNSUPPORTED, "K=%lld above %d", (long long)K, TFQ_QUANT_MAX_K);
+    if (rows >= (int64_t(1) << 31)) return fail(TFQ_EUNSUPPORTED, "rows=%lld too large", (long long)rows);
+    if (rows == 0 || K == 0) return TFQ_OK;
+    if (x_bf16 == nullptr || q_e4m3 == nullptr || sf_e8m0 == nullptr) return fail(TFQ_EINVAL, "null pointer");
+    if (!aligned16(x_bf16) || !aligned16(q_e4m3) || !aligned16(sf_e8m0))
+        return fail(TFQ_EINVAL, "pointer not 16-byte aligned");
+    tfq_status st;
+    DeviceState* ds = current_device_state(&st);
+    if (ds == nullptr) return st;
+    return launch_quant_mxfp8(x_bf16, rows, K, q_e4m3, sf_e8m0, static_cast<cudaStream_t>(stream), ds);
+}
+
+tfq_status tfq_mxfp8_linear(const void* A_q, const void* sf_a, const void* W_q, const void* sf_w,
+                            const void* bias_bf16, int64_t M, int64_t N, int64_t K, void* out_bf16, void* stream) {
+    if (M < 0 || N < 0 || K < 0) return fail(TFQ_EINVAL, "negative size");
+    if (K == 0 || K % TFQ_MX_BLOCK != 0)
+        return fail(TFQ_EINVAL, "K=%lld must be a positive multiple of %d", (long long)K, TFQ_MX_BLOCK);
+    if (N % 8 != 0) return fail(TFQ_EINVAL, "N=%lld is not a multiple of 8", (long long)N);
+    const int64_t lim = int64_t(1) << 31;
+    if (M >= lim || N >= lim || K >= lim) return fail(TFQ_EUNSUPPORTED, "size too large");
+    if (M == 0 || N == 0) return TFQ_OK;
+    if (A_q == nullptr || sf_a == nullptr || W_q == nullptr || sf_w == nullptr || out_bf16 == nullptr)
+        return fail(TFQ_EINVAL, "null pointer");
+    if (!aligned16(A_q) || !aligned16(sf_a) || !aligned16(W_q) || !aligned16(sf_w) || !aligned16(out_bf16) ||
+        (bias_bf16 != nullptr && !aligned16(bias_bf16)))
+        return fail(TFQ_EINVAL, "pointer not 16-byte aligned");
+    tfq_status st;
+    DeviceState* ds = current_device_state(&st);
+    if (ds == nullptr) return st;
+    return launch_mxfp8_gemm(A_q, static_cast<const uint8_t*>(sf_a), W_q, static_cast<const uint8_t*>(sf_w),
+                             bias_bf16, M, N, K, out_bf16, static_cast<cudaStream_t>(stream), ds);
+}
+
 tfq_status tfq_scaled_fp8_linear(const void* A_q, const float* s_a, const void* W_q, const float* s_w,
                                  const void* bias_bf16, int64_t M, int64_t N, int64_t K, void* out_bf16,
                                  void* stream) {

@@ -31,7 +31,7 @@ struct DeviceState {
     unsigned* round_ctrs = nullptr;
     int round_slots = 0;
     int next_round_slot = 0;
-    bool gemm_attr_set[3] = {false, false, false};  // FP8, INT8, FP8 with FP16 accumulator
+    bool gemm_attr_set[4] = {false, false, false, false};  // FP8, INT8, FP8 with FP16 accumulator, MXFP8
 };
 
 // Per-device state of the current device, created on first use.  Returns
@@ -57,6 +57,8 @@ tfq_status launch_quant_rows(const void* x, int64_t rows, int64_t K, float qmax,
                              cudaStream_t stream, DeviceState* ds);
 
 // Self-check: the quantizer's division next to the IEEE division.
+tfq_status launch_quant_mxfp8(const void* x, int64_t rows, int64_t K, void* q, void* sf, cudaStream_t stream,
+                              DeviceState* ds);
 tfq_status launch_div_selftest(const float* a, const float* b, int64_t n, float* ours, float* ieee,
                                cudaStream_t stream);
 
@@ -77,6 +79,8 @@ tfq_status launch_scaled_fp8_gemm_f16acc(const void* A, const float* s_a, const 
                                          cudaStream_t stream, DeviceState* ds);
 
 // Scaled INT8 GEMM (S8 x S8 -> S32 on the tensor cores) with the same epilogue.
+tfq_status launch_mxfp8_gemm(const void* A, const uint8_t* sf_a, const void* W, const uint8_t* sf_w, const void* bias,
+                             int64_t M, int64_t N, int64_t K, void* out, cudaStream_t stream, DeviceState* ds);
 tfq_status launch_scaled_int8_gemm(const void* A, const float* s_a, const void* W, const float* s_w,
                                    const void* bias, int64_t M, int64_t N, int64_t K, void* out,
                                    cudaStream_t stream, DeviceState* ds);

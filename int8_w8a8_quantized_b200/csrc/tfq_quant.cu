@@ -341,6 +341,114 @@ __global__ void __launch_bounds__(256, grouped_ctas_per_sm<J>()) quant_grouped_r
     }
 }
 
+// ------------------------------------------------------------------ MXFP8
+// One E8M0 scale per 32 consecutive elements of a row (the OCP MX v1.0
+// conversion): E = floor(log2(block max)) - 8, clamped to [-127, 127], code
+// E + 127 (0 for a block of zeros); q = E4M3_rn_satfinite(x * 2^-E).  The
+// product with the power of two is exact (it only rounds when the result is
+// far below the smallest E4M3 subnormal, where the code is a signed zero
+// anyway), so no division is needed.  The matrix is streamed as a flat
+// sequence of 16-byte units (a 32-element block is 4 units and never crosses
+// a row because K % 32 == 0): lane l of a warp holds units base + l + 32 j,
+// j < kMxJ, so a block sits in 4 adjacent lanes and its maximum takes two
+// shuffles.  Scale codes go to the tensor-core scale-factor layout.
+
+constexpr int kMxJ = 8;  // 16-byte units per lane per iteration: 4 KiB in flight per warp
+
+__device__ __forceinline__ uint32_t e8m0_code(float amax) {
+    const uint32_t bits = __float_as_uint(amax);
+    if (bits == 0u) return 0u;
+    const int biased = static_cast<int>(bits >> 23);
+    // floor(log2(amax)): from the exponent field, or for a subnormal from the
+    // position of the leading mantissa bit (value m * 2^-149)
+    const int fl = biased != 0 ? biased - 127 : -118 - __clz(bits);
+    return static_cast<uint32_t>(min(max(fl + 119, 0), 254));
+}
+
+// 2^(127 - code) as fp32; code 254 gives 2^-127, a subnormal.
+__device__ __forceinline__ float e8m0_inverse(uint32_t code) {
+    const int k = 127 - static_cast<int>(code);
+    return k >= -126 ? __uint_as_float(static_cast<uint32_t>(k + 127) << 23) : __uint_as_float(0x00400000u);
+}
+
+__device__ __forceinline__ uint32_t mx_pair(uint32_t w, float2 inv2) {
+    const float2 t = __fmul2_rn(make_float2(bf16_lo(w), bf16_hi(w)), inv2);
+    return cvt_e4m3x2(t.x, t.y);
+}
+
+__device__ __forceinline__ uint2 quantize8_mx(const uint4& v, float inv) {
+    const float2 inv2 = make_float2(inv, inv);
+    const uint32_t lo = mx_pair(v.x, inv2) | (mx_pair(v.y, inv2) << 16);
+    const uint32_t hi = mx_pair(v.z, inv2) | (mx_pair(v.w, inv2) << 16);
+    return make_uint2(lo | sign_bytes(v.x, v.y), hi | sign_bytes(v.z, v.w));
+}
+
+// Byte offset of the scale code of (row r, K block b) in the scale-factor
+// layout: 512-byte atoms of 128 rows x 4 blocks, atom (b / 4) * ra + r / 128;
+// inside it row r % 32 owns 16 bytes, (r % 128) / 32 picks the 4-byte word
+// and b % 4 the byte.
+__device__ __forceinline__ int64_t mx_sf_offset(int64_t r, int64_t b, int64_t ra) {
+    return ((b >> 2) * ra + (r >> 7)) * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4 + (b & 3);
+}
+
+__global__ void __launch_bounds__(256) quant_mxfp8_kernel(const uint4* __restrict__ x, int64_t rows, int K,
+                                                          uint8_t* __restrict__ q, uint8_t* __restrict__ sf) {
+    const int lane = threadIdx.x & 31;
+    const int nb = K >> 5;  // blocks per row
+    const int64_t ra = (rows + 127) >> 7;
+    const int64_t total = rows * static_cast<int64_t>(K >> 3);
+    const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+    uint2* q2 = reinterpret_cast<uint2*>(q);
+    for (int64_t base = warp * (32 * kMxJ); base < total; base += nwarps * (32 * kMxJ)) {
+        uint4 v[kMxJ];
+#pragma unroll
+        for (int j = 0; j < kMxJ; ++j) {
+            const int64_t u = base + lane + 32 * j;
+            v[j] = u < total ? ldg_nc_v4(x + u) : make_uint4(0u, 0u, 0u, 0u);
+        }
+        const int64_t blk0 = base >> 2;  // the warp's first block
+        const int64_t r0 = blk0 / nb;
+        const int b0 = static_cast<int>(blk0 - r0 * nb);
+#pragma unroll
+        for (int j = 0; j < kMxJ; ++j) {
+            const uint32_t m = max_abs4(0u, v[j]) & 0x7FFF7FFFu;
+            float amax = fmaxf(bf16_lo(m), bf16_hi(m));
+            amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
+            amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 2));
+            const uint32_t code = e8m0_code(amax);
+            const int64_t u = base + lane + 32 * j;
+            if (u < total) {
+                q2[u] = quantize8_mx(v[j], e8m0_inverse(code));
+                if ((lane & 3) == 0) {
+                    const int d = b0 + (lane >> 2) + 8 * j;  // blocks past the start of row r0
+                    const int dr = d / nb;
+                    sf[mx_sf_offset(r0 + dr, d - dr * nb, ra)] = static_cast<uint8_t>(code);
+                }
+            }
+        }
+    }
+    // Padding entries of the layout (rows past `rows`, blocks past K / 32):
+    // scale code 127 (2^0), so that a padded block multiplies zeros by 1.
+    const int64_t nbp = static_cast<int64_t>((K + 127) >> 7) * 4;
+    const int64_t n1 = (ra * 128 - rows) * nbp;
+    const int64_t n2 = rows * (nbp - nb);
+    const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    const int64_t nthreads = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    for (int64_t i = tid; i < n1 + n2; i += nthreads) {
+        int64_t r, b;
+        if (i < n1) {
+            r = rows + i / nbp;
+            b = i % nbp;
+        } else {
+            const int64_t w = nbp - nb, k = i - n1;
+            r = k / w;
+            b = nb + k % w;
+        }
+        sf[mx_sf_offset(r, b, ra)] = 127;
+    }
+}
+
 // Element-wise self-check of div_rn_from_rcp against the IEEE division.
 __global__ void div_selftest_kernel(const float* __restrict__ a, const float* __restrict__ b, int64_t n,
                                     float* __restrict__ ours, float* __restrict__ ieee) {
@@ -446,6 +554,18 @@ tfq_status launch_div_selftest(const float* a, const float* b, int64_t n, float*
     div_selftest_kernel<<<static_cast<unsigned>(blocks), threads, 0, stream>>>(a, b, n, ours, ieee);
     const cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? TFQ_OK : fail(TFQ_ECUDA, "self-test launch: %s", cudaGetErrorString(e));
+}
+
+tfq_status launch_quant_mxfp8(const void* x, int64_t rows, int64_t K, void* q, void* sf, cudaStream_t stream,
+                              DeviceState* ds) {
+    if (rows == 0 || K == 0) return TFQ_OK;
+    const int threads = 256;
+    const int64_t warps = (rows * (K / 8) + 32 * kMxJ - 1) / (32 * kMxJ);
+    const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>((warps + 7) / 8, static_cast<int64_t>(ds->sm_count) * 3));  // 80 registers: 3 CTAs per SM
+    quant_mxfp8_kernel<<<static_cast<unsigned>(blocks), threads, 0, stream>>>(
+        static_cast<const uint4*>(x), rows, static_cast<int>(K), static_cast<uint8_t*>(q), static_cast<uint8_t*>(sf));
+    const cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? TFQ_OK : fail(TFQ_ECUDA, "quantizer launch: %s", cudaGetErrorString(e));
 }
 
 tfq_status launch_quant_rows(const void* x, int64_t rows, int64_t K, float qmax, bool out_int8, void* q, float* s,

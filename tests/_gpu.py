@@ -108,3 +108,57 @@ def sample_rows(M: int, n: int, seed: int, tail: int = 128) -> np.ndarray:
     pick = rng.choice(M, size=min(n, M), replace=False)
     last = np.arange(max(0, M - (M % tail or tail)), M)
     return np.unique(np.concatenate([pick, last, [0]])).astype(np.int64)
+
+
+# MXFP8 scale-factor layout (include/tfq.h): 512-byte atoms of 128 rows x 4
+# K blocks, atom (b // 4) * RA + r // 128; inside it row r % 32 owns 16 bytes,
+# (r % 128) // 32 picks the 4-byte word, b % 4 the byte.
+def mx_scale_bytes(R: int, K: int) -> int:
+    return ((R + 127) // 128) * ((K + 127) // 128) * 512
+
+
+def mx_sf_offsets(R: int, K: int) -> np.ndarray:
+    ra = (R + 127) // 128
+    r = np.arange(R, dtype=np.int64)[:, None]
+    b = np.arange(K // 32, dtype=np.int64)[None, :]
+    return ((b // 4) * ra + r // 128) * 512 + (r % 32) * 16 + ((r % 128) // 32) * 4 + b % 4
+
+
+def mx_untile(sf: np.ndarray, R: int, K: int) -> np.ndarray:
+    """Scale buffer in the layout -> row-major [R, K // 32] codes."""
+    return np.asarray(sf)[mx_sf_offsets(R, K)]
+
+
+def mx_tile(codes: np.ndarray, K: int) -> np.ndarray:
+    """Row-major [R, K // 32] codes -> scale buffer (padding entries 127)."""
+    R = codes.shape[0]
+    out = np.full(mx_scale_bytes(R, K), 127, dtype=np.uint8)
+    out[mx_sf_offsets(R, K)] = codes
+    return out
+
+
+def quant_mxfp8(x: torch.Tensor):
+    """GPU MXFP8 quantization through the C ABI; checks guard bytes.
+    Returns (codes [R, K], scale buffer in the layout)."""
+    R, K = x.shape
+    nsf = mx_scale_bytes(R, K)
+    q = guarded(R * K, torch.uint8, 0xA5)
+    sf = guarded(nsf, torch.uint8, 0x5A)
+    st = _capi.raw.tfq_quant_mxfp8(x.data_ptr(), R, K, q.data_ptr(), sf.data_ptr(), stream_handle())
+    assert st == _capi.TFQ_OK, _capi.last_error_message()
+    check_device_error()
+    assert torch.all(q[R * K:] == 0xA5) and torch.all(sf[nsf:] == 0x5A), "write past the end of an output"
+    return q[:R * K].view(R, K), sf[:nsf]
+
+
+def mxfp8_linear(A_q, sf_a, W_q, sf_w, bias):
+    M, K = A_q.shape
+    N = W_q.shape[0]
+    y = guarded(M * N, torch.bfloat16, 7.0)
+    st = _capi.raw.tfq_mxfp8_linear(A_q.data_ptr(), sf_a.data_ptr(), W_q.data_ptr(), sf_w.data_ptr(),
+                                    None if bias is None else bias.data_ptr(), M, N, K, y.data_ptr(),
+                                    stream_handle())
+    assert st == _capi.TFQ_OK, _capi.last_error_message()
+    check_device_error()
+    assert torch.all(y[M * N:] == 7.0), "write past the end of the output"
+    return y[:M * N].view(M, N)

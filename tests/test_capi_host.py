@@ -113,3 +113,35 @@ def test_valid_call_without_gpu_fails_loudly(lib):
 def test_wait_selftest_rejects_bad_limits_before_any_launch(lib):
     assert lib.tfq_selftest_wait_timeout(0, None) == _capi.TFQ_EINVAL
     assert lib.tfq_selftest_wait_timeout(10_000_001, None) == _capi.TFQ_EINVAL
+
+
+def test_mxfp8_scale_bytes(lib):
+    assert lib.tfq_mxfp8_scale_bytes(1, 32) == 512
+    assert lib.tfq_mxfp8_scale_bytes(128, 128) == 512
+    assert lib.tfq_mxfp8_scale_bytes(129, 160) == 2 * 2 * 512
+    assert lib.tfq_mxfp8_scale_bytes(75600, 5120) == 591 * 40 * 512
+    assert lib.tfq_mxfp8_scale_bytes(0, 64) == 0
+    assert lib.tfq_mxfp8_scale_bytes(-1, 64) == -1
+
+
+def test_mxfp8_validation(lib):
+    q = lib.tfq_quant_mxfp8
+    assert q(ALIGNED, 4, 48, ALIGNED, ALIGNED, None) == _capi.TFQ_EINVAL          # K % 32
+    assert q(ALIGNED, -1, 64, ALIGNED, ALIGNED, None) == _capi.TFQ_EINVAL
+    assert q(ALIGNED, 4, 64, ALIGNED, None, None) == _capi.TFQ_EINVAL             # null sf
+    assert q(ALIGNED, 4, 64, ALIGNED, ALIGNED + 4, None) == _capi.TFQ_EINVAL      # misaligned sf
+    assert q(ALIGNED, 4, (1 << 24) + 32, ALIGNED, ALIGNED, None) == _capi.TFQ_EUNSUPPORTED
+    assert q(None, 0, 64, None, None, None) == _capi.TFQ_OK                       # empty: no-op
+    g = lib.tfq_mxfp8_linear
+    assert g(ALIGNED, ALIGNED, ALIGNED, ALIGNED, None, 4, 16, 48, ALIGNED, None) == _capi.TFQ_EINVAL  # K % 32
+    assert g(ALIGNED, ALIGNED, ALIGNED, ALIGNED, None, 4, 12, 64, ALIGNED, None) == _capi.TFQ_EINVAL  # N % 8
+    assert g(ALIGNED, None, ALIGNED, ALIGNED, None, 4, 16, 64, ALIGNED, None) == _capi.TFQ_EINVAL     # null sf_a
+    assert g(ALIGNED, ALIGNED, ALIGNED, ALIGNED + 8, None, 4, 16, 64, ALIGNED, None) == _capi.TFQ_EINVAL
+    assert g(ALIGNED, ALIGNED, ALIGNED, ALIGNED, None, 0, 16, 64, ALIGNED, None) == _capi.TFQ_OK
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU behaviour")
+def test_mxfp8_valid_call_without_gpu_fails_loudly(lib):
+    assert lib.tfq_quant_mxfp8(ALIGNED, 4, 64, ALIGNED, ALIGNED, None) in (_capi.TFQ_ECUDA, _capi.TFQ_EUNSUPPORTED)
+    assert lib.tfq_mxfp8_linear(ALIGNED, ALIGNED, ALIGNED, ALIGNED, None, 4, 16, 64, ALIGNED, None) \
+        in (_capi.TFQ_ECUDA, _capi.TFQ_EUNSUPPORTED)
