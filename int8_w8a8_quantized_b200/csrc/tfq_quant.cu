@@ -347,13 +347,19 @@ __global__ void __launch_bounds__(256, grouped_ctas_per_sm<J>()) quant_grouped_r
 // E + 127 (0 for a block of zeros); q = E4M3_rn_satfinite(x * 2^-E).  The
 // product with the power of two is exact (it only rounds when the result is
 // far below the smallest E4M3 subnormal, where the code is a signed zero
-// anyway), so no division is needed.  The matrix is streamed as a flat
-// sequence of 16-byte units (a 32-element block is 4 units and never crosses
-// a row because K % 32 == 0): lane l of a warp holds units base + l + 32 j,
-// j < kMxJ, so a block sits in 4 adjacent lanes and its maximum takes two
-// shuffles.  Scale codes go to the tensor-core scale-factor layout.
-
-constexpr int kMxJ = 8;  // 16-byte units per lane per iteration: 4 KiB in flight per warp
+// anyway), so no division is needed.
+//
+// The work unit is one 512-byte atom of the scale-factor layout: 128 rows x
+// 128 columns of x (4 blocks per row).  Inside an atom, row r owns the word
+// 4 ((r % 128) / 32) of the 16-byte line r % 32, so the 16 rows
+// {4w .. 4w+3} + {0, 32, 64, 96} own lines 4w .. 4w+3: 64 contiguous bytes.
+// Warp w of a CTA takes exactly those rows, two per load instruction (16
+// lanes x 16 bytes = one row's 128 columns), all 16 in flight at once; a
+// block is 4 adjacent lanes (maximum in two shuffles), and each row's four
+// codes leave as one 32-bit word.  Every line of codes and of scales is thus
+// written whole by one warp -- no partially written sectors for the memory
+// system to merge -- and the padding entries (rows past `rows`, blocks past
+// K / 32) come out of the same loop with code 127.
 
 __device__ __forceinline__ uint32_t e8m0_code(float amax) {
     const uint32_t bits = __float_as_uint(amax);
@@ -383,69 +389,58 @@ __device__ __forceinline__ uint2 quantize8_mx(const uint4& v, float inv) {
     return make_uint2(lo | sign_bytes(v.x, v.y), hi | sign_bytes(v.z, v.w));
 }
 
-// Byte offset of the scale code of (row r, K block b) in the scale-factor
-// layout: 512-byte atoms of 128 rows x 4 blocks, atom (b / 4) * ra + r / 128;
-// inside it row r % 32 owns 16 bytes, (r % 128) / 32 picks the 4-byte word
-// and b % 4 the byte.
-__device__ __forceinline__ int64_t mx_sf_offset(int64_t r, int64_t b, int64_t ra) {
-    return ((b >> 2) * ra + (r >> 7)) * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4 + (b & 3);
-}
+#ifndef TFQ_MX_CTAS
+#define TFQ_MX_CTAS 3  // resident CTAs of 8 warps per SM (~75 registers)
+#endif
 
-__global__ void __launch_bounds__(256) quant_mxfp8_kernel(const uint4* __restrict__ x, int64_t rows, int K,
-                                                          uint8_t* __restrict__ q, uint8_t* __restrict__ sf) {
+__global__ void __launch_bounds__(256, TFQ_MX_CTAS) quant_mxfp8_kernel(const uint4* __restrict__ x, int64_t rows,
+                                                                       int K, uint8_t* __restrict__ q,
+                                                                       uint8_t* __restrict__ sf) {
     const int lane = threadIdx.x & 31;
-    const int nb = K >> 5;  // blocks per row
+    const int warp = threadIdx.x >> 5;  // 0..7
+    const int half = lane >> 4;         // which of the two rows of a load
+    const int lu = lane & 15;           // 16-byte unit within the atom's 128 columns
+    const int units = K >> 3;
+    const int nb = K >> 5;
     const int64_t ra = (rows + 127) >> 7;
-    const int64_t total = rows * static_cast<int64_t>(K >> 3);
-    const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-    const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+    const int ka_n = (K + 127) >> 7;
+    const int64_t tiles = ra * ka_n;
     uint2* q2 = reinterpret_cast<uint2*>(q);
-    for (int64_t base = warp * (32 * kMxJ); base < total; base += nwarps * (32 * kMxJ)) {
-        uint4 v[kMxJ];
+    for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x) {
+        const int64_t rp = t / ka_n;  // 128-row panel
+        const int ka = static_cast<int>(t - rp * ka_n);
+        const int u = ka * 16 + lu;
+        const bool col_ok = u < units;
+        uint4 v[8];
 #pragma unroll
-        for (int j = 0; j < kMxJ; ++j) {
-            const int64_t u = base + lane + 32 * j;
-            v[j] = u < total ? ldg_nc_v4(x + u) : make_uint4(0u, 0u, 0u, 0u);
+        for (int j = 0; j < 8; ++j) {
+            const int ri = 2 * j + half;
+            const int rl = 4 * warp + (ri & 3) + 32 * (ri >> 2);
+            const int64_t r = rp * 128 + rl;
+            v[j] = (r < rows && col_ok) ? ldg_nc_v4(x + r * units + u) : make_uint4(0u, 0u, 0u, 0u);
         }
-        const int64_t blk0 = base >> 2;  // the warp's first block
-        const int64_t r0 = blk0 / nb;
-        const int b0 = static_cast<int>(blk0 - r0 * nb);
+        const bool block_ok = ka * 4 + (lu >> 2) < nb;
+        uint8_t* atom = sf + (static_cast<int64_t>(ka) * ra + rp) * 512;
 #pragma unroll
-        for (int j = 0; j < kMxJ; ++j) {
+        for (int j = 0; j < 8; ++j) {
+            const int ri = 2 * j + half;
+            const int rl = 4 * warp + (ri & 3) + 32 * (ri >> 2);
+            const int64_t r = rp * 128 + rl;
             const uint32_t m = max_abs4(0u, v[j]) & 0x7FFF7FFFu;
             float amax = fmaxf(bf16_lo(m), bf16_hi(m));
             amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
             amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 2));
-            const uint32_t code = e8m0_code(amax);
-            const int64_t u = base + lane + 32 * j;
-            if (u < total) {
-                q2[u] = quantize8_mx(v[j], e8m0_inverse(code));
-                if ((lane & 3) == 0) {
-                    const int d = b0 + (lane >> 2) + 8 * j;  // blocks past the start of row r0
-                    const int dr = d / nb;
-                    sf[mx_sf_offset(r0 + dr, d - dr * nb, ra)] = static_cast<uint8_t>(code);
-                }
-            }
+            const bool row_ok = r < rows;
+            const uint32_t code = (row_ok && block_ok) ? e8m0_code(amax) : 127u;
+            if (row_ok && col_ok) q2[r * units + u] = quantize8_mx(v[j], e8m0_inverse(code));
+            // codes of the row's four blocks (lanes 16 half + 0, 4, 8, 12) -> one word
+            const uint32_t c1 = __shfl_down_sync(0xFFFFFFFFu, code, 4);
+            const uint32_t c2 = __shfl_down_sync(0xFFFFFFFFu, code, 8);
+            const uint32_t c3 = __shfl_down_sync(0xFFFFFFFFu, code, 12);
+            if (lu == 0)
+                *reinterpret_cast<uint32_t*>(atom + 16 * (rl & 31) + 4 * (rl >> 5)) =
+                    code | (c1 << 8) | (c2 << 16) | (c3 << 24);
         }
-    }
-    // Padding entries of the layout (rows past `rows`, blocks past K / 32):
-    // scale code 127 (2^0), so that a padded block multiplies zeros by 1.
-    const int64_t nbp = static_cast<int64_t>((K + 127) >> 7) * 4;
-    const int64_t n1 = (ra * 128 - rows) * nbp;
-    const int64_t n2 = rows * (nbp - nb);
-    const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-    const int64_t nthreads = static_cast<int64_t>(gridDim.x) * blockDim.x;
-    for (int64_t i = tid; i < n1 + n2; i += nthreads) {
-        int64_t r, b;
-        if (i < n1) {
-            r = rows + i / nbp;
-            b = i % nbp;
-        } else {
-            const int64_t w = nbp - nb, k = i - n1;
-            r = k / w;
-            b = nb + k % w;
-        }
-        sf[mx_sf_offset(r, b, ra)] = 127;
     }
 }
 
@@ -559,10 +554,9 @@ tfq_status launch_div_selftest(const float* a, const float* b, int64_t n, float*
 tfq_status launch_quant_mxfp8(const void* x, int64_t rows, int64_t K, void* q, void* sf, cudaStream_t stream,
                               DeviceState* ds) {
     if (rows == 0 || K == 0) return TFQ_OK;
-    const int threads = 256;
-    const int64_t warps = (rows * (K / 8) + 32 * kMxJ - 1) / (32 * kMxJ);
-    const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>((warps + 7) / 8, static_cast<int64_t>(ds->sm_count) * 3));  // 80 registers: 3 CTAs per SM
-    quant_mxfp8_kernel<<<static_cast<unsigned>(blocks), threads, 0, stream>>>(
+    const int64_t tiles = ((rows + 127) / 128) * ((K + 127) / 128);
+    const int64_t blocks = std::min<int64_t>(tiles, static_cast<int64_t>(ds->sm_count) * TFQ_MX_CTAS);
+    quant_mxfp8_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
         static_cast<const uint4*>(x), rows, static_cast<int>(K), static_cast<uint8_t*>(q), static_cast<uint8_t*>(sf));
     const cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? TFQ_OK : fail(TFQ_ECUDA, "quantizer launch: %s", cudaGetErrorString(e));
