@@ -31,7 +31,7 @@ struct DeviceState {
     unsigned* round_ctrs = nullptr;
     int round_slots = 0;
     int next_round_slot = 0;
-    bool gemm_attr_set[4] = {false, false, false, false};  // FP8, INT8, FP8 with FP16 accumulator, MXFP8
+    bool gemm_attr_set[5] = {false, false, false, false, false};  // FP8, INT8, FP8/FP16 acc, MXFP8, MXFP8 pair
 };
 
 // Per-device state of the current device, created on first use.  Returns

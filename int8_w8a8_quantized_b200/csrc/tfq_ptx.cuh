@@ -358,6 +358,26 @@ __device__ __forceinline__ void tmem_cp_32x128b_warpx4(uint32_t taddr, uint64_t 
     asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
 }
 
+// The same for a CTA pair (cta_group::2), issued by the even CTA: the MMA
+// reads A and the A scales of each CTA from that CTA, and B from both; every
+// CTA's TMEM holds the B scales of all N columns of the tile.
+__device__ __forceinline__ void mma_mxf8_block_scaled_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                                           uint32_t idesc, uint32_t sfa, uint32_t sfb,
+                                                           uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+        : "memory");
+}
+
+// tmem_cp_32x128b_warpx4 for a CTA pair: in each CTA of the pair, from that
+// CTA's shared memory at the descriptor's offset into its own TMEM.
+__device__ __forceinline__ void tmem_cp_32x128b_warpx4_pair(uint32_t taddr, uint64_t sdesc) {
+    asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
 // Shared-memory descriptor of an unswizzled K-major block of rows 16 bytes
 // wide, stored contiguously: 8-row core matrices 128 bytes apart (stride
 // byte offset), a single core-matrix column (leading byte offset unused).
