@@ -44,6 +44,8 @@ def metric_name(dtype: str) -> str:
         return METRIC.replace("FP8", "INT8").replace("TFLOP/s", "TOPS")
     if dtype == "fp8_f16acc":
         return METRIC.replace("scaled-FP8 Linear", "scaled-FP8 Linear (FP16 accumulator)")
+    if dtype == "mxfp8":
+        return METRIC.replace("scaled-FP8 Linear", "MXFP8 Linear (E4M3, E8M0 scale per 32 values)")
     return METRIC
 
 
@@ -59,9 +61,9 @@ def parse_args():
     ap.add_argument("--workload", default="video_dit_block",
                     choices=["video_dit_block", "image_dit_block", "reduced_qmax_ffn_out", "tiny_w8a8_linear"])
     ap.add_argument("--impl", default="tfq", choices=["tfq", "reference"])
-    ap.add_argument("--dtype", default="fp8", choices=["fp8", "int8", "fp8_f16acc"],
+    ap.add_argument("--dtype", default="fp8", choices=["fp8", "int8", "fp8_f16acc", "mxfp8"],
                     help="fp8: E4M3 W8A8 (the headline); int8: the INT8 W8A8 path; "
-                         "fp8_f16acc: E4M3 with an FP16 accumulator")
+                         "fp8_f16acc: E4M3 with an FP16 accumulator; mxfp8: E4M3 with block-32 E8M0 scales")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -190,7 +192,13 @@ def aggregate_throughput(world: int, flops_per_step: int, ms_per_step_max: float
 
 # ------------------------------------------------------------ GPU arm
 def act_qmaxes(wl, dtype):
-    return (127.0,) if dtype == "int8" else wl.act_qmax
+    """Activation quantization passes per step: one per qmax; INT8 uses 127,
+    MXFP8 has no qmax (its scale comes from each block's exponent)."""
+    if dtype == "int8":
+        return (127.0,)
+    if dtype == "mxfp8":
+        return (0.0,)
+    return wl.act_qmax
 
 
 def build_block(wl, dev, dtype="fp8"):
@@ -198,16 +206,25 @@ def build_block(wl, dev, dtype="fp8"):
     import torch
     from int8_w8a8_quantized_b200 import tfq_quant_weight_per_channel
 
+    from int8_w8a8_quantized_b200 import tfq_mxfp8_scale_bytes, tfq_quant_mxfp8
     xs = {name: wl.make_x(name, device=dev) for name in sorted(wl.x_shapes())}
     lins = []
     for lin in wl.linears:
         w = wl.make_w(lin, device=dev)
-        wdt = "int8" if dtype == "int8" else "fp8"
-        Wq, sw = tfq_quant_weight_per_channel(w, wdt, 127.0 if dtype == "int8" else 448.0)
+        if dtype == "mxfp8":
+            Wq, sw = tfq_quant_mxfp8(w)
+        else:
+            wdt = "int8" if dtype == "int8" else "fp8"
+            Wq, sw = tfq_quant_weight_per_channel(w, wdt, 127.0 if dtype == "int8" else 448.0)
         del w
         b = wl.make_bias(lin, device=dev)
         lins.append((lin, Wq, sw, b))
-    aq = {(name, q): (torch.empty_like(x, dtype=torch.uint8), torch.empty(x.shape[0], device=dev))
+
+    def act_scales(x):
+        if dtype == "mxfp8":  # E8M0 codes in the tensor-core scale layout
+            return torch.empty(tfq_mxfp8_scale_bytes(x.shape[0], x.shape[1]), dtype=torch.uint8, device=dev)
+        return torch.empty(x.shape[0], device=dev)
+    aq = {(name, q): (torch.empty_like(x, dtype=torch.uint8), act_scales(x))
           for name, x in xs.items() for q in act_qmaxes(wl, dtype)}
     ys = {(lin.name, q): torch.empty((wl.M, lin.N), dtype=torch.bfloat16, device=dev)
           for lin in wl.linears for q in act_qmaxes(wl, dtype)}
@@ -227,9 +244,14 @@ def gpu_arm(args, wl, rank, world, local_rank):
     sh = int(stream.cuda_stream)
     xs, lins, aq, ys = build_block(wl, dev, args.dtype)
     qmaxes = act_qmaxes(wl, args.dtype)
-    quant_fn = lib.tfq_quant_act_int8_per_token if args.dtype == "int8" else lib.tfq_quant_act_fp8_per_token
+    if args.dtype == "mxfp8":
+        def quant_fn(x, M, K, q, A, sf, s):
+            return lib.tfq_quant_mxfp8(x, M, K, A, sf, s)
+    else:
+        quant_fn = lib.tfq_quant_act_int8_per_token if args.dtype == "int8" else lib.tfq_quant_act_fp8_per_token
     gemm_fn = {"fp8": lib.tfq_scaled_fp8_linear, "int8": lib.tfq_scaled_int8_linear,
-               "fp8_f16acc": lib.tfq_scaled_fp8_linear_f16acc}[args.dtype]
+               "fp8_f16acc": lib.tfq_scaled_fp8_linear_f16acc, "mxfp8": lib.tfq_mxfp8_linear}[args.dtype]
+    mx = args.dtype == "mxfp8"
 
     # per-kernel events, recorded on the launching stream
     ev = {"quant": [], "gemm": []}
@@ -250,8 +272,9 @@ def gpu_arm(args, wl, rank, world, local_rank):
                 launches[0] += 1
                 if record:
                     e1 = torch.cuda.Event(enable_timing=True); e1.record(stream)
-                    # algorithmic bytes: read bf16, write e4m3 codes, 4 B of scale per row
-                    ev["quant"].append((e0, e1, 3 * x.numel() + 4 * x.shape[0]))
+                    # algorithmic bytes: read bf16, write 8-bit codes, 4 B of scale per row
+                    # (MXFP8: 1 B of scale per 32 values)
+                    ev["quant"].append((e0, e1, 3 * x.numel() + (x.numel() // 32 if mx else 4 * x.shape[0])))
             for lin, Wq, sw, b in lins:
                 A, sa = aq[(lin.x, q)]
                 y = ys[(lin.name, q)]
@@ -292,7 +315,10 @@ def gpu_arm(args, wl, rank, world, local_rank):
     gemm_ms = [a.elapsed_time(b) for a, b, _ in ev["gemm"]]
     quant_ms = [a.elapsed_time(b) for a, b, _ in ev["quant"]]
     gemm_flops = [2 * m * n * k for _, _, (m, n, k) in ev["gemm"]]
-    gemm_bytes = [m * k + n * k + 2 * m * n + 4 * m + 6 * n for _, _, (m, n, k) in ev["gemm"]]
+    if mx:  # codes, block scales (1 B per 32 values of each operand), bf16 output, bias
+        gemm_bytes = [m * k + n * k + (m + n) * k // 32 + 2 * m * n + 2 * n for _, _, (m, n, k) in ev["gemm"]]
+    else:
+        gemm_bytes = [m * k + n * k + 2 * m * n + 4 * m + 6 * n for _, _, (m, n, k) in ev["gemm"]]
     quant_bytes = [nbytes for _, _, nbytes in ev["quant"]]
     out = {
         "ms_per_step": ms_per_step,
@@ -415,15 +441,21 @@ def oracle_sample(wl, seconds: float, seed: int = 0, dtype: str = "fp8"):
             if key not in cache:
                 w = wl.make_w(lin)
                 wbits = w.contiguous().view(torch.int16).numpy().view(np.uint16)
-                Wq, sw = oracle.quant_rows_int8(wbits) if dtype == "int8" else oracle.quant_rows_fp8(wbits, 448.0)
+                if dtype == "mxfp8":
+                    Wq, sw = oracle.quant_mxfp8(wbits)
+                else:
+                    Wq, sw = oracle.quant_rows_int8(wbits) if dtype == "int8" else oracle.quant_rows_fp8(wbits, 448.0)
                 b = wl.make_bias(lin)
                 bbits = None if b is None else b.contiguous().view(torch.int16).numpy().view(np.uint16)
                 cache[key] = (Wq, sw, bbits)
             Wq, sw, bbits = cache[key]
             x = _x_rows(wl, lin, rows_per_linear, int(rng.integers(1 << 30)))
-            for q in ((127.0,) if dtype == "int8" else wl.act_qmax):
+            for q in act_qmaxes(wl, dtype):
                 t0 = time.perf_counter()
-                if dtype != "int8":  # the oracle's GEMM accumulates exactly for both FP8 variants
+                if dtype == "mxfp8":
+                    A, sa = oracle.quant_mxfp8(x)
+                    oracle.mxfp8_linear(A, sa, Wq, sw, bbits)
+                elif dtype != "int8":  # the oracle's GEMM accumulates exactly for both FP8 variants
                     A, sa = oracle.quant_rows_fp8(x, q)
                     oracle.scaled_fp8_linear(A, sa, Wq, sw, bbits)
                 else:
@@ -465,7 +497,9 @@ def main():
     wl = workloads.WORKLOADS[args.workload]
     cfg = {"workload": wl.name, "M": wl.M, "dtype": args.dtype,
            "linears": [f"{l.name}:{l.K}->{l.N}" for l in wl.linears],
-           "act_qmax": list(wl.act_qmax), "weight_qmax": 448.0, "bias": wl.has_bias,
+           "act_qmax": list(wl.act_qmax) if args.dtype != "mxfp8" else "none (E8M0 scale per 32 values)",
+           "weight_qmax": 448.0 if args.dtype != "mxfp8" else "none (E8M0 scale per 32 values)",
+           "bias": wl.has_bias,
            "l2": "inputs larger than L2 (126 MB)" if wl.M * min(l.K for l in wl.linears) * 2 > L2_BYTES
            else "working set of one step larger than L2; no flush",
            "parallelism": f"replicas x{world}"}
@@ -501,7 +535,12 @@ def main():
     bf16_burst = peaks.get("bf16_tflops", FALLBACK_BF16_TFLOPS)
     fp8_peak = bf16_sus * FP8_OVER_BF16
     pair = wl.M >= 512
-    kname = ("scaled_mm_pair_kernel" if pair else "scaled_mm_kernel") + f"<{args.dtype}>"
+    if args.dtype == "mxfp8":
+        kname = "mxfp8_mm_pair_kernel" if pair else "mxfp8_mm_kernel"
+        qname = "quant_mxfp8_kernel"
+    else:
+        kname = ("scaled_mm_pair_kernel" if pair else "scaled_mm_kernel") + f"<{args.dtype}>"
+        qname = "quant_rows_kernel<" + args.dtype + ">"
     quant_gbs = res["quant_bytes_total"] / (res["quant_ms_total"] * 1e-3) / 1e9 if res["quant_ms_total"] else None
     line = {
         "metric": metric_name(args.dtype),
@@ -515,7 +554,8 @@ def main():
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": {"fp8": "e4m3", "int8": "s8", "fp8_f16acc": "e4m3 (f16 accumulate)"}[args.dtype],
+        "dtype": {"fp8": "e4m3", "int8": "s8", "fp8_f16acc": "e4m3 (f16 accumulate)",
+                  "mxfp8": "e4m3 (e8m0 block-32 scales)"}[args.dtype],
         "data": "synthetic",
         "config": cfg,
         "roofline": {
@@ -533,7 +573,7 @@ def main():
             "frac_of_fp8_spec": round(gemm_tflops / FP8_SPEC_TFLOPS, 4),
         },
         "quantizer": {
-            "kernel": "quant_rows_kernel<" + args.dtype + ">",
+            "kernel": qname,
             "bound": "hbm",
             "achieved": None if quant_gbs is None else round(quant_gbs, 1),
             "peak": peaks.get("hbm_gbs", FALLBACK_HBM_GBS),
