@@ -72,8 +72,10 @@ def parse_args():
 
 
 KERNEL_SOURCES = {
-    "gemm": ("int8_w8a8_quantized_b200/csrc/tfq_gemm.cu", "int8_w8a8_quantized_b200/csrc/tfq_ptx.cuh"),
-    "quant": ("int8_w8a8_quantized_b200/csrc/tfq_quant.cu", "int8_w8a8_quantized_b200/csrc/tfq_ptx.cuh"),
+    "gemm": ("int8_w8a8_quantized_b200/csrc/tfq_gemm.cu", "int8_w8a8_quantized_b200/csrc/tfq_gemm_common.cuh",
+             "int8_w8a8_quantized_b200/csrc/tfq_ptx.cuh"),
+    "quant": ("int8_w8a8_quantized_b200/csrc/tfq_quant.cu", "int8_w8a8_quantized_b200/csrc/tfq_quant_common.cuh",
+              "int8_w8a8_quantized_b200/csrc/tfq_ptx.cuh"),
 }
 TRAFFIC_RECORD = os.path.join(ROOT, "profiles", "roofline_traffic_video_dit_block.md")
 

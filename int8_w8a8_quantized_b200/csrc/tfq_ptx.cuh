@@ -333,57 +333,4 @@ __device__ __forceinline__ uint64_t sw128_kmajor_desc(const void* smem_tile) {
     return ((addr >> 4) & 0x3FFFull) | (1ull << 16) | ((1024ull >> 4) << 32) | (1ull << 46) | (2ull << 61);
 }
 
-// Block-scaled MMA (MXFP8: E4M3 x E4M3, one E8M0 scale per 32 elements of K
-// for every row of A and of B), single CTA.  sfa / sfb are TMEM addresses of
-// the scale factors; their top two bits select the byte of each 32-bit TMEM
-// cell (the scale of K block 0..3 of the stage), and must equal the scale
-// factor ids carried in idesc.
-__device__ __forceinline__ void mma_mxf8_block_scaled(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                                      uint32_t idesc, uint32_t sfa, uint32_t sfb,
-                                                      uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
-        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
-        : "memory");
-}
-
-// Copies 32 rows x 16 bytes of shared memory (row r at byte 16 r) into TMEM
-// lanes 0..31, columns taddr..taddr+3, and the same data into lanes 32..63,
-// 64..95 and 96..127 (the .warpx4 broadcast): the scale-factor staging of a
-// block-scaled MMA.  Issued by the thread that issues the MMAs; it is
-// ordered before them.
-__device__ __forceinline__ void tmem_cp_32x128b_warpx4(uint32_t taddr, uint64_t sdesc) {
-    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
-}
-
-// The same for a CTA pair (cta_group::2), issued by the even CTA: the MMA
-// reads A and the A scales of each CTA from that CTA, and B from both; every
-// CTA's TMEM holds the B scales of all N columns of the tile.
-__device__ __forceinline__ void mma_mxf8_block_scaled_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                                           uint32_t idesc, uint32_t sfa, uint32_t sfb,
-                                                           uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::2.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
-        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
-        : "memory");
-}
-
-// tmem_cp_32x128b_warpx4 for a CTA pair: in each CTA of the pair, from that
-// CTA's shared memory at the descriptor's offset into its own TMEM.
-__device__ __forceinline__ void tmem_cp_32x128b_warpx4_pair(uint32_t taddr, uint64_t sdesc) {
-    asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
-}
-
-// Shared-memory descriptor of an unswizzled K-major block of rows 16 bytes
-// wide, stored contiguously: 8-row core matrices 128 bytes apart (stride
-// byte offset), a single core-matrix column (leading byte offset unused).
-__device__ __forceinline__ uint64_t plain_rows16_desc(const void* smem_rows) {
-    const uint64_t addr = smem_u32(smem_rows);
-    return ((addr >> 4) & 0x3FFFull) | ((128ull >> 4) << 32) | (1ull << 46);
-}
-
 }  // namespace tfq
