@@ -17,6 +17,7 @@ enum : uint32_t {
     kErrGemmEpilogue = 1u << 6,
     kErrGemmDrain = 1u << 7,
     kErrSelfTest = 1u << 8,
+    kErrQuantStage = 1u << 9,  // a staged-row quantizer gave up waiting for a row load
 };
 
 struct DeviceState {
@@ -32,6 +33,7 @@ struct DeviceState {
     int round_slots = 0;
     int next_round_slot = 0;
     bool gemm_attr_set[5] = {false, false, false, false, false};  // FP8, INT8, FP8/FP16 acc, MXFP8, MXFP8 pair
+    bool quant_attr_set = false;   // dynamic shared memory limit of the staged-row quantizers
 };
 
 // Per-device state of the current device, created on first use.  Returns

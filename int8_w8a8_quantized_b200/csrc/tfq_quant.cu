@@ -232,6 +232,116 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(const uint4* __restrict
     }
 }
 
+// Rows of 16384 <= K <= TFQ_QUANT_STAGED_MAX_K: the row is staged in shared
+// memory.  (Measured on B200: below K = 16384 the one-warp-per-row loop above
+// is as fast or faster inside the DiT block -- staging its K = 13824
+// activation made the block's quantizers 6 % slower, though that row length
+// ran 10 % faster alone -- while for K >= 16384 staging is 20 to 35 % faster
+// alone.)  A CTA of
+// 256 threads quantizes one row at a time while the TMA
+// engine brings its next rows (one bulk copy of a whole row into each of 2 to
+// 4 row buffers, completion counted on that buffer's mbarrier).  Pass 1
+// reduces max |x| over the buffer (warp shuffles, then the 8 warp maxima
+// through shared memory), pass 2 quantizes from the same buffer.  HBM sees the
+// row read once and L2 carries it once; the one-warp-per-row loop above reads
+// rows longer than one segment twice from L2.
+#ifndef TFQ_QUANT_STAGED_MAX_K
+#define TFQ_QUANT_STAGED_MAX_K 32768  // two row buffers of 2 K bytes: 128 KiB at this K
+#endif
+#ifndef TFQ_QUANT_STAGED_MIN_K
+#define TFQ_QUANT_STAGED_MIN_K 16384  // shorter rows: grouped kernel or one warp per row
+#endif
+constexpr int kStagedThreads = 256;
+constexpr int kStagedMaxSlots = 4;
+constexpr int kStagedSmemLimit = 200 * 1024;
+#ifndef TFQ_QUANT_STAGED_SLOT_BYTES
+#define TFQ_QUANT_STAGED_SLOT_BYTES (96 * 1024)  // row buffers per CTA: as many as fit here, 2 to 4
+#endif
+
+template <bool kInt8, bool kClamp>
+__global__ void __launch_bounds__(kStagedThreads) quant_rows_staged_kernel(const uint4* __restrict__ x, int64_t M,
+                                                                           int K, int slots, float qmax,
+                                                                           uint8_t* __restrict__ q,
+                                                                           float* __restrict__ s, uint32_t* err) {
+    extern __shared__ __align__(128) uint8_t staged_smem[];
+    __shared__ uint64_t bar[kStagedMaxSlots];
+    __shared__ float wmax[kStagedThreads / 32];
+    __shared__ int abort_flag;
+    const int tid = threadIdx.x;
+    const int lane = tid & 31;
+    const int warp = tid >> 5;
+    const int units = K >> 3;
+    const uint32_t row_bytes = static_cast<uint32_t>(K) * 2u;
+    const int64_t stride = gridDim.x;
+    if (tid == 0) {
+        for (int i = 0; i < slots; ++i) mbar_init(&bar[i], 1);
+        abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (tid == 0) {
+        for (int i = 0; i < slots; ++i) {
+            const int64_t r = blockIdx.x + i * stride;
+            if (r < M) {
+                mbar_arrive_expect_tx(&bar[i], row_bytes);
+                bulk_g2s(staged_smem + static_cast<size_t>(i) * row_bytes, x + r * units, row_bytes, &bar[i]);
+            }
+        }
+    }
+    int it = 0;
+    for (int64_t r = blockIdx.x; r < M; r += stride, ++it) {
+        const int sl = it % slots;
+        const uint32_t ph = static_cast<uint32_t>(it / slots) & 1u;
+        if (tid == 0 && !mbar_wait(&bar[sl], ph, &abort_flag)) {
+            abort_flag = 1;
+            atomicOr(err, kErrQuantStage);
+        }
+        __syncthreads();
+        if (abort_flag) break;
+        (void)mbar_try_wait(&bar[sl], ph);  // completed: makes the copied row visible to this thread
+        const uint4* row = reinterpret_cast<const uint4*>(staged_smem + static_cast<size_t>(sl) * row_bytes);
+        uint32_t m = 0;
+        for (int u = tid; u < units; u += kStagedThreads) m = max_abs4(m, row[u]);
+        m &= 0x7FFF7FFFu;
+        float amax = fmaxf(bf16_lo(m), bf16_hi(m));
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+        if (lane == 0) wmax[warp] = amax;
+        __syncthreads();
+        amax = wmax[0];
+#pragma unroll
+        for (int w = 1; w < kStagedThreads / 32; ++w) amax = fmaxf(amax, wmax[w]);
+        const float sc = __fdiv_rn(fmaxf(amax, 1e-12f), qmax);
+        if (tid == 0) s[r] = sc;
+        uint2* qrow = reinterpret_cast<uint2*>(q + r * K);
+        if (sc <= 0x1p125f) {
+            const float rcp = __frcp_rn(sc);
+            for (int u = tid; u < units; u += kStagedThreads)
+                qrow[u] = quantize8<kInt8, kClamp, false>(row[u], sc, rcp, qmax);
+        } else {  // reciprocal would be subnormal: IEEE division (uniform across the CTA)
+            for (int u = tid; u < units; u += kStagedThreads)
+                qrow[u] = quantize8<kInt8, kClamp, true>(row[u], sc, 0.0f, qmax);
+        }
+        __syncthreads();  // every thread is done with this buffer and with wmax
+        if (tid == 0) {
+            const int64_t rn = r + slots * stride;
+            if (rn < M) {
+                mbar_arrive_expect_tx(&bar[sl], row_bytes);
+                bulk_g2s(staged_smem + static_cast<size_t>(sl) * row_bytes, x + rn * units, row_bytes, &bar[sl]);
+            }
+        }
+    }
+    // After giving up, the copies still in flight must land (bounded) before
+    // this CTA's shared memory is released.
+    if (abort_flag && tid == 0) {
+        for (int k = 0; k < slots; ++k) {
+            const int j = it + k;
+            if (blockIdx.x + static_cast<int64_t>(j) * stride < M)
+                (void)mbar_wait(&bar[j % slots], static_cast<uint32_t>(j / slots) & 1u, nullptr);
+        }
+    }
+}
+
 #ifndef TFQ_QUANT_J4_CTAS
 #define TFQ_QUANT_J4_CTAS 4  // resident CTAs of 8 warps per SM for the grouped kernel with 4 units per lane
 #endif
@@ -410,6 +520,38 @@ tfq_status launch_div_selftest(const float* a, const float* b, int64_t n, float*
     return e == cudaSuccess ? TFQ_OK : fail(TFQ_ECUDA, "self-test launch: %s", cudaGetErrorString(e));
 }
 
+namespace {
+
+tfq_status launch_staged_rows(const void* x, int64_t rows, int64_t K, float qmax, bool out_int8, bool clamp, void* q,
+                              float* s, cudaStream_t stream, DeviceState* ds) {
+    auto kernel = out_int8 ? quant_rows_staged_kernel<true, false>
+                           : (clamp ? quant_rows_staged_kernel<false, true> : quant_rows_staged_kernel<false, false>);
+    if (!ds->quant_attr_set) {
+        const void* fns[3] = {reinterpret_cast<const void*>(quant_rows_staged_kernel<true, false>),
+                              reinterpret_cast<const void*>(quant_rows_staged_kernel<false, true>),
+                              reinterpret_cast<const void*>(quant_rows_staged_kernel<false, false>)};
+        for (const void* f : fns) {
+            const cudaError_t e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, kStagedSmemLimit);
+            if (e != cudaSuccess) return fail(TFQ_ECUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+        }
+        ds->quant_attr_set = true;
+    }
+    const int slots = static_cast<int>(std::min<int64_t>(
+        kStagedMaxSlots, std::max<int64_t>(2, TFQ_QUANT_STAGED_SLOT_BYTES / (2 * K))));
+    const size_t smem = static_cast<size_t>(slots) * 2 * static_cast<size_t>(K);
+    int per_sm = 0;
+    const cudaError_t eo = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kStagedThreads, smem);
+    if (eo != cudaSuccess || per_sm < 1) return fail(TFQ_ECUDA, "staged quantizer occupancy: %s", cudaGetErrorString(eo));
+    const int64_t blocks = std::min<int64_t>(rows, static_cast<int64_t>(ds->sm_count) * per_sm);
+    kernel<<<static_cast<unsigned>(blocks), kStagedThreads, smem, stream>>>(
+        static_cast<const uint4*>(x), rows, static_cast<int>(K), slots, qmax, static_cast<uint8_t*>(q), s,
+        ds->err_word);
+    const cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? TFQ_OK : fail(TFQ_ECUDA, "quantizer launch: %s", cudaGetErrorString(e));
+}
+
+}  // namespace
+
 tfq_status launch_quant_rows(const void* x, int64_t rows, int64_t K, float qmax, bool out_int8, void* q, float* s,
                              cudaStream_t stream, DeviceState* ds) {
     if (rows == 0) return TFQ_OK;
@@ -422,6 +564,8 @@ tfq_status launch_quant_rows(const void* x, int64_t rows, int64_t K, float qmax,
     }
     const bool clamp = !out_int8 && !is_e4m3_value(qmax);
     if (K / 8 <= kGroupMaxUnits) return launch_grouped_rows(x, rows, K, qmax, out_int8, clamp, q, s, stream, ds);
+    if (K >= TFQ_QUANT_STAGED_MIN_K && K <= TFQ_QUANT_STAGED_MAX_K)
+        return launch_staged_rows(x, rows, K, qmax, out_int8, clamp, q, s, stream, ds);
     auto kernel = out_int8 ? quant_rows_kernel<true, false>
                            : (clamp ? quant_rows_kernel<false, true> : quant_rows_kernel<false, false>);
     const int threads = 256;  // 8 warps, one row per warp at a time

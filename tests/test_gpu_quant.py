@@ -34,7 +34,8 @@ def test_tiny_config_activation():
 
 @pytest.mark.parametrize("qmax", [448.0, 14.0, 7.0, 21.0, 100.0, 12.0])
 @pytest.mark.parametrize("M,K", [(1, 16), (3, 48), (37, 256), (129, 1024), (65, 3072), (33, 5120),
-                                 (17, 12288), (9, 13824), (5, 32768), (300, 160), (3, 65536), (2, 100000)])
+                                 (17, 12288), (9, 13824), (7, 16384), (130, 20480), (5, 32768), (300, 160), (3, 65536),
+                                 (2, 100000)])
 def test_ragged_shapes(M, K, qmax):
     """qmax 21 and 100 are not E4M3 numbers (21 is the midpoint of 20 and
     22): the kernel clamps x/s there; for the others it needs no clamp."""
@@ -66,7 +67,7 @@ def test_weight_fp8_per_channel(qmax):
     np.testing.assert_array_equal(q.cpu().numpy(), q_ref)
 
 
-@pytest.mark.parametrize("K", [16, 256, 5120, 13824])
+@pytest.mark.parametrize("K", [16, 256, 5120, 13824, 16384, 24576])
 def test_int8_ragged(K):
     x = workloads.activations(77, K, seed=K, nu=4, outlier_cols=3, outlier_mult=20.0, zero_rows=2, device="cuda")
     q, s = _gpu.quant_weight(x, _capi.TFQ_DTYPE_INT8, 127.0)
@@ -94,11 +95,13 @@ def test_rounding_edges():
         _assert_fp8_equal(x, qmax)
 
 
+@pytest.mark.parametrize("K", [256, 5120, 16384])
 @pytest.mark.parametrize("qmax", [1.0, 2.0, 448.0])
-def test_huge_magnitude_rows(qmax):
+def test_huge_magnitude_rows(qmax, K):
     """Rows near the bf16 maximum: with a small qmax the scale exceeds 2^125
-    and the kernel takes its IEEE-division branch for the row."""
-    x = workloads.activations(40, 256, seed=3, device="cuda").float()
+    and the kernel takes its IEEE-division branch for the row (grouped,
+    one-warp-per-row and shared-memory-staged kernels)."""
+    x = workloads.activations(40, K, seed=3, device="cuda").float()
     x[:20] *= 3.0e38 / x[:20].abs().amax(dim=1, keepdim=True)
     x[20:30] *= 1.0e30
     x = x.to(torch.bfloat16)
