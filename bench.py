@@ -116,17 +116,58 @@ def measured_peaks():
 
 # ---------------------------------------------------------------- clocks
 class ClockSampler:
-    """nvidia-smi clocks / throttle reasons sampled every 200 ms."""
+    """SM clock, power and clock-event reasons sampled during the timed region:
+    through NVML every 10 ms from a background thread (so that even a timed
+    region of a few milliseconds has samples), else nvidia-smi every 200 ms."""
     QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASON_BITS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
+                   "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80}
 
     def __init__(self, gpu_index: int):
         self.gpu = gpu_index
         self.proc = None
         self.path = None
+        self.nvml = None
+        self.thread = None
+        self.samples = []
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            handle = None
+            props = torch.cuda.get_device_properties(gpu_index)
+            try:  # the NVML device with this CUDA device's PCI address
+                bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+                handle = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+            except Exception:
+                handle = pynvml.nvmlDeviceGetHandleByIndex(gpu_index)
+            self.nvml = (pynvml, handle)
+        except Exception:
+            self.nvml = None
+
+    def _poll(self):
+        import time as _t
+        pynvml, h = self.nvml
+        reasons_fn = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            pynvml.nvmlDeviceGetCurrentClocksThrottleReasons
+        while not self.stop_flag:
+            try:
+                self.samples.append((pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM),
+                                     pynvml.nvmlDeviceGetPowerUsage(h) / 1000.0, int(reasons_fn(h))))
+            except Exception:
+                pass
+            _t.sleep(0.01)
 
     def start(self):
+        if self.nvml is not None:
+            import threading
+            self.stop_flag = False
+            self.samples = []
+            self.thread = threading.Thread(target=self._poll, daemon=True)
+            self.thread.start()
+            return
         try:
             fd, self.path = tempfile.mkstemp(prefix="clocks", suffix=".csv")
             os.close(fd)
@@ -138,6 +179,21 @@ class ClockSampler:
             self.proc = None
 
     def stop(self):
+        if self.thread is not None:
+            self.stop_flag = True
+            self.thread.join(timeout=5)
+            self.thread = None
+            pynvml, h = self.nvml
+            try:
+                sm_max = float(pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM))
+            except Exception:
+                sm_max = None
+            if not self.samples:
+                return None
+            reasons = sorted(n for n, bit in self.REASON_BITS.items() if any(r & bit for _, _, r in self.samples))
+            return {"sm_mhz": statistics.median(c for c, _, _ in self.samples), "sm_max_mhz": sm_max,
+                    "power_w_max": max(p for _, p, _ in self.samples), "samples": len(self.samples),
+                    "source": "nvml, 10 ms", "reasons": reasons}
         if self.proc is None:
             return None
         self.proc.terminate()
@@ -172,6 +228,7 @@ class ClockSampler:
                 "sm_max_mhz": num(rows[0][2]),
                 "power_w_max": max(pw) if pw else None,
                 "samples": len(rows),
+                "source": "nvidia-smi, 200 ms",
                 "reasons": sorted(reasons)}
 
 
