@@ -59,7 +59,10 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=30)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="video_dit_block",
-                    choices=["video_dit_block", "image_dit_block", "reduced_qmax_ffn_out", "tiny_w8a8_linear"])
+                    choices=["video_dit_block", "image_dit_block", "reduced_qmax_ffn_out", "tiny_w8a8_linear",
+                             "activation_quantizer"],
+                    help="activation_quantizer: X [8192, 3072] (1 %% outlier columns x50, 16 zero rows) quantized "
+                         "per token to FP8 (448) and per row to INT8 (127); reports GB/s")
     ap.add_argument("--impl", default="tfq", choices=["tfq", "reference"])
     ap.add_argument("--dtype", default="fp8", choices=["fp8", "int8", "fp8_f16acc", "mxfp8"],
                     help="fp8: E4M3 W8A8 (the headline); int8: the INT8 W8A8 path; "
@@ -381,6 +384,7 @@ def gpu_arm(args, wl, rank, world, local_rank):
     quant_bytes = [nbytes for _, _, nbytes in ev["quant"]]
     out = {
         "ms_per_step": ms_per_step,
+        "gemm_flops_each": gemm_flops, "gemm_bytes_each": gemm_bytes,
         "gemm_ms_total": sum(gemm_ms), "gemm_flops_total": sum(gemm_flops), "gemm_bytes_total": sum(gemm_bytes),
         "quant_ms_total": sum(quant_ms), "quant_bytes_total": sum(quant_bytes),
         "gemm_launches": len(gemm_ms), "quant_launches": len(quant_ms),
@@ -546,13 +550,185 @@ def cpu_baseline(wl, seconds, dtype="fp8"):
             "sample": desc, "seconds": secs}
 
 
+def path_roofline(res, steps, peaks, fp8_peak):
+    """Floor of one step: every quantizer at the measured HBM copy bandwidth plus
+    every GEMM at max(FLOPs / tensor peak, bytes / HBM bandwidth), against the
+    measured step time; with the measured sustained 8-bit peak and with the
+    4.5 PFLOP/s spec."""
+    hbm = peaks.get("hbm_gbs", FALLBACK_HBM_GBS) * 1e9
+    q_s = res["quant_bytes_total"] / hbm
+    per_launch = [(f, b) for f, b in zip(res["gemm_flops_each"], res["gemm_bytes_each"])]
+
+    def floor_ms(peak_tflops):
+        g_s = sum(max(f / (peak_tflops * 1e12), b / hbm) for f, b in per_launch)
+        return 1e3 * (q_s + g_s) / steps
+
+    measured = res["ms_per_step"]
+    f_meas, f_spec = floor_ms(fp8_peak), floor_ms(FP8_SPEC_TFLOPS)
+    return {"floor_ms_measured_peaks": round(f_meas, 4), "frac_measured_peaks": round(f_meas / measured, 4),
+            "floor_ms_spec": round(f_spec, 4), "frac_spec": round(f_spec / measured, 4),
+            "model": "sum over quantizers of bytes / HBM + sum over GEMMs of max(FLOPs / peak, bytes / HBM)"}
+
+
+# ------------------------------------------------- quantizer-only workload
+def quantizer_arm(args, rank, world, local_rank):
+    """The activation-quantizer configuration: each step quantizes X [8192, 3072]
+    per token to FP8 (qmax 448) and per row to INT8 (qmax 127).  X (48 MiB) fits
+    in L2, so a 256 MiB buffer is written between timed steps and only the
+    quantizer launches are timed (CUDA events around each step's two launches).
+    The flush buffer is then read back, so that the dirty lines the write left
+    in L2 are written back before the timed launches instead of during them."""
+    import torch
+    from int8_w8a8_quantized_b200 import _capi, workloads
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    lib = _capi.load_library()
+    stream = torch.cuda.current_stream()
+    sh = int(stream.cuda_stream)
+    x = workloads.quantizer_input(device=dev)
+    M, K = x.shape
+    q8 = torch.empty((M, K), dtype=torch.uint8, device=dev)
+    s8 = torch.empty(M, device=dev)
+    qi = torch.empty((M, K), dtype=torch.int8, device=dev)
+    si = torch.empty(M, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def check(st, what):
+        if st != 0:
+            raise RuntimeError(f"{what}: {_capi.status_string(st)}: {_capi.last_error_message()}")
+
+    def step():
+        check(lib.tfq_quant_act_fp8_per_token(x.data_ptr(), M, K, 448.0, q8.data_ptr(), s8.data_ptr(), sh), "fp8")
+        check(lib.tfq_quant_weight_per_channel(x.data_ptr(), M, K, _capi.TFQ_DTYPE_INT8, 127.0, qi.data_ptr(),
+                                               si.data_ptr(), sh), "int8")
+
+    sink = torch.empty(1, dtype=torch.int64, device=dev)
+    flush_words = flush.view(torch.int64)
+
+    def flush_l2():
+        flush.zero_()
+        torch.sum(flush_words, dim=0, keepdim=True, out=sink)
+
+    for _ in range(args.warmup):
+        flush_l2()
+        step()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    evs = []
+    for _ in range(args.steps):
+        flush_l2()
+        e0 = torch.cuda.Event(enable_timing=True); e0.record(stream)
+        step()
+        e1 = torch.cuda.Event(enable_timing=True); e1.record(stream)
+        evs.append((e0, e1))
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    check(lib.tfq_device_error(sh), "device error")
+    ms = sum(a.elapsed_time(b) for a, b in evs) / args.steps
+    if world > 1:
+        ms = max_over_ranks(ms, dev)
+    nbytes = 2 * (3 * M * K + 4 * M)  # two quantizations: bf16 in, 8-bit codes + fp32 scale out
+    value = world * nbytes / (ms * 1e-3) / 1e9
+    peaks, peak_src = measured_peaks()
+    hbm = peaks.get("hbm_gbs", FALLBACK_HBM_GBS)
+    # end to end: X from pinned host memory, codes and scales back, every step
+    hx = torch.empty(x.shape, dtype=x.dtype, pin_memory=True)
+    hx.copy_(x)
+    outs = [q8, s8, qi, si]
+    hout = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in outs]
+    t0 = torch.cuda.Event(enable_timing=True); t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(args.e2e_steps):
+        x.copy_(hx, non_blocking=True)
+        step()
+        for h, t in zip(hout, outs):
+            h.copy_(t, non_blocking=True)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = t0.elapsed_time(t1) / args.e2e_steps
+    if rank != 0:
+        return
+    line = {
+        "metric": "activation quantizer GB/s (per-token FP8 qmax 448 + per-row INT8 127), algorithmic bytes",
+        "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "e4m3 + s8", "data": "synthetic",
+        "config": {"workload": "activation_quantizer", "M": M, "K": K, "outlier_cols": "1 % x50",
+                   "zero_rows": 16, "l2": "256 MiB written, then read, between timed steps (flush), not timed",
+                   "parallelism": f"replicas x{world}"},
+        "roofline": {"kernel": "quant_rows_kernel<fp8>, quant_rows_kernel<int8>", "bound": "hbm",
+                     "achieved": round(value / world, 1), "peak": hbm, "unit": "GB/s",
+                     "frac": round(value / world / hbm, 4), "frac_of_nominal_8tbs": round(value / world / 8000.0, 4),
+                     "traffic": None, "algorithmic_bytes_per_launch": nbytes // 2, "peak_source": peak_src},
+        "gpu_launches": 2 * args.steps, "clocks": clk,
+        "e2e": {"value": round(world * nbytes / (e2e_ms * 1e-3) / 1e9, 1), "unit": "GB/s", "ms_per_step": e2e_ms,
+                "h2d_bytes_per_step": x.numel() * 2,
+                "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t in outs)},
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = quantizer_cpu_baseline(x.cpu())
+    print(json.dumps(line), flush=True)
+
+
+def quantizer_cpu_baseline(x_cpu):
+    import numpy as np
+    import torch
+    import oracle
+    bits = x_cpu.contiguous().view(torch.int16).numpy().view(np.uint16)
+    M, K = bits.shape
+    t0 = time.perf_counter()
+    n = 0
+    while time.perf_counter() - t0 < 10.0 or n == 0:
+        oracle.quant_rows_fp8(bits, 448.0)
+        oracle.quant_rows_int8(bits, 127.0)
+        n += 1
+    secs = time.perf_counter() - t0
+    return {"value": n * 2 * (3 * M * K + 4 * M) / secs / 1e9, "unit": "GB/s", "cores": oracle.num_threads(),
+            "kind": "oracle", "sample": f"{n} passes over the full [{M}, {K}] input (FP8 and INT8)", "seconds": secs,
+            "ms_per_pass": 1e3 * secs / n}
+
+
 # ------------------------------------------------------------------ main
+def quantizer_main(args, rank, world, local_rank):
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        from int8_w8a8_quantized_b200 import workloads
+        import oracle
+        x = workloads.quantizer_input()
+        cb = quantizer_cpu_baseline(x)
+        line = {"metric": "activation quantizer GB/s (per-token FP8 qmax 448 + per-row INT8 127), algorithmic bytes",
+                "impl": "reference", "value": cb["value"], "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": cb["ms_per_pass"], "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+                "config": {"workload": "activation_quantizer", "M": 8192, "K": 3072},
+                "cpu_baseline": {"value": cb["value"], "unit": "GB/s", "cores": oracle.num_threads(), "kind": "oracle",
+                                 "sample": cb["sample"]},
+                "e2e": {"value": cb["value"], "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return 0
+    import torch
+    import torch.distributed as dist
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    quantizer_arm(args, rank, world, local_rank)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
 def main():
     args = parse_args()
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     from int8_w8a8_quantized_b200 import workloads
+    if args.workload == "activation_quantizer":
+        return quantizer_main(args, rank, world, local_rank)
     wl = workloads.WORKLOADS[args.workload]
     cfg = {"workload": wl.name, "M": wl.M, "dtype": args.dtype,
            "linears": [f"{l.name}:{l.K}->{l.N}" for l in wl.linears],
@@ -638,10 +814,12 @@ def main():
             "peak": peaks.get("hbm_gbs", FALLBACK_HBM_GBS),
             "unit": "GB/s",
             "frac": None if quant_gbs is None else round(quant_gbs / peaks.get("hbm_gbs", FALLBACK_HBM_GBS), 4),
+            "frac_of_nominal_8tbs": None if quant_gbs is None else round(quant_gbs / 8000.0, 4),
             "share_of_step": round(res["quant_ms_total"] / (res["ms_per_step"] * args.steps), 4),
             "traffic": recorded_traffic("quant", wl.name, args.dtype),
             "algorithmic_bytes_per_launch": round(res["quant_bytes_total"] / max(1, res["quant_launches"])),
         },
+        "path_roofline": path_roofline(res, args.steps, peaks, fp8_peak),
         "per_linear_ms": {k: round(statistics.median(v), 4) for k, v in res["per_linear"].items()},
         "gpu_launches": res["gpu_launches"],
         "clocks": res["clocks"],

@@ -185,3 +185,14 @@ def test_mid_rows_grouped(M, K):
     q_ref, s_ref = _gpu.oracle_quant_int8(x, 127.0)
     np.testing.assert_array_equal(s.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
     np.testing.assert_array_equal(q.cpu().numpy().view(np.int8), q_ref)
+
+
+@pytest.mark.parametrize("M,K", [(40000, 3072), (33000, 2176)])
+def test_many_short_rows_sampled(M, K):
+    """More than 32768 rows of K <= 3072 take the two-CTA-per-SM warp-per-row
+    variant (fewer rows take the three-CTA one); sampled rows + the tail."""
+    x = workloads.activations(M, K, seed=M + K, nu=4, outlier_cols=K // 100, outlier_mult=20.0, zero_rows=3,
+                              device="cuda")
+    rows = _gpu.sample_rows(M, 512, seed=K)
+    _assert_fp8_equal(x, 448.0, rows)
+    _assert_fp8_equal(x, 21.0, rows)
