@@ -74,32 +74,50 @@ def parse_args():
     return ap.parse_args()
 
 
+_CSRC = "int8_w8a8_quantized_b200/csrc/"
+# Sources of the kernels a traffic record was captured on, per dtype and kind.
 KERNEL_SOURCES = {
-    "gemm": ("int8_w8a8_quantized_b200/csrc/tfq_gemm.cu", "int8_w8a8_quantized_b200/csrc/tfq_gemm_common.cuh",
-             "int8_w8a8_quantized_b200/csrc/tfq_ptx.cuh"),
-    "quant": ("int8_w8a8_quantized_b200/csrc/tfq_quant.cu", "int8_w8a8_quantized_b200/csrc/tfq_quant_common.cuh",
-              "int8_w8a8_quantized_b200/csrc/tfq_ptx.cuh"),
+    ("fp8", "gemm"): ("tfq_gemm.cu", "tfq_gemm_common.cuh", "tfq_ptx.cuh"),
+    ("fp8", "quant"): ("tfq_quant.cu", "tfq_quant_common.cuh", "tfq_ptx.cuh"),
+    ("int8", "gemm"): ("tfq_gemm.cu", "tfq_gemm_common.cuh", "tfq_ptx.cuh"),
+    ("int8", "quant"): ("tfq_quant.cu", "tfq_quant_common.cuh", "tfq_ptx.cuh"),
+    ("fp8_f16acc", "gemm"): ("tfq_gemm.cu", "tfq_gemm_common.cuh", "tfq_ptx.cuh"),
+    ("fp8_f16acc", "quant"): ("tfq_quant.cu", "tfq_quant_common.cuh", "tfq_ptx.cuh"),
+    ("mxfp8", "gemm"): ("tfq_gemm_mx.cu", "tfq_gemm_common.cuh", "tfq_ptx.cuh"),
+    ("mxfp8", "quant"): ("tfq_quant_mx.cu", "tfq_quant_common.cuh"),
 }
-TRAFFIC_RECORD = os.path.join(ROOT, "profiles", "roofline_traffic_video_dit_block.md")
+
+
+def traffic_record_path(workload: str, dtype: str) -> str:
+    suffix = "" if dtype == "fp8" else f"_{dtype}"
+    return os.path.join(ROOT, "profiles", f"roofline_traffic_{workload}{suffix}.md")
+
+
+TRAFFIC_RECORD = traffic_record_path("video_dit_block", "fp8")
+
+
+def sources_sha256(dtype: str, kind: str) -> str:
+    import hashlib
+    m = hashlib.sha256()
+    for f in KERNEL_SOURCES[(dtype, kind)]:
+        with open(os.path.join(ROOT, _CSRC + f), "rb") as fh:
+            m.update(fh.read())
+    return m.hexdigest()
 
 
 def recorded_traffic(kind: str, workload: str, dtype: str):
-    """DRAM bytes per launch from the committed ncu capture, or None when the
-    capture is for another workload or the kernel sources changed since."""
-    import hashlib
+    """DRAM bytes per launch from the committed ncu capture of this workload and
+    dtype (profiles/roofline_traffic_<workload>[_<dtype>].md), or None when there
+    is none or the kernel sources changed since it was taken."""
     try:
         kv = {}
-        for line in open(TRAFFIC_RECORD, encoding="utf-8"):
+        for line in open(traffic_record_path(workload, dtype), encoding="utf-8"):
             if " = " in line:
                 k, v = line.strip().split(" = ", 1)
                 kv[k] = v
         if kv.get("workload") != workload or kv.get("dtype") != dtype:
             return None
-        m = hashlib.sha256()
-        for f in KERNEL_SOURCES[kind]:
-            with open(os.path.join(ROOT, f), "rb") as fh:
-                m.update(fh.read())
-        if m.hexdigest() != kv.get(f"{kind}.sources_sha256"):
+        if sources_sha256(dtype, kind) != kv.get(f"{kind}.sources_sha256"):
             return None
         return float(kv[f"{kind}.traffic_bytes_per_launch"])
     except (OSError, KeyError, ValueError):
