@@ -48,8 +48,11 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
 #ifndef TFQ_WAIT_HINT_NS
 // Suspend-time hint of one try_wait: a waiting thread sleeps up to this long
 // (it wakes as soon as the phase completes) instead of spinning and taking
-// issue slots from the warps that do work.  0 = no hint.
-#define TFQ_WAIT_HINT_NS 0
+// issue slots from the warps that do work -- in the GEMMs the MMA-issuing
+// warp shares its scheduler with an epilogue warp that mostly waits.
+// Measured on B200: FP8 GEMMs 3-5 % and MXFP8 GEMMs 5-15 % faster than with
+// no hint; 100, 500 and 2000 ns perform alike.  0 = no hint.
+#define TFQ_WAIT_HINT_NS 500
 #endif
 
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
