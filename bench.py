@@ -70,6 +70,7 @@ def parse_args():
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-context", action="store_true", help="skip the torch._scaled_mm context line")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle sample")
     return ap.parse_args()
 
@@ -413,11 +414,52 @@ def gpu_arm(args, wl, rank, world, local_rank):
         key = f"{m}x{n}x{k}"
         out["per_linear"].setdefault(key, []).append(a.elapsed_time(b))
 
+    out["context"] = torch_scaled_mm_context(args, wl, lins, aq, ys, qmaxes, stream) if not args.no_context else None
+
     # -------- end-to-end through the C ABI with host buffers
     e2e = None
     if not args.no_e2e:
         e2e = e2e_arm(args, wl, qmaxes, quant_fn, gemm_fn, xs, lins, aq, ys, stream, sh, check)
     return out, e2e
+
+
+def torch_scaled_mm_context(args, wl, lins, aq, ys, qmaxes, stream):
+    """Context line, outside the timed region: the block's GEMMs through
+    torch._scaled_mm (cuBLASLt; row-wise fp32 scales, bias, bf16 out) on the same
+    quantized operands, CUDA events per call after two warm-up calls.  FP8 only."""
+    import torch
+    if args.dtype not in ("fp8", "fp8_f16acc"):
+        return None
+    try:
+        flops = 0
+        ms = 0.0
+        per = {}
+        for q in qmaxes:
+            for lin, Wq, sw, b in lins:
+                A, sa = aq[(lin.x, q)]
+                a8, w8 = A.view(torch.float8_e4m3fn), Wq.view(torch.float8_e4m3fn)
+
+                def call():
+                    return torch._scaled_mm(a8, w8.t(), scale_a=sa.view(-1, 1), scale_b=sw.view(1, -1), bias=b,
+                                            out_dtype=torch.bfloat16)
+                for _ in range(2):
+                    call()
+                times = []
+                for _ in range(3):
+                    e0 = torch.cuda.Event(enable_timing=True); e1 = torch.cuda.Event(enable_timing=True)
+                    e0.record(stream); r = call(); e1.record(stream)
+                    torch.cuda.synchronize()
+                    times.append(e0.elapsed_time(e1))
+                    del r
+                t = statistics.median(times)
+                ms += t
+                flops += 2 * wl.M * lin.N * lin.K
+                per[f"{wl.M}x{lin.N}x{lin.K}"] = round(t, 4)
+        return {"torch_scaled_mm_tflops": round(flops / (ms * 1e-3) / 1e12, 1), "per_linear_ms": per,
+                "what": "the block's GEMMs through torch._scaled_mm (cuBLASLt, row-wise fp32 scales, bias, bf16 "
+                        "out) on the same quantized operands; median of 3 calls each, outside the timed region"}
+    except Exception as e:  # a torch build without FP8 scaled_mm on this device
+        return {"error": f"{type(e).__name__}: {str(e)[:200]}"}
 
 
 def e2e_arm(args, wl, qmaxes, quant_fn, gemm_fn, xs, lins, aq, ys, stream, sh, check):
@@ -838,6 +880,7 @@ def main():
             "algorithmic_bytes_per_launch": round(res["quant_bytes_total"] / max(1, res["quant_launches"])),
         },
         "path_roofline": path_roofline(res, args.steps, peaks, fp8_peak),
+        "context": res.get("context"),
         "per_linear_ms": {k: round(statistics.median(v), 4) for k, v in res["per_linear"].items()},
         "gpu_launches": res["gpu_launches"],
         "clocks": res["clocks"],
