@@ -202,11 +202,65 @@ __device__ __forceinline__ void l2_policies(const GemmArgs& p, uint64_t& pol_a, 
     }
 }
 
+// Chunk c (EPI_COLS columns) of the epilogue of one 32-row slice of a
+// finished tile; nothing past column N.  Its TMEM loads have completed when
+// it returns, so the caller may hand those accumulator columns back.
+template <int kBN, int kAcc>
+__device__ __forceinline__ void store_tile_chunk(const GemmArgs& p, const CUtensorMap& tmY, uint32_t t_row,
+                                                 uint8_t* ebuf, const float* colp, int n_tile0, int row0,
+                                                 float2 sa2, uint64_t y_policy, int lane, int c) {
+    const int n0 = n_tile0 + c * EPI_COLS;
+    if (n0 >= p.N) return;  // uniform across the warp
+    uint32_t acc[2][32];
+    tmem_ld_32x32b_x32(t_row + c * EPI_COLS, acc[0]);
+    tmem_ld_32x32b_x32(t_row + c * EPI_COLS + 32, acc[1]);
+    tmem_ld_wait();
+    uint32_t packed[2][16];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {  // 8 columns
+            const int nl = c * EPI_COLS + h * 32 + g * 8;
+            const float4 w0 = *reinterpret_cast<const float4*>(colp + nl);
+            const float4 w1 = *reinterpret_cast<const float4*>(colp + nl + 4);
+            const float4 b0 = *reinterpret_cast<const float4*>(colp + kBN + nl);
+            const float4 b1 = *reinterpret_cast<const float4*>(colp + kBN + nl + 4);
+            const float2 sw[4] = {make_float2(w0.x, w0.y), make_float2(w0.z, w0.w), make_float2(w1.x, w1.y),
+                                  make_float2(w1.z, w1.w)};
+            const float2 bb[4] = {make_float2(b0.x, b0.y), make_float2(b0.z, b0.w), make_float2(b1.x, b1.y),
+                                  make_float2(b1.z, b1.w)};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const float2 a2 = make_float2(acc_value<kAcc>(acc[h][g * 8 + 2 * j]),
+                                              acc_value<kAcc>(acc[h][g * 8 + 2 * j + 1]));
+                const float2 y = __ffma2_rn(__fmul2_rn(a2, sa2), sw[j], bb[j]);
+                packed[h][g * 4 + j] = pack_bf16x2(y.x, y.y);
+            }
+        }
+    }
+    // The staging buffer's previous TMA store must have finished reading it.
+    if (lane == 0) bulk_wait_read<0>();
+    __syncwarp();
+#pragma unroll
+    for (int unit = 0; unit < 8; ++unit) {  // 128-byte swizzle: unit u of row r at u ^ (r % 8)
+        uint4* dst = reinterpret_cast<uint4*>(ebuf + lane * 128 + ((unit ^ (lane & 7)) << 4));
+        const uint32_t* w = &packed[unit >> 2][(unit & 3) * 4];
+        *dst = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+        tma_store_2d_hint(&tmY, ebuf, n0, row0, y_policy);  // the output streams out of L2
+        bulk_commit();
+    }
+}
+
 // Epilogue of one 32-row slice of a finished tile: TMEM -> registers ->
 // y = acc * s_a[m] * s_w[n] + bias[n] in fp32 (packed fp32x2 operations) ->
 // bf16 -> 128-byte swizzled staging buffer -> TMA store, EPI_COLS columns
-// at a time.  `t_row` is the TMEM address of this warp's 32 lanes at the
-// tile's first column; colp holds the tile's column scales and bias.
+// at a time (store_tile_chunk).  `t_row` is the TMEM address of this warp's
+// 32 lanes at the tile's first column; colp holds the tile's column scales
+// and bias.
 template <int kBN, int kAcc>
 __device__ __forceinline__ void store_tile_rows(const GemmArgs& p, const CUtensorMap& tmY, uint32_t t_row,
                                                 uint8_t* ebuf, const float* colp, int n_tile0, int row0, float sa,
@@ -214,52 +268,8 @@ __device__ __forceinline__ void store_tile_rows(const GemmArgs& p, const CUtenso
     const float2 sa2 = make_float2(sa, sa);
     const uint64_t y_policy = make_l2_policy_evict_first();
 #pragma unroll 1
-    for (int c = 0; c < kBN / EPI_COLS; ++c) {
-        const int n0 = n_tile0 + c * EPI_COLS;
-        if (n0 >= p.N) break;  // uniform across the warp
-        uint32_t acc[2][32];
-        tmem_ld_32x32b_x32(t_row + c * EPI_COLS, acc[0]);
-        tmem_ld_32x32b_x32(t_row + c * EPI_COLS + 32, acc[1]);
-        tmem_ld_wait();
-        uint32_t packed[2][16];
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-#pragma unroll
-            for (int g = 0; g < 4; ++g) {  // 8 columns
-                const int nl = c * EPI_COLS + h * 32 + g * 8;
-                const float4 w0 = *reinterpret_cast<const float4*>(colp + nl);
-                const float4 w1 = *reinterpret_cast<const float4*>(colp + nl + 4);
-                const float4 b0 = *reinterpret_cast<const float4*>(colp + kBN + nl);
-                const float4 b1 = *reinterpret_cast<const float4*>(colp + kBN + nl + 4);
-                const float2 sw[4] = {make_float2(w0.x, w0.y), make_float2(w0.z, w0.w), make_float2(w1.x, w1.y),
-                                      make_float2(w1.z, w1.w)};
-                const float2 bb[4] = {make_float2(b0.x, b0.y), make_float2(b0.z, b0.w), make_float2(b1.x, b1.y),
-                                      make_float2(b1.z, b1.w)};
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const float2 a2 = make_float2(acc_value<kAcc>(acc[h][g * 8 + 2 * j]),
-                                                  acc_value<kAcc>(acc[h][g * 8 + 2 * j + 1]));
-                    const float2 y = __ffma2_rn(__fmul2_rn(a2, sa2), sw[j], bb[j]);
-                    packed[h][g * 4 + j] = pack_bf16x2(y.x, y.y);
-                }
-            }
-        }
-        // The staging buffer's previous TMA store must have finished reading it.
-        if (lane == 0) bulk_wait_read<0>();
-        __syncwarp();
-#pragma unroll
-        for (int unit = 0; unit < 8; ++unit) {  // 128-byte swizzle: unit u of row r at u ^ (r % 8)
-            uint4* dst = reinterpret_cast<uint4*>(ebuf + lane * 128 + ((unit ^ (lane & 7)) << 4));
-            const uint32_t* w = &packed[unit >> 2][(unit & 3) * 4];
-            *dst = make_uint4(w[0], w[1], w[2], w[3]);
-        }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-            tma_store_2d_hint(&tmY, ebuf, n0, row0, y_policy);  // the output streams out of L2
-            bulk_commit();
-        }
-    }
+    for (int c = 0; c < kBN / EPI_COLS; ++c)
+        store_tile_chunk<kBN, kAcc>(p, tmY, t_row, ebuf, colp, n_tile0, row0, sa2, y_policy, lane, c);
 }
 
 __device__ __forceinline__ void pair_tile_coords(int t, int m_tiles, int n_tiles, int group_m, int band_n, int& tm,

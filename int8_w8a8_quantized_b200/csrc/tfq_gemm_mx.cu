@@ -287,16 +287,31 @@ __global__ void __launch_bounds__(THREADS, 1)
 // MXFP8 CTA-pair kernel: a cluster of two CTAs computes a 256 x 192 tile with
 // tcgen05.mma.cta_group::2.kind::mxf8f6f4.block_scale (M = 256, N = 192).  As
 // in scaled_mm_pair_kernel, CTA r loads rows [128 r, 128 r + 128) of the A
-// panel and rows [96 r, 96 r + 96) of the B panel; in addition each CTA loads
-// the scale atom of its own 128 A rows and both atoms that cover the tile's
-// 192 B rows, all by TMA (the scale buffer viewed as rows of 512 bytes), all
+// panel and rows [128 r, 128 r + 128) of the B panel; in addition each CTA
+// loads the scale atom of its own 128 A rows and the two atoms of the tile's
+// 256 B rows, all by TMA (the scale buffer viewed as rows of 512 bytes), all
 // completing on the even CTA's "full" barrier.  The even CTA's MMA thread
 // copies the scales of each stage into both CTAs' TMEM with one
-// tcgen05.cp.cta_group::2 per atom (each CTA from its own shared memory), so
-// the three copies per stage now serve twice the FLOPs of the one-CTA kernel.
+// tcgen05.cp.cta_group::2 per atom (each CTA from its own shared memory).
+//
+// N = 256 with two accumulators and 12 scale columns needs 524 TMEM columns,
+// 12 more than there are, so the two accumulators overlap by 32 columns:
+// buffer 0 is columns [0, 256), buffer 1 [224, 480), the scales [480, 492).
+// The epilogue of a tile reads the shared 32 columns first -- the last 64-
+// column chunk of buffer 0, the first of buffer 1 -- and hands them back on
+// an "overlap_free" barrier; the first MMA of the next tile (the other
+// buffer) waits for that, besides the usual "tmem_empty" of its own buffer.
+// Against 256 x 192 tiles with disjoint accumulators this gives each scale
+// copy a third more FLOPs and each MMA its full width.
+constexpr int MXP_BN = 256;
+constexpr int MXP_OVERLAP = 32;                           // TMEM columns shared by the two accumulators
+constexpr uint32_t MXP_BUF_STRIDE = MXP_BN - MXP_OVERLAP; // buffer b starts at column 224 b
+constexpr uint32_t MXP_SFA_COL = MXP_BUF_STRIDE + MXP_BN; // 480
+constexpr uint32_t MXP_SFB_COL = MXP_SFA_COL + 4;
+static_assert(MXP_SFB_COL + 8 <= 512, "TMEM budget exceeded");
 constexpr int MXP_STAGES = 6;
-constexpr int MXP_BHALF = MX_BN / 2;                     // 96 B rows per CTA
-constexpr int MXP_B_STAGE_BYTES = MXP_BHALF * BK;        // 12 KiB
+constexpr int MXP_BHALF = MXP_BN / 2;                    // 128 B rows per CTA
+constexpr int MXP_B_STAGE_BYTES = MXP_BHALF * BK;        // 16 KiB
 constexpr size_t MXP_SMEM_RING =
     static_cast<size_t>(MXP_STAGES) * (A_STAGE_BYTES + MXP_B_STAGE_BYTES + MX_SFA_BYTES + MX_SFB_BYTES);
 constexpr size_t MXP_SMEM_BYTES = 1024 + MXP_SMEM_RING + SMEM_EPI + (2 * MXP_STAGES + 4 + 1) * 8 + 16;
@@ -328,6 +343,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     const int n_clusters = gridDim.x >> 1;
     const int m_tiles = (p.M + 255) / 256;
     const int total_tiles = m_tiles * p.n_tiles;
+    __shared__ uint64_t overlap_free[2];  // epilogues of both CTAs: shared columns of buffer b read
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < MXP_STAGES; ++i) {
@@ -339,6 +355,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             mbar_init(&tmem_empty[i], 2 * EPI_WARPS);
         }
         mbar_init(drain, 1);
+        for (int i = 0; i < 2; ++i) mbar_init(&overlap_free[i], 2 * EPI_WARPS);
         *abort_flag = 0;
         fence_mbar_init();
         prefetch_tensormap(&tmA);
@@ -372,9 +389,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                 int tm, tn;
                 pair_tile_coords(t, m_tiles, p.n_tiles, p.group_m, p.band_n, tm, tn);
                 const int a_row = tm * 256 + static_cast<int>(rank) * 128;
-                const int b_row = tn * MX_BN + static_cast<int>(rank) * MXP_BHALF;
+                const int b_row = tn * MXP_BN + static_cast<int>(rank) * MXP_BHALF;
                 const int a_atom = tm * 2 + static_cast<int>(rank);  // this CTA's 128-row scale panel
-                const int b_atom = (tn * MX_BN) >> 7;                // first of the two B scale atoms
+                const int b_atom = tn * 2;                           // the tile's two B scale atoms
                 for (int kb = 0; kb < p.k_blocks; ++kb, ++it) {
                     const int st = it % MXP_STAGES;
                     const uint32_t ph = static_cast<uint32_t>(it / MXP_STAGES) & 1u;
@@ -407,22 +424,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     } else if (warp == 1) {
         // ------------------------------------------- MMA issuer (even CTA)
         if (lane == 0 && rank == 0) {
-            const uint32_t sfa_t = tmem_base + MX_SFA_COL;
-            const uint32_t sfb_t = tmem_base + MX_SFB_COL;
+            const uint32_t sfa_t = tmem_base + MXP_SFA_COL;
+            const uint32_t sfb_t = tmem_base + MXP_SFB_COL;
             int it = 0, tcount = 0;
             bool ok = true;
             for (int t = cluster; t < total_tiles && ok; t += n_clusters, ++tcount) {
-                int tm, tn;
-                pair_tile_coords(t, m_tiles, p.n_tiles, p.group_m, p.band_n, tm, tn);
-                const uint32_t sfb_shift = static_cast<uint32_t>(((tn * MX_BN) & 127) >> 5);
                 const int buf = tcount & 1;
                 const uint32_t use = static_cast<uint32_t>(tcount >> 1);
-                if (!mbar_wait(&tmem_empty[buf], (use & 1u) ^ 1u, abort_flag)) {
+                // own buffer free (tile tcount - 2), and the columns it shares with the
+                // other buffer read by the epilogue of tile tcount - 1
+                if (!mbar_wait(&tmem_empty[buf], (use & 1u) ^ 1u, abort_flag) ||
+                    (tcount >= 1 &&
+                     !mbar_wait(&overlap_free[buf ^ 1], static_cast<uint32_t>((tcount - 1) >> 1) & 1u, abort_flag))) {
                     give_up(abort_flag, p.err, kErrGemmMma);
                     break;
                 }
                 tc_fence_after();
-                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * MX_BN);
+                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf) * MXP_BUF_STRIDE;
                 for (int kb = 0; kb < p.k_blocks; ++kb, ++it) {
                     const int st = it % MXP_STAGES;
                     const uint32_t ph = static_cast<uint32_t>(it / MXP_STAGES) & 1u;
@@ -441,9 +459,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                     for (int k = 0; k < BK / UMMA_K; ++k) {
                         const uint64_t koff = static_cast<uint64_t>((k * UMMA_K) >> 4);
                         const uint32_t id = static_cast<uint32_t>(k);
-                        const uint32_t idesc = make_mx_idesc(256, MX_BN) | (id << 29) | (id << 4);
+                        const uint32_t idesc = make_mx_idesc(256, MXP_BN) | (id << 29) | (id << 4);
                         mma_mxf8_block_scaled_pair(d_tmem, a_desc + koff, b_desc + koff, idesc, sfa_t | (id << 30),
-                                                   (sfb_t + sfb_shift) | (id << 30), (kb | k) != 0 ? 1u : 0u);
+                                                   sfb_t | (id << 30), (kb | k) != 0 ? 1u : 0u);
                     }
                     mma_commit_pair(&empty[st], 0x3);
                 }
@@ -460,11 +478,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         float* colp = reinterpret_cast<float*>(sE + EPI_WARPS * EPI_BUF_BYTES + ew * COLP_BYTES);
         const uint32_t tmem_empty_leader0 = mapa_shared(smem_u32(&tmem_empty[0]), 0);
         const uint32_t tmem_empty_leader1 = mapa_shared(smem_u32(&tmem_empty[1]), 0);
+        const uint32_t overlap_leader0 = mapa_shared(smem_u32(&overlap_free[0]), 0);
+        const uint32_t overlap_leader1 = mapa_shared(smem_u32(&overlap_free[1]), 0);
+        const uint64_t y_policy = make_l2_policy_evict_first();
+        constexpr int kChunks = MXP_BN / EPI_COLS;
         int tcount = 0;
         for (int t = cluster; t < total_tiles; t += n_clusters, ++tcount) {
             int tm, tn;
             pair_tile_coords(t, m_tiles, p.n_tiles, p.group_m, p.band_n, tm, tn);
-            stage_col_params<MX_BN, true>(p, colp, tn * MX_BN, lane);
+            stage_col_params<MXP_BN, true>(p, colp, tn * MXP_BN, lane);
             const int buf = tcount & 1;
             const uint32_t use = static_cast<uint32_t>(tcount >> 1);
             if (!mbar_wait_warp(&tmem_full[buf], use & 1u, abort_flag)) {
@@ -474,8 +496,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             tc_fence_after();
             const int row0 = tm * 256 + static_cast<int>(rank) * 128 + quarter * 32;
             const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
-                                   static_cast<uint32_t>(buf * MX_BN);
-            store_tile_rows<MX_BN, kAccF32>(p, tmY, t_row, ebuf, colp, tn * MX_BN, row0, 1.0f, lane);
+                                   static_cast<uint32_t>(buf) * MXP_BUF_STRIDE;
+            // the chunk holding the shared columns first: last of buffer 0, first of buffer 1
+            const int first = buf == 0 ? kChunks - 1 : 0;
+            const float2 one2 = make_float2(1.0f, 1.0f);
+            store_tile_chunk<MXP_BN, kAccF32>(p, tmY, t_row, ebuf, colp, tn * MXP_BN, row0, one2, y_policy, lane,
+                                              first);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(buf == 0 ? overlap_leader0 : overlap_leader1);
+#pragma unroll 1
+            for (int c = 0; c < kChunks; ++c)
+                if (c != first)
+                    store_tile_chunk<MXP_BN, kAccF32>(p, tmY, t_row, ebuf, colp, tn * MXP_BN, row0, one2, y_policy,
+                                                      lane, c);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(buf == 0 ? tmem_empty_leader0 : tmem_empty_leader1);
@@ -539,8 +573,10 @@ tfq_status launch_mxfp8_mm(const void* A, const uint8_t* sf_a, const void* W, co
     const int64_t tiles = static_cast<int64_t>(a.m_tiles) * a.n_tiles;
     if (tiles > INT32_MAX) return fail(TFQ_EUNSUPPORTED, "too many output tiles");
     if (use_pair_kernel(M, ds->sm_count)) {
-        // B halves of 96 rows; the scale buffers as [KA * RA, 128] 32-bit words
-        // (one 512-byte atom per row): one atom for A, two for B per stage.
+        // 256-wide tiles; B halves of 128 rows; the scale buffers as [KA * RA, 128]
+        // 32-bit words (one 512-byte atom per row): one atom for A, two for B per stage.
+        a.n_tiles = static_cast<int>((N + MXP_BN - 1) / MXP_BN);
+        choose_raster(K, MXP_BN, a.band_n, a.group_m);
         CUtensorMap tmBh, tmSA, tmSB;
         const uint64_t ka = static_cast<uint64_t>((K + 127) / 128);
         st = encode_tensor_map_2d(&tmBh, CU_TENSOR_MAP_DATA_TYPE_UINT8, W, K, N, K, BK, MXP_BHALF,
