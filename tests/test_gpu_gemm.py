@@ -141,3 +141,11 @@ def test_tensor_wrapper_linear():
     A_ref, sa_ref = _gpu.oracle_quant_fp8(x, 448.0)
     y_ref = oracle.scaled_fp8_linear(A_ref, sa_ref, Wq.cpu().numpy(), sw.cpu().numpy(), _gpu.bf16_bits_np(b))
     _gpu.gemm_tolerance_check(y, y_ref, "wrapper")
+
+
+@pytest.mark.parametrize("M,N,K", [(4096, 4096, 256), (3000, 5120, 384)])
+def test_pair_kernel_several_tiles_per_cluster(M, N, K):
+    """256 / 240 pair tiles over the 74 clusters: every cluster runs 3-4
+    tiles, so both TMEM accumulators are reused and the cluster pacing,
+    the band raster and the accumulator hand-over run for real; full compare."""
+    _run_case(M, N, K, True, seed=M + N + K)

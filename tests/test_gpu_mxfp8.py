@@ -172,3 +172,11 @@ def test_wrapper_linear():
     y_ref = oracle.mxfp8_linear(A_ref, sfa_ref, Wq.cpu().numpy(), _gpu.mx_untile(sfw.cpu().numpy(), 264, 512),
                                 _gpu.bf16_bits_np(b))
     _gpu.gemm_tolerance_check(y, y_ref, "mx wrapper")
+
+
+@pytest.mark.parametrize("M,N,K", [(4096, 4096, 128), (2600, 5120, 256)])
+def test_gemm_pair_several_tiles_per_cluster(M, N, K):
+    """Several 256x256 pair tiles per cluster: both overlapping TMEM
+    accumulators are reused, so every tile's first MMA waits for the other
+    buffer's shared columns to be read; full compare."""
+    _gemm_case(M, N, K, True, seed=M + 7 * N + K)

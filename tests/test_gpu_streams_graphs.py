@@ -95,3 +95,35 @@ def test_cuda_graph_capture_and_replay():
         assert torch.equal(y_graph, y)
     del graph
     _gpu.check_device_error()
+
+
+def test_mxfp8_and_int8_concurrent_streams_match_serial():
+    """The MXFP8 and INT8 paths on two streams at once give the results of the
+    same calls run one after the other."""
+    from int8_w8a8_quantized_b200 import tfq_mxfp8_linear, tfq_quant_mxfp8, tfq_quant_weight_per_channel
+    from int8_w8a8_quantized_b200 import tfq_quant_act_int8_per_token, tfq_scaled_int8_linear
+    _gpu.lib()
+    x = workloads.activations(2048, 1024, seed=21, device="cuda")
+    w = workloads.weights(2560, 1024, seed=22, std=0.02, device="cuda")
+    b = workloads.bias(2560, seed=23, device="cuda")
+    Wm, sfw = tfq_quant_mxfp8(w)
+    Wi, swi = tfq_quant_weight_per_channel(w, "int8")
+    Am, sfa = tfq_quant_mxfp8(x)
+    Ai, sai = tfq_quant_act_int8_per_token(x)
+    torch.cuda.synchronize()
+    ref_m = tfq_mxfp8_linear(Am, sfa, Wm, sfw, b)
+    ref_i = tfq_scaled_int8_linear(Ai, sai, Wi, swi, b)
+    torch.cuda.synchronize()
+    s1, s2 = torch.cuda.Stream(), torch.cuda.Stream()
+    for _ in range(3):
+        s1.wait_stream(torch.cuda.current_stream())
+        s2.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s1):
+            y_m = tfq_mxfp8_linear(Am, sfa, Wm, sfw, b, stream=s1)
+        with torch.cuda.stream(s2):
+            y_i = tfq_scaled_int8_linear(Ai, sai, Wi, swi, b, stream=s2)
+        torch.cuda.current_stream().wait_stream(s1)
+        torch.cuda.current_stream().wait_stream(s2)
+        torch.cuda.synchronize()
+        assert torch.equal(y_m, ref_m) and torch.equal(y_i, ref_i)
+    _gpu.check_device_error()
