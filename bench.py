@@ -97,12 +97,23 @@ def traffic_record_path(workload: str, dtype: str) -> str:
 TRAFFIC_RECORD = traffic_record_path("video_dit_block", "fp8")
 
 
+def _code_only(text: str) -> str:
+    """C/C++/CUDA source without comments and blank lines (the kernels'
+    sources hold no '//' or '/*' inside string literals)."""
+    import re
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    return "\n".join(line.rstrip() for line in text.splitlines() if line.strip())
+
+
 def sources_sha256(dtype: str, kind: str) -> str:
+    """SHA-256 of the code (comments stripped) of the sources of a dtype's
+    kernels: a traffic record stays valid while that code is unchanged."""
     import hashlib
     m = hashlib.sha256()
     for f in KERNEL_SOURCES[(dtype, kind)]:
-        with open(os.path.join(ROOT, _CSRC + f), "rb") as fh:
-            m.update(fh.read())
+        with open(os.path.join(ROOT, _CSRC + f), encoding="utf-8") as fh:
+            m.update(_code_only(fh.read()).encode())
     return m.hexdigest()
 
 

@@ -7,7 +7,14 @@
 // checkpoints" and "tf-kernel FP8: online W8A8": per-token activation
 // scales, per-output-channel weight scales, BF16 output).
 //
-// Kernel structure (one persistent CTA per SM, 192 threads):
+// Two kernels: scaled_mm_pair_kernel (clusters of two CTAs computing 256 x
+// 256 tiles with tcgen05.mma.cta_group::2; every problem of 512 rows or more)
+// and scaled_mm_kernel (one CTA per 128 x 256 tile, smaller problems).  Both
+// are templated on the operand kind: E4M3 with an fp32 or fp16 accumulator,
+// or S8 with an s32 accumulator (the INT8 W8A8 path).
+//
+// One-CTA structure (one persistent CTA per SM, 192 threads; the pair kernel
+// below follows it):
 //   warp 0      TMA producer: streams 128x128 A tiles and 256x128 B tiles
 //               (K-major, 128-byte swizzle) into a 4-stage shared-memory
 //               ring, completion counted on "full" mbarriers.
@@ -23,8 +30,11 @@
 //               a 128-byte-swizzled staging buffer and TMA-store them; the
 //               accumulator is handed back through "tmem_empty" so the MMA
 //               of the next tile overlaps this epilogue.
-// Tiles are visited in M-grouped raster order so that the CTAs running at
-// the same time share A and B panels in L2.  M and N tails are handled by
+// Tiles are visited in bands of N tiles holding ~40 MB of weight, each band
+// sweeping every M tile, so that the CTAs running at the same time share the
+// band's weight panels (kept in L2) and each activation panel; the pair
+// kernel also keeps its clusters within one tile of each other (pacing,
+// see tfq_gemm_common.cuh).  M and N tails are handled by
 // TMA (zero fill on load, clipping on store); K tails by zero fill.
 // Every wait is bounded (see tfq_ptx.cuh); a CTA that gives up records it in
 // the error word, drains its own outstanding copies and MMAs, frees TMEM and
