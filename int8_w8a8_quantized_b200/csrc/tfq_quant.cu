@@ -186,6 +186,9 @@ __device__ __forceinline__ void load_segment(uint4 (&v)[SEG], const uint4* row, 
 #ifndef TFQ_QUANT_SHORT_SEG
 #define TFQ_QUANT_SHORT_SEG 12  // segment of the variant for rows of K <= 32 * 12 * 8 = 3072
 #endif
+#ifndef TFQ_QUANT_WIDE_SEG
+#define TFQ_QUANT_WIDE_SEG 20   // segment of the variant that holds a K = 5120 row in one pass
+#endif
 #ifndef TFQ_QUANT_SHORT_SEG_MAX_ROWS
 #define TFQ_QUANT_SHORT_SEG_MAX_ROWS 32768  // ... used for at most this many rows
 #endif
@@ -580,20 +583,30 @@ tfq_status launch_quant_rows(const void* x, int64_t rows, int64_t K, float qmax,
     if (K / 8 <= kGroupMaxUnits) return launch_grouped_rows(x, rows, K, qmax, out_int8, clamp, q, s, stream, ds);
     if (K >= TFQ_QUANT_STAGED_MIN_K && K <= TFQ_QUANT_STAGED_MAX_K)
         return launch_staged_rows(x, rows, K, qmax, out_int8, clamp, q, s, stream, ds);
-    constexpr int kLong = TFQ_QUANT_SEG, kShort = TFQ_QUANT_SHORT_SEG;
+    constexpr int kLong = TFQ_QUANT_SEG, kWide = TFQ_QUANT_WIDE_SEG, kShort = TFQ_QUANT_SHORT_SEG;
     // Few rows (each warp gets only a handful): the variant with three CTAs per
     // SM hides more latency -- [8192, 3072] 4.2 vs 3.8 TB/s; many rows: the
     // two-CTA one is faster ([174762, 3072] 6.3 vs 5.7 TB/s), measured on B200.
     const bool short_seg = K <= 32 * kShort * 8 && rows <= TFQ_QUANT_SHORT_SEG_MAX_ROWS;
-    auto kernel = short_seg
-                      ? (out_int8 ? quant_rows_kernel<true, false, kShort>
-                                  : (clamp ? quant_rows_kernel<false, true, kShort>
-                                           : quant_rows_kernel<false, false, kShort>))
-                      : (out_int8 ? quant_rows_kernel<true, false, kLong>
-                                  : (clamp ? quant_rows_kernel<false, true, kLong>
-                                           : quant_rows_kernel<false, false, kLong>));
+    // Otherwise the segment (16 or 20 units per lane) that leaves fewer lane
+    // slots of the last segment empty: K = 5120 fits one 20-unit segment (a
+    // single pass, no re-read from L2), K = 13824 three instead of four; 16 on
+    // a tie.  Measured on B200 inside the video-DiT block: 4.7-4.9 vs 4.0 TB/s.
+    const int64_t units = K / 8;
+    auto waste = [&](int seg) { return (units + 32 * seg - 1) / (32 * seg) * (32 * seg) - units; };
+    const bool wide = !short_seg && waste(kWide) < waste(kLong);
+    const int variant = out_int8 ? 0 : (clamp ? 1 : 2);
+    using Kernel = void (*)(const uint4*, int64_t, int, float, uint8_t*, float*);
+    const Kernel short_k[3] = {quant_rows_kernel<true, false, kShort>, quant_rows_kernel<false, true, kShort>,
+                               quant_rows_kernel<false, false, kShort>};
+    const Kernel wide_k[3] = {quant_rows_kernel<true, false, kWide>, quant_rows_kernel<false, true, kWide>,
+                              quant_rows_kernel<false, false, kWide>};
+    const Kernel long_k[3] = {quant_rows_kernel<true, false, kLong>, quant_rows_kernel<false, true, kLong>,
+                              quant_rows_kernel<false, false, kLong>};
+    const Kernel kernel = short_seg ? short_k[variant] : (wide ? wide_k[variant] : long_k[variant]);
     const int threads = 256;  // 8 warps, one row per warp at a time
-    const int ctas_per_sm = short_seg ? rows_ctas_per_sm<kShort>() : rows_ctas_per_sm<kLong>();
+    const int ctas_per_sm = short_seg ? rows_ctas_per_sm<kShort>()
+                                      : (wide ? rows_ctas_per_sm<kWide>() : rows_ctas_per_sm<kLong>());
     const int64_t blocks = std::min<int64_t>((rows + 7) / 8, static_cast<int64_t>(ds->sm_count) * ctas_per_sm);
     kernel<<<static_cast<unsigned>(blocks), threads, 0, stream>>>(static_cast<const uint4*>(x), rows,
                                                                  static_cast<int>(K), qmax,
