@@ -196,3 +196,20 @@ def test_many_short_rows_sampled(M, K):
     rows = _gpu.sample_rows(M, 512, seed=K)
     _assert_fp8_equal(x, 448.0, rows)
     _assert_fp8_equal(x, 21.0, rows)
+
+
+@pytest.mark.parametrize("K", [4112, 5120, 5136, 6400, 7680, 10240, 12800])
+@pytest.mark.parametrize("M", [3, 300])
+def test_segment_choice_boundaries(M, K):
+    """Row lengths around the 16- / 20-unit segment choice of the
+    warp-per-row kernel: one 20-unit segment (K = 4112, 5120), two
+    (10240), three (12800), and lengths where 16 units waste less (5136,
+    6400, 7680); FP8 with and without the clamp, INT8."""
+    x = workloads.activations(M, K, seed=M * 11 + K, nu=3, outlier_cols=3, outlier_mult=30.0,
+                              zero_rows=1 if M > 2 else 0, device="cuda")
+    for qmax in (448.0, 21.0):
+        _assert_fp8_equal(x, qmax)
+    q, s = _gpu.quant_weight(x, _capi.TFQ_DTYPE_INT8, 127.0)
+    q_ref, s_ref = _gpu.oracle_quant_int8(x, 127.0)
+    np.testing.assert_array_equal(s.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
+    np.testing.assert_array_equal(q.cpu().numpy().view(np.int8), q_ref)
