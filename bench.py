@@ -700,6 +700,23 @@ def quantizer_arm(args, rank, world, local_rank):
     if world > 1:
         ms = max_over_ranks(ms, dev)
     nbytes = 2 * (3 * M * K + 4 * M)  # two quantizations: bf16 in, 8-bit codes + fp32 scale out
+    # What this size allows: two device copies of the same traffic per step
+    # (each reads and writes half of one launch's algorithmic bytes), timed
+    # the same way.  Context for the fraction, not part of the metric.
+    src = torch.empty(nbytes // 4, dtype=torch.uint8, device=dev)
+    dst = torch.empty_like(src)
+    cevs = []
+    for i in range(args.warmup + args.steps):
+        flush_l2()
+        e0 = torch.cuda.Event(enable_timing=True); e0.record(stream)
+        dst.copy_(src)
+        dst.copy_(src)
+        e1 = torch.cuda.Event(enable_timing=True); e1.record(stream)
+        if i >= args.warmup:
+            cevs.append((e0, e1))
+    torch.cuda.synchronize()
+    copy_ms = sum(a.elapsed_time(b) for a, b in cevs) / len(cevs)
+    del src, dst
     value = world * nbytes / (ms * 1e-3) / 1e9
     peaks, peak_src = measured_peaks()
     hbm = peaks.get("hbm_gbs", FALLBACK_HBM_GBS)
@@ -731,7 +748,11 @@ def quantizer_arm(args, rank, world, local_rank):
         "roofline": {"kernel": "quant_rows_kernel<fp8>, quant_rows_kernel<int8>", "bound": "hbm",
                      "achieved": round(value / world, 1), "peak": hbm, "unit": "GB/s",
                      "frac": round(value / world / hbm, 4), "frac_of_nominal_8tbs": round(value / world / 8000.0, 4),
-                     "traffic": None, "algorithmic_bytes_per_launch": nbytes // 2, "peak_source": peak_src},
+                     "traffic": None, "algorithmic_bytes_per_launch": nbytes // 2, "peak_source": peak_src,
+                     "same_traffic_copy": {"gbs": round(nbytes / (copy_ms * 1e-3) / 1e9, 1),
+                                           "ms_per_step": round(copy_ms, 4),
+                                           "frac": round(copy_ms / ms, 4),
+                                           "what": "two device copies of the same bytes per step, same timing"}},
         "gpu_launches": 2 * args.steps, "clocks": clk,
         "e2e": {"value": round(world * nbytes / (e2e_ms * 1e-3) / 1e9, 1), "unit": "GB/s", "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": x.numel() * 2,

@@ -40,10 +40,15 @@ namespace {
 
 constexpr int kCtasPerSm = 2;  // 8 warps per CTA; ~125 registers per thread allow two per SM
 
-__device__ __forceinline__ uint32_t to_int8_byte(float t) {
-    int i = __float2int_rn(t);  // round half to even
-    i = min(max(i, -128), 127);
-    return static_cast<uint32_t>(i) & 0xFFu;
+// Two fp32 quotients t -> their INT8 codes rint_half_even(t) in bytes 0 and
+// 1 (bytes 2 and 3 are don't-care).  Adding 1.5 * 2^23 rounds a |t| < 2^22
+// to an integer, half to even, by the addition's own rounding, and leaves
+// that integer in two's complement in the low bits of the sum.  No clamp to
+// [-128, 127] is needed: with s = RN(amax / qmax), |x| <= amax and
+// qmax <= 127, |t| <= RN(qmax * (1 + 2^-23)) < 127.5.
+__device__ __forceinline__ uint32_t int8x2_rn(float2 t) {
+    const float2 u = __fadd2_rn(t, make_float2(0x1.8p23f, 0x1.8p23f));
+    return __byte_perm(__float_as_uint(u.x), __float_as_uint(u.y), 0x0040);
 }
 
 }  // namespace
@@ -81,7 +86,8 @@ namespace {
 // (s = RN(amax/qmax) and |x| <= amax), and qmax + 1 ulp encodes like qmax
 // because the nearest E4M3 midpoint is 2^-4 of a binade away (448 + ulp
 // saturates to 448).
-// Two bf16 values (one 32-bit word) -> two codes in the low 16 bits.
+// Two bf16 values (one 32-bit word) -> two codes in the low 16 bits (INT8:
+// the high 16 bits are don't-care).
 // (The Markstein quotient here may come out as +0 for a = -0; the caller
 // restores the sign of zero codes from the inputs' sign bits, which is
 // exact because every other quotient already carries the sign of a, and an
@@ -99,7 +105,7 @@ __device__ __forceinline__ uint32_t quantize2(uint32_t w, float sc, float rcp, f
         b = t.y;
     }
     if constexpr (kInt8) {
-        return to_int8_byte(a) | (to_int8_byte(b) << 8);
+        return int8x2_rn(make_float2(a, b));
     } else {
         if constexpr (kClamp) {
             a = fminf(fmaxf(a, -qmax), qmax);
@@ -115,11 +121,10 @@ __device__ __forceinline__ uint2 quantize8(uint4 v, float sc, float rcp, float q
     const uint32_t p1 = quantize2<kInt8, kClamp, kIeeeDiv>(v.y, sc, rcp, qmax);
     const uint32_t p2 = quantize2<kInt8, kClamp, kIeeeDiv>(v.z, sc, rcp, qmax);
     const uint32_t p3 = quantize2<kInt8, kClamp, kIeeeDiv>(v.w, sc, rcp, qmax);
-    uint32_t lo = p0 | (p1 << 16), hi = p2 | (p3 << 16);
-    if constexpr (!kInt8) {  // E4M3 codes keep the sign of (negative) zero
-        lo |= sign_bytes(v.x, v.y);
-        hi |= sign_bytes(v.z, v.w);
-    }
+    if constexpr (kInt8) return make_uint2(__byte_perm(p0, p1, 0x5410), __byte_perm(p2, p3, 0x5410));
+    // E4M3 codes keep the sign of (negative) zero
+    const uint32_t lo = p0 | (p1 << 16) | sign_bytes(v.x, v.y);
+    const uint32_t hi = p2 | (p3 << 16) | sign_bytes(v.z, v.w);
     return make_uint2(lo, hi);
 }
 

@@ -121,3 +121,31 @@ def test_int8_tensor_wrappers():
     A_ref, sa_ref = _gpu.oracle_quant_int8(x, 127.0)
     y_ref = oracle.scaled_int8_linear(A_ref, sa_ref, Wq.cpu().numpy(), sw.cpu().numpy(), None)
     _gpu.gemm_tolerance_check(y, y_ref, "int8 wrapper")
+
+
+@pytest.mark.parametrize("K", [528, 5120, 16384])
+def test_int8_rounding_edges(K):
+    """INT8 codes where x/s is an exact half-integer (round half to even
+    decides), signed zeros, values that round to 0, rows below the 1e-12
+    floor and rows whose scale exceeds 2^125 (the IEEE-division branch), for
+    the grouped, one-warp-per-row and shared-memory-staged kernels."""
+    halves = torch.arange(-127, 127, dtype=torch.float32) + 0.5
+    row = torch.cat([torch.tensor([127.0, -127.0]), halves, torch.tensor([-0.0, 0.0, 0.25, -0.25, 0.75, 1e-30])])
+    reps = (K + row.numel() - 1) // row.numel()
+    base = row.repeat(reps)[:K]
+    x = torch.zeros(8, K)
+    x[0] = base                        # s = 1: x/s = x exactly
+    x[1] = base * 2.0 ** -20           # s = 2^-20, same quotients
+    x[2] = base * 2.0 ** 100           # s = 2^100
+    x[3] = -0.0
+    x[4, :4] = torch.tensor([1e-13, -3e-13, 2e-13, -1e-14])   # below the floor
+    x[5] = base * 3.0                  # a scale that is not a power of two
+    x[6] = base * (3.0e38 / 127.0)     # with qmax <= 2: s > 2^125
+    x[7] = -base
+    x = x.to(torch.bfloat16).cuda()
+    assert torch.isfinite(x.float()).all()
+    for qmax in (127.0, 100.0, 63.5, 2.0, 1.0):
+        q, s = _gpu.quant_weight(x, _capi.TFQ_DTYPE_INT8, qmax)
+        q_ref, s_ref = _gpu.oracle_quant_int8(x, qmax)
+        np.testing.assert_array_equal(s.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
+        np.testing.assert_array_equal(q.cpu().numpy().view(np.int8), q_ref)
