@@ -235,7 +235,8 @@ struct PairCfg {
 template <int PBN, int kAcc>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     scaled_mm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                                const __grid_constant__ CUtensorMap tmY, GemmArgs p) {
+                                const __grid_constant__ CUtensorMap tmBq, const __grid_constant__ CUtensorMap tmY,
+                                GemmArgs p) {
     using C = PairCfg<PBN>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -272,6 +273,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         fence_mbar_init();
         prefetch_tensormap(&tmA);
         prefetch_tensormap(&tmB);
+        if (p.tail_halves) prefetch_tensormap(&tmBq);
         prefetch_tensormap(&tmY);
     }
     if (warp == 1) {
@@ -292,13 +294,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             int issued_phase[PAIR_STAGES];
             for (int i = 0; i < PAIR_STAGES; ++i) issued_phase[i] = -1;
             bool ok = true;
-            int round = 0;
-            for (int t = cluster; t < total_tiles && ok; t += n_clusters, ++round) {
+            int round = 0, t, half;
+            for (int w = cluster; ok && pair_work_item(w, total_tiles, n_clusters, p.tail_halves, t, half);
+                 w += n_clusters, ++round) {
                 if (rank == 0) pace_round(p.round_ctr, round, total_tiles, n_clusters);
                 int tm, tn;
                 pair_tile_coords(t, m_tiles, p.n_tiles, p.group_m, p.band_n, tm, tn);
+                // a half tile: PBN / 2 columns, PBN / 4 B rows per CTA (tmBq's box)
+                const int b_rows = half < 0 ? C::kBHalf : C::kBHalf / 2;
+                const CUtensorMap* tmb = half < 0 ? &tmB : &tmBq;
+                const uint32_t stage_tx = 2 * static_cast<uint32_t>(C::kAStage + b_rows * BK);
                 const int a_row = tm * 256 + static_cast<int>(rank) * 128;
-                const int b_row = tn * PBN + static_cast<int>(rank) * C::kBHalf;
+                const int b_row = tn * PBN + (half > 0 ? PBN / 2 : 0) + static_cast<int>(rank) * b_rows;
                 for (int kb = 0; kb < p.k_blocks; ++kb, ++it) {
                     const int st = it % PAIR_STAGES;
                     const uint32_t ph = static_cast<uint32_t>(it / PAIR_STAGES) & 1u;
@@ -308,9 +315,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                         break;
                     }
                     const uint32_t full_leader = mapa_shared(smem_u32(&full[st]), 0);
-                    if (rank == 0) mbar_arrive_expect_tx(&full[st], 2 * (C::kAStage + C::kBStage));
+                    if (rank == 0) mbar_arrive_expect_tx(&full[st], stage_tx);
                     tma_load_2d_pair(sA + st * C::kAStage, &tmA, kb * BK, a_row, full_leader, pol_a);
-                    tma_load_2d_pair(sB + st * C::kBStage, &tmB, kb * BK, b_row, full_leader, pol_b);
+                    tma_load_2d_pair(sB + st * C::kBStage, tmb, kb * BK, b_row, full_leader, pol_b);
                     issued_phase[st] = static_cast<int>(ph);
                 }
                 if (ok && rank == 0 && p.round_ctr != nullptr) atomicAdd(p.round_ctr, 1u);
@@ -328,9 +335,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     } else if (warp == 1) {
         // ------------------------------------------- MMA issuer (even CTA)
         if (lane == 0 && rank == 0) {
-            int it = 0, tcount = 0;
+            int it = 0, tcount = 0, t, half;
             bool ok = true;
-            for (int t = cluster; t < total_tiles && ok; t += n_clusters, ++tcount) {
+            for (int w = cluster; ok && pair_work_item(w, total_tiles, n_clusters, p.tail_halves, t, half);
+                 w += n_clusters, ++tcount) {
                 const int buf = tcount & 1;
                 const uint32_t use = static_cast<uint32_t>(tcount >> 1);
                 if (!mbar_wait(&tmem_empty[buf], (use & 1u) ^ 1u, abort_flag)) {
@@ -338,6 +346,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                     break;
                 }
                 tc_fence_after();
+                const uint32_t idesc = make_idesc<kAcc>(256, half < 0 ? PBN : PBN / 2);
                 const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * PBN);
                 for (int kb = 0; kb < p.k_blocks; ++kb, ++it) {
                     const int st = it % PAIR_STAGES;
@@ -353,8 +362,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
 #pragma unroll
                     for (int k = 0; k < BK / UMMA_K; ++k) {
                         const uint64_t koff = static_cast<uint64_t>((k * UMMA_K) >> 4);
-                        mma_e4m3_pair<kAcc == kAccS32>(d_tmem, a_desc + koff, b_desc + koff, make_idesc<kAcc>(256, PBN),
-                                           (kb | k) != 0 ? 1u : 0u);
+                        mma_e4m3_pair<kAcc == kAccS32>(d_tmem, a_desc + koff, b_desc + koff, idesc,
+                                                       (kb | k) != 0 ? 1u : 0u);
                     }
                     mma_commit_pair(&empty[st], 0x3);
                 }
@@ -371,11 +380,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         float* colp = reinterpret_cast<float*>(sE + EPI_WARPS * EPI_BUF_BYTES + ew * COLP_BYTES);
         const uint32_t tmem_empty_leader0 = mapa_shared(smem_u32(&tmem_empty[0]), 0);
         const uint32_t tmem_empty_leader1 = mapa_shared(smem_u32(&tmem_empty[1]), 0);
-        int tcount = 0;
-        for (int t = cluster; t < total_tiles; t += n_clusters, ++tcount) {
+        int tcount = 0, t, half;
+        for (int w = cluster; pair_work_item(w, total_tiles, n_clusters, p.tail_halves, t, half);
+             w += n_clusters, ++tcount) {
             int tm, tn;
             pair_tile_coords(t, m_tiles, p.n_tiles, p.group_m, p.band_n, tm, tn);
-            stage_col_params<PBN>(p, colp, tn * PBN, lane);
+            const int n0 = tn * PBN + (half > 0 ? PBN / 2 : 0);
+            stage_col_params<PBN>(p, colp, n0, lane);
             const int buf = tcount & 1;
             const uint32_t use = static_cast<uint32_t>(tcount >> 1);
             if (!mbar_wait_warp(&tmem_full[buf], use & 1u, abort_flag)) {
@@ -388,7 +399,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             const float sa = (m < p.M) ? __ldg(p.s_a + m) : 0.0f;
             const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
                                    static_cast<uint32_t>(buf * PBN);
-            store_tile_rows<PBN, kAcc>(p, tmY, t_row, ebuf, colp, tn * PBN, row0, sa, lane);
+            store_tile_rows<PBN, kAcc>(p, tmY, t_row, ebuf, colp, n0, row0, sa, lane, half < 0 ? PBN : PBN / 2);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(buf == 0 ? tmem_empty_leader0 : tmem_empty_leader1);
@@ -463,18 +474,23 @@ tfq_status launch_scaled_mm(const void* A, const float* s_a, const void* W, cons
     const int64_t tiles = static_cast<int64_t>(a.m_tiles) * a.n_tiles;
     if (tiles > INT32_MAX) return fail(TFQ_EUNSUPPORTED, "too many output tiles");
     if (use_pair_kernel(M, ds->sm_count)) {
-        CUtensorMap tmBh;
+        CUtensorMap tmBh, tmBq;
         st = encode_tensor_map_2d(&tmBh, CU_TENSOR_MAP_DATA_TYPE_UINT8, W, K, N, K, BK, PairCfg<256>::kBHalf,
+                                  CU_TENSOR_MAP_SWIZZLE_128B);
+        if (st != TFQ_OK) return st;
+        st = encode_tensor_map_2d(&tmBq, CU_TENSOR_MAP_DATA_TYPE_UINT8, W, K, N, K, BK, PairCfg<256>::kBHalf / 2,
                                   CU_TENSOR_MAP_SWIZZLE_128B);
         if (st != TFQ_OK) return st;
         const int64_t pair_tiles = ((M + 255) / 256) * static_cast<int64_t>(a.n_tiles);
         const int clusters = static_cast<int>(std::min<int64_t>(pair_tiles, ds->sm_count / 2));
+        a.tail_halves = choose_tail_halves(pair_tiles, clusters);
         a.round_ctr = take_round_counter(ds);
         if (a.round_ctr != nullptr) {
             const cudaError_t e = cudaMemsetAsync(a.round_ctr, 0, sizeof(unsigned), stream);
             if (e != cudaSuccess) return fail(TFQ_ECUDA, "clearing the round counter: %s", cudaGetErrorString(e));
         }
-        scaled_mm_pair_kernel<256, kAcc><<<2 * clusters, THREADS, PairCfg<256>::kSmem, stream>>>(tmA, tmBh, tmY, a);
+        scaled_mm_pair_kernel<256, kAcc><<<2 * clusters, THREADS, PairCfg<256>::kSmem, stream>>>(tmA, tmBh, tmBq,
+                                                                                              tmY, a);
     } else {
         CUtensorMap tmB;
         st = encode_tensor_map_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, W, K, N, K, BK, BN,

@@ -75,6 +75,11 @@ struct GemmArgs {
     // tiles of a band that share an activation panel read it from L2 together
     // instead of drifting apart and re-reading it from DRAM.  Null: no pacing.
     unsigned* round_ctr;
+    // CTA-pair kernel: when the last round has at most half as many tiles as
+    // there are clusters, each of its tiles is split along N into two
+    // half-width tiles (PBN / 2 columns, two clusters each), so that the
+    // round takes about half a tile's time instead of a whole one.
+    int tail_halves = 0;
 };
 
 #ifndef TFQ_PACING_WAIT_NS
@@ -261,14 +266,15 @@ __device__ __forceinline__ void store_tile_chunk(const GemmArgs& p, const CUtens
 // at a time (store_tile_chunk).  `t_row` is the TMEM address of this warp's
 // 32 lanes at the tile's first column; colp holds the tile's column scales
 // and bias.
+// `ncols` (a multiple of EPI_COLS, at most kBN): columns of the tile to store.
 template <int kBN, int kAcc>
 __device__ __forceinline__ void store_tile_rows(const GemmArgs& p, const CUtensorMap& tmY, uint32_t t_row,
                                                 uint8_t* ebuf, const float* colp, int n_tile0, int row0, float sa,
-                                                int lane) {
+                                                int lane, int ncols = kBN) {
     const float2 sa2 = make_float2(sa, sa);
     const uint64_t y_policy = make_l2_policy_evict_first();
 #pragma unroll 1
-    for (int c = 0; c < kBN / EPI_COLS; ++c)
+    for (int c = 0; c < ncols / EPI_COLS; ++c)
         store_tile_chunk<kBN, kAcc>(p, tmY, t_row, ebuf, colp, n_tile0, row0, sa2, y_policy, lane, c);
 }
 
@@ -291,6 +297,35 @@ __device__ __forceinline__ void pair_tile_coords(int t, int m_tiles, int n_tiles
     const int r = t - gid * per_group;
     tm = first_m + r % gsize;
     tn = r / gsize;
+}
+
+// Work item w of a cluster of the CTA-pair kernel (w = cluster, cluster +
+// n_clusters, ...): tile t whole (half = -1) or, in a split last round
+// (GemmArgs::tail_halves), half `half` (0: first PBN / 2 columns, 1: the
+// rest) of tile t.  Returns false past the last item.
+__device__ __forceinline__ bool pair_work_item(int w, int total_tiles, int n_clusters, int tail_halves, int& t,
+                                               int& half) {
+    const int whole = tail_halves ? (total_tiles / n_clusters) * n_clusters : total_tiles;
+    if (w < whole) {
+        t = w;
+        half = -1;
+        return true;
+    }
+    const int j = w - whole;
+    if (!tail_halves || j >= 2 * (total_tiles - whole)) return false;
+    t = whole + (j >> 1);
+    half = j & 1;
+    return true;
+}
+
+// Host side: split the last round when it holds at most n_clusters / 2 tiles.
+inline int choose_tail_halves(int64_t total_tiles, int64_t n_clusters) {
+#ifdef TFQ_GEMM_NO_TAIL_HALVES
+    return 0;
+#else
+    const int64_t last = total_tiles % n_clusters;
+    return (last > 0 && 2 * last <= n_clusters) ? 1 : 0;
+#endif
 }
 
 #ifndef TFQ_GEMM_PAIR_MIN_M

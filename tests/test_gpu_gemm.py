@@ -149,3 +149,13 @@ def test_pair_kernel_several_tiles_per_cluster(M, N, K):
     tiles, so both TMEM accumulators are reused and the cluster pacing,
     the band raster and the accumulator hand-over run for real; full compare."""
     _run_case(M, N, K, True, seed=M + N + K)
+
+
+@pytest.mark.parametrize("M,N,K", [(2523, 1864, 400), (2523, 1992, 256), (4096, 4096, 256), (6889, 3072, 384)])
+def test_pair_kernel_split_last_round(M, N, K):
+    """Shapes whose last round holds at most half as many tiles as there are
+    clusters (80 of 74, 256, 324 tiles): the last round's tiles run as two
+    half-width tiles on two clusters each.  Ragged N puts the split on a
+    partial tile (72 valid columns: the second half is empty; 200: the second
+    half holds 72), ragged M and K tails; full compare."""
+    _run_case(M, N, K, True, seed=5 * M + N + K)

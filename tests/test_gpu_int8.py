@@ -149,3 +149,9 @@ def test_int8_rounding_edges(K):
         q_ref, s_ref = _gpu.oracle_quant_int8(x, qmax)
         np.testing.assert_array_equal(s.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
         np.testing.assert_array_equal(q.cpu().numpy().view(np.int8), q_ref)
+
+
+@pytest.mark.parametrize("M,N,K", [(2523, 1992, 256), (4096, 4096, 128)])
+def test_int8_split_last_round(M, N, K):
+    """The INT8 pair kernel with its last round split into half-width tiles."""
+    _case(M, N, K, True, seed=M + 5 * N + K)
