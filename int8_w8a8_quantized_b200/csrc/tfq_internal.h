@@ -58,9 +58,11 @@ tfq_status encode_tensor_map_2d(CUtensorMap* map, CUtensorMapDataType dtype, con
 tfq_status launch_quant_rows(const void* x, int64_t rows, int64_t K, float qmax, bool out_int8, void* q, float* s,
                              cudaStream_t stream, DeviceState* ds);
 
-// Self-check: the quantizer's division next to the IEEE division.
+// MXFP8 quantizer (E4M3 codes, one E8M0 scale per 32 values).
 tfq_status launch_quant_mxfp8(const void* x, int64_t rows, int64_t K, void* q, void* sf, cudaStream_t stream,
                               DeviceState* ds);
+
+// Self-check: the quantizer's division next to the IEEE division.
 tfq_status launch_div_selftest(const float* a, const float* b, int64_t n, float* ours, float* ieee,
                                cudaStream_t stream);
 
