@@ -253,14 +253,15 @@ TFQ_API tfq_status tfq_scaled_fp8_linear_noalloc(const void *A_q, const float *s
 
 /*
  * Self-check of the division the quantizers use (a branch-free correctly
- * rounded fp32 division from the row's reciprocal, Markstein's method; the
- * pages fix x / s, see the conventions above).  For i < n writes
+ * rounded fp32 division from a two-term reciprocal of the row scale and one
+ * Markstein correction; the pages fix x / s, see the conventions above).
+ * For i < n writes
  *   ours[i] = the quantizers' quotient a[i] / b[i],
  *   ieee[i] = the CUDA IEEE round-to-nearest quotient __fdiv_rn(a[i], b[i]);
- * the two agree bit for bit when |a| >= 2^-102 and 2^-49 <= b <= 2^125
- * (every row scale the quantizers use this division for); for smaller |a|
- * both quotients are below 2^-53 in magnitude with the sign of a, so they
- * give the same E4M3 and INT8 codes.  All pointers are device
+ * the two agree bit for bit when |a / b| >= 2^-58 and 2^-49 <= b <= 2^64
+ * (every row scale the quantizers use this division for); for smaller
+ * |a / b| both quotients are below 2^-53 in magnitude with the sign of a,
+ * so they give the same E4M3 and INT8 codes.  All pointers are device
  * pointers of n floats, 4-byte aligned.  Errors: TFQ_EINVAL (n < 0, null
  * pointer with n > 0).
  */

@@ -107,18 +107,30 @@ def _stream_handle(stream) -> int:
     return int(stream.cuda_stream) if hasattr(stream, "cuda_stream") else int(stream)
 
 
-def _require(t, dtype, ndim, name):
+def _require(t, dtype, ndim, name, device=None):
+    """Checks a tensor argument: a contiguous CUDA tensor of `dtype` (an E4M3
+    code tensor may also be torch.float8_e4m3fn: the same bytes) with `ndim`
+    dimensions, on `device` when given (every operand of one call must live
+    on one GPU)."""
     import torch
     if not isinstance(t, torch.Tensor):
         raise TypeError(f"{name} must be a torch.Tensor")
     if not t.is_cuda:
         raise ValueError(f"{name} must be a CUDA tensor")
-    if t.dtype != dtype:
+    e4m3 = getattr(torch, "float8_e4m3fn", None)
+    if t.dtype != dtype and not (dtype == torch.uint8 and e4m3 is not None and t.dtype == e4m3 and
+                                 name in _E4M3_OPERANDS):
         raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
     if t.dim() != ndim:
         raise ValueError(f"{name} must be {ndim}-D")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, the other operands on {device}")
+
+
+# Arguments that hold E4M3FN codes (uint8, or torch.float8_e4m3fn views of them).
+_E4M3_OPERANDS = ("q", "A_q", "W_q")
 
 
 def tfq_quant_act_fp8_per_token(x, qmax: float = 448.0, q=None, s=None, stream=None):
@@ -130,8 +142,8 @@ def tfq_quant_act_fp8_per_token(x, qmax: float = 448.0, q=None, s=None, stream=N
         q = torch.empty((M, K), dtype=torch.uint8, device=x.device)
     if s is None:
         s = torch.empty((M,), dtype=torch.float32, device=x.device)
-    _require(q, torch.uint8, 2, "q")
-    _require(s, torch.float32, 1, "s")
+    _require(q, torch.uint8, 2, "q", x.device)
+    _require(s, torch.float32, 1, "s", x.device)
     if tuple(q.shape) != (M, K) or tuple(s.shape) != (M,):
         raise ValueError("output shapes do not match x")
     with torch.cuda.device(x.device):
@@ -156,8 +168,8 @@ def tfq_quant_weight_per_channel(w, dtype: str = "fp8", qmax: float | None = Non
         q = torch.empty((N, K), dtype=qdt, device=w.device)
     if s is None:
         s = torch.empty((N,), dtype=torch.float32, device=w.device)
-    _require(q, qdt, 2, "q")
-    _require(s, torch.float32, 1, "s")
+    _require(q, qdt, 2, "q", w.device)
+    _require(s, torch.float32, 1, "s", w.device)
     if tuple(q.shape) != (N, K) or tuple(s.shape) != (N,):
         raise ValueError("output shapes do not match w")
     with torch.cuda.device(w.device):
@@ -172,20 +184,21 @@ def tfq_scaled_fp8_linear(A_q, s_a, W_q, s_w, bias=None, out=None, stream=None):
     -> out bf16 [M, N]."""
     import torch
     _require(A_q, torch.uint8, 2, "A_q")
-    _require(W_q, torch.uint8, 2, "W_q")
-    _require(s_a, torch.float32, 1, "s_a")
-    _require(s_w, torch.float32, 1, "s_w")
+    dev = A_q.device
+    _require(W_q, torch.uint8, 2, "W_q", dev)
+    _require(s_a, torch.float32, 1, "s_a", dev)
+    _require(s_w, torch.float32, 1, "s_w", dev)
     M, K = A_q.shape
     N, K2 = W_q.shape
     if K2 != K or s_a.shape[0] != M or s_w.shape[0] != N:
         raise ValueError("shape mismatch")
     if bias is not None:
-        _require(bias, torch.bfloat16, 1, "bias")
+        _require(bias, torch.bfloat16, 1, "bias", dev)
         if bias.shape[0] != N:
             raise ValueError("bias shape")
     if out is None:
         out = torch.empty((M, N), dtype=torch.bfloat16, device=A_q.device)
-    _require(out, torch.bfloat16, 2, "out")
+    _require(out, torch.bfloat16, 2, "out", dev)
     if tuple(out.shape) != (M, N):
         raise ValueError("out shape")
     with torch.cuda.device(A_q.device):
@@ -205,8 +218,8 @@ def tfq_quant_act_int8_per_token(x, qmax: float = 127.0, q=None, s=None, stream=
         q = torch.empty((M, K), dtype=torch.int8, device=x.device)
     if s is None:
         s = torch.empty((M,), dtype=torch.float32, device=x.device)
-    _require(q, torch.int8, 2, "q")
-    _require(s, torch.float32, 1, "s")
+    _require(q, torch.int8, 2, "q", x.device)
+    _require(s, torch.float32, 1, "s", x.device)
     if tuple(q.shape) != (M, K) or tuple(s.shape) != (M,):
         raise ValueError("output shapes do not match x")
     with torch.cuda.device(x.device):
@@ -221,20 +234,21 @@ def tfq_scaled_int8_linear(A_q, s_a, W_q, s_w, bias=None, out=None, stream=None)
     -> out bf16 [M, N]."""
     import torch
     _require(A_q, torch.int8, 2, "A_q")
-    _require(W_q, torch.int8, 2, "W_q")
-    _require(s_a, torch.float32, 1, "s_a")
-    _require(s_w, torch.float32, 1, "s_w")
+    dev = A_q.device
+    _require(W_q, torch.int8, 2, "W_q", dev)
+    _require(s_a, torch.float32, 1, "s_a", dev)
+    _require(s_w, torch.float32, 1, "s_w", dev)
     M, K = A_q.shape
     N, K2 = W_q.shape
     if K2 != K or s_a.shape[0] != M or s_w.shape[0] != N:
         raise ValueError("shape mismatch")
     if bias is not None:
-        _require(bias, torch.bfloat16, 1, "bias")
+        _require(bias, torch.bfloat16, 1, "bias", dev)
         if bias.shape[0] != N:
             raise ValueError("bias shape")
     if out is None:
         out = torch.empty((M, N), dtype=torch.bfloat16, device=A_q.device)
-    _require(out, torch.bfloat16, 2, "out")
+    _require(out, torch.bfloat16, 2, "out", dev)
     if tuple(out.shape) != (M, N):
         raise ValueError("out shape")
     with torch.cuda.device(A_q.device):
@@ -269,8 +283,8 @@ def tfq_quant_mxfp8(x, q=None, sf=None, stream=None):
         q = torch.empty((R, K), dtype=torch.uint8, device=x.device)
     if sf is None:
         sf = torch.empty((tfq_mxfp8_scale_bytes(R, K),), dtype=torch.uint8, device=x.device)
-    _require(q, torch.uint8, 2, "q")
-    _require(sf, torch.uint8, 1, "sf")
+    _require(q, torch.uint8, 2, "q", x.device)
+    _require(sf, torch.uint8, 1, "sf", x.device)
     if tuple(q.shape) != (R, K) or sf.numel() < tfq_mxfp8_scale_bytes(R, K):
         raise ValueError("output shapes do not match x")
     with torch.cuda.device(x.device):
@@ -284,20 +298,21 @@ def tfq_mxfp8_linear(A_q, sf_a, W_q, sf_w, bias=None, out=None, stream=None):
     from tfq_quant_mxfp8, bias bf16 [N] or None -> out bf16 [M, N]."""
     import torch
     _require(A_q, torch.uint8, 2, "A_q")
-    _require(W_q, torch.uint8, 2, "W_q")
-    _require(sf_a, torch.uint8, 1, "sf_a")
-    _require(sf_w, torch.uint8, 1, "sf_w")
+    dev = A_q.device
+    _require(W_q, torch.uint8, 2, "W_q", dev)
+    _require(sf_a, torch.uint8, 1, "sf_a", dev)
+    _require(sf_w, torch.uint8, 1, "sf_w", dev)
     M, K = A_q.shape
     N, K2 = W_q.shape
     if K2 != K or sf_a.numel() < tfq_mxfp8_scale_bytes(M, K) or sf_w.numel() < tfq_mxfp8_scale_bytes(N, K):
         raise ValueError("shape mismatch")
     if bias is not None:
-        _require(bias, torch.bfloat16, 1, "bias")
+        _require(bias, torch.bfloat16, 1, "bias", dev)
         if bias.shape[0] != N:
             raise ValueError("bias shape")
     if out is None:
         out = torch.empty((M, N), dtype=torch.bfloat16, device=A_q.device)
-    _require(out, torch.bfloat16, 2, "out")
+    _require(out, torch.bfloat16, 2, "out", dev)
     if tuple(out.shape) != (M, N):
         raise ValueError("out shape")
     with torch.cuda.device(A_q.device):

@@ -23,9 +23,10 @@
 // at most one segment (K <= 4096) is still in registers; a longer row is
 // read again, which hits L2 because pass 1 loaded it with an evict_last
 // cache policy (so HBM sees 2 bytes read and 1 written per element).  The
-// division is a branch-free correctly rounded one (Markstein's method from
-// the row's reciprocal); two values are converted per cvt instruction and a
-// lane stores 8 codes at a time (a warp writes 256 contiguous bytes).
+// division is a branch-free correctly rounded one (a two-term reciprocal of
+// the row scale and one Markstein correction, four packed instructions per
+// pair of values); two values are converted per cvt instruction and a lane
+// stores 8 codes at a time (a warp writes 256 contiguous bytes).
 #include <cuda_bf16.h>
 
 #include <algorithm>
@@ -68,14 +69,52 @@ __device__ __forceinline__ uint32_t int8x2_rn(float2 t) {
 // (a = -0 may give +0 here; the caller restores the sign, see quantize8).
 // Five packed fp32x2 instructions (sm_100: two IEEE round-to-nearest
 // operations each, exactly the scalar ones) per pair of elements, no
-// branch; nb = -b.  Checked against the IEEE division __fdiv_rn by
-// tfq_selftest_div_rn.
+// branch; nb = -b.  Kept as the reference form (TFQ_QUANT_DW_RCP=0); the
+// quantizers use the four-instruction form below.  Both are checked against
+// the IEEE division __fdiv_rn by tfq_selftest_div_rn.
 __device__ __forceinline__ float2 div2_rn_from_rcp_unsigned_zero(float2 a, float2 nb, float2 y) {
     const float2 q0 = __fmul2_rn(a, y);
     const float2 r0 = __ffma2_rn(q0, nb, a);
     const float2 q1 = __ffma2_rn(r0, y, q0);
     const float2 r1 = __ffma2_rn(q1, nb, a);
     return __ffma2_rn(r1, y, q1);
+}
+
+// The same quotient in four packed instructions, from a two-term reciprocal
+// y = RN(1/b), yl = RN((1 - b*y) * y) (1 - b*y is exact in one FMA and at
+// most 2^-24 in magnitude, so y + yl is 1/b within 2^-47 relative).  Then
+// q1 = RN(a*y + RN(a*yl)) is within half an ulp plus 2^-46 relative of a/b,
+// hence faithful, and one Markstein step rounds it correctly.  Needs yl and
+// a*yl normal, which holds for 2^-49 <= b <= 2^64 wherever |a/b| >= 2^-58
+// (rows with a larger scale take the IEEE division; smaller quotients are
+// below every code's rounding threshold and keep the sign of a, +0 for
+// a = -0 as above).
+__device__ __forceinline__ float2 div2_rn_from_rcp2_unsigned_zero(float2 a, float2 nb, float2 y, float2 yl) {
+    const float2 q1 = __ffma2_rn(a, y, __fmul2_rn(a, yl));
+    const float2 r = __ffma2_rn(q1, nb, a);
+    return __ffma2_rn(r, y, q1);
+}
+
+#ifndef TFQ_QUANT_DW_RCP
+#define TFQ_QUANT_DW_RCP 1  // 1: the four-instruction division from a two-term reciprocal
+#endif
+
+// Largest row scale the reciprocal-based division takes; larger ones use __fdiv_rn.
+constexpr float kDivMaxScale = TFQ_QUANT_DW_RCP ? 0x1p64f : 0x1p125f;
+
+// Low term of the row's reciprocal (0 when the five-instruction division is used).
+__device__ __forceinline__ float rcp_low(float sc, float rcp) {
+    return TFQ_QUANT_DW_RCP ? __fmul_rn(__fmaf_rn(-sc, rcp, 1.0f), rcp) : 0.0f;
+}
+
+// a / b for the quantizers (see the two functions above).
+__device__ __forceinline__ float2 div2_rn_unsigned_zero(float2 a, float b, float y, float yl) {
+#if TFQ_QUANT_DW_RCP
+    return div2_rn_from_rcp2_unsigned_zero(a, make_float2(-b, -b), make_float2(y, y), make_float2(yl, yl));
+#else
+    (void)yl;
+    return div2_rn_from_rcp_unsigned_zero(a, make_float2(-b, -b), make_float2(y, y));
+#endif
 }
 
 namespace {
@@ -93,14 +132,13 @@ namespace {
 // exact because every other quotient already carries the sign of a, and an
 // INT8 code has no negative zero.)
 template <bool kInt8, bool kClamp, bool kIeeeDiv>
-__device__ __forceinline__ uint32_t quantize2(uint32_t w, float sc, float rcp, float qmax) {
+__device__ __forceinline__ uint32_t quantize2(uint32_t w, float sc, float rcp, float rcp_lo, float qmax) {
     float a, b;
     if constexpr (kIeeeDiv) {
         a = __fdiv_rn(bf16_lo(w), sc);
         b = __fdiv_rn(bf16_hi(w), sc);
     } else {
-        const float2 t = div2_rn_from_rcp_unsigned_zero(make_float2(bf16_lo(w), bf16_hi(w)), make_float2(-sc, -sc),
-                                                       make_float2(rcp, rcp));
+        const float2 t = div2_rn_unsigned_zero(make_float2(bf16_lo(w), bf16_hi(w)), sc, rcp, rcp_lo);
         a = t.x;
         b = t.y;
     }
@@ -116,11 +154,11 @@ __device__ __forceinline__ uint32_t quantize2(uint32_t w, float sc, float rcp, f
 }
 
 template <bool kInt8, bool kClamp, bool kIeeeDiv>
-__device__ __forceinline__ uint2 quantize8(uint4 v, float sc, float rcp, float qmax) {
-    const uint32_t p0 = quantize2<kInt8, kClamp, kIeeeDiv>(v.x, sc, rcp, qmax);
-    const uint32_t p1 = quantize2<kInt8, kClamp, kIeeeDiv>(v.y, sc, rcp, qmax);
-    const uint32_t p2 = quantize2<kInt8, kClamp, kIeeeDiv>(v.z, sc, rcp, qmax);
-    const uint32_t p3 = quantize2<kInt8, kClamp, kIeeeDiv>(v.w, sc, rcp, qmax);
+__device__ __forceinline__ uint2 quantize8(uint4 v, float sc, float rcp, float rcp_lo, float qmax) {
+    const uint32_t p0 = quantize2<kInt8, kClamp, kIeeeDiv>(v.x, sc, rcp, rcp_lo, qmax);
+    const uint32_t p1 = quantize2<kInt8, kClamp, kIeeeDiv>(v.y, sc, rcp, rcp_lo, qmax);
+    const uint32_t p2 = quantize2<kInt8, kClamp, kIeeeDiv>(v.z, sc, rcp, rcp_lo, qmax);
+    const uint32_t p3 = quantize2<kInt8, kClamp, kIeeeDiv>(v.w, sc, rcp, rcp_lo, qmax);
     if constexpr (kInt8) return make_uint2(__byte_perm(p0, p1, 0x5410), __byte_perm(p2, p3, 0x5410));
     // E4M3 codes keep the sign of (negative) zero
     const uint32_t lo = p0 | (p1 << 16) | sign_bytes(v.x, v.y);
@@ -156,11 +194,11 @@ __device__ __forceinline__ uint64_t l2_policy_evict_first() {
 
 template <bool kInt8, bool kClamp, bool kIeeeDiv, int SEG>
 __device__ __forceinline__ void quantize_segment(const uint4 (&v)[SEG], uint2* qrow, int base, int lane, int units,
-                                                 float sc, float rcp, float qmax) {
+                                                 float sc, float rcp, float rcp_lo, float qmax) {
 #pragma unroll
     for (int j = 0; j < SEG; ++j) {
         const int idx = base + lane + 32 * j;
-        if (idx < units) qrow[idx] = quantize8<kInt8, kClamp, kIeeeDiv>(v[j], sc, rcp, qmax);
+        if (idx < units) qrow[idx] = quantize8<kInt8, kClamp, kIeeeDiv>(v[j], sc, rcp, rcp_lo, qmax);
     }
 }
 
@@ -231,22 +269,23 @@ __global__ void __launch_bounds__(256, rows_ctas_per_sm<SEG>()) quant_rows_kerne
         for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
         const float sc = __fdiv_rn(fmaxf(amax, 1e-12f), qmax);
         const float rcp = __frcp_rn(sc);
+        const float rcp_lo = rcp_low(sc, rcp);
         if (lane == 0) s[r] = sc;
         uint2* qrow = reinterpret_cast<uint2*>(q + r * K);
         // pass 2: a row of one segment is still in registers; longer rows are
         // read again (from L2: the same row was read microseconds earlier)
-        if (sc <= 0x1p125f) {
+        if (sc <= kDivMaxScale) {
             if (one_segment) {
-                quantize_segment<kInt8, kClamp, false, SEG>(v, qrow, 0, lane, units, sc, rcp, qmax);
+                quantize_segment<kInt8, kClamp, false, SEG>(v, qrow, 0, lane, units, sc, rcp, rcp_lo, qmax);
             } else {
                 for (int base = 0; base < units; base += 32 * SEG) {
                     load_segment<SEG>(v, row, base, lane, units, drop);
-                    quantize_segment<kInt8, kClamp, false, SEG>(v, qrow, base, lane, units, sc, rcp, qmax);
+                    quantize_segment<kInt8, kClamp, false, SEG>(v, qrow, base, lane, units, sc, rcp, rcp_lo, qmax);
                 }
             }
-        } else {  // reciprocal would be subnormal: IEEE division (warp-uniform branch)
+        } else {  // a huge scale: IEEE division (warp-uniform branch)
             for (int u = lane; u < units; u += 32)
-                qrow[u] = quantize8<kInt8, kClamp, true>(ldg_nc_v4(row + u), sc, rcp, qmax);
+                qrow[u] = quantize8<kInt8, kClamp, true>(ldg_nc_v4(row + u), sc, rcp, 0.0f, qmax);
         }
 #if TFQ_QUANT_L2_KEEP
         if (!one_segment) release_row_l2(row, units, lane);
@@ -336,13 +375,14 @@ __global__ void __launch_bounds__(kStagedThreads) quant_rows_staged_kernel(const
         const float sc = __fdiv_rn(fmaxf(amax, 1e-12f), qmax);
         if (tid == 0) s[r] = sc;
         uint2* qrow = reinterpret_cast<uint2*>(q + r * K);
-        if (sc <= 0x1p125f) {
+        if (sc <= kDivMaxScale) {
             const float rcp = __frcp_rn(sc);
+            const float rcp_lo = rcp_low(sc, rcp);
             for (int u = tid; u < units; u += kStagedThreads)
-                qrow[u] = quantize8<kInt8, kClamp, false>(row[u], sc, rcp, qmax);
-        } else {  // reciprocal would be subnormal: IEEE division (uniform across the CTA)
+                qrow[u] = quantize8<kInt8, kClamp, false>(row[u], sc, rcp, rcp_lo, qmax);
+        } else {  // a huge scale: IEEE division (uniform across the CTA)
             for (int u = tid; u < units; u += kStagedThreads)
-                qrow[u] = quantize8<kInt8, kClamp, true>(row[u], sc, 0.0f, qmax);
+                qrow[u] = quantize8<kInt8, kClamp, true>(row[u], sc, 0.0f, 0.0f, qmax);
         }
         __syncthreads();  // every thread is done with this buffer and with wmax
         if (tid == 0) {
@@ -417,18 +457,19 @@ __global__ void __launch_bounds__(256, grouped_ctas_per_sm<J>()) quant_grouped_r
         if (row_ok) {
             if (sub == 0) s[r] = sc;
             uint2* qrow = reinterpret_cast<uint2*>(q + r * K);
-            if (sc <= 0x1p125f) {
+            if (sc <= kDivMaxScale) {
                 const float rcp = __frcp_rn(sc);
+                const float rcp_lo = rcp_low(sc, rcp);
 #pragma unroll
                 for (int j = 0; j < J; ++j) {
                     const int u = sub + LPR * j;
-                    if (u < units) qrow[u] = quantize8<kInt8, kClamp, false>(v[j], sc, rcp, qmax);
+                    if (u < units) qrow[u] = quantize8<kInt8, kClamp, false>(v[j], sc, rcp, rcp_lo, qmax);
                 }
-            } else {  // reciprocal would be subnormal: IEEE division for this row
+            } else {  // a huge scale: IEEE division for this row
 #pragma unroll
                 for (int j = 0; j < J; ++j) {
                     const int u = sub + LPR * j;
-                    if (u < units) qrow[u] = quantize8<kInt8, kClamp, true>(v[j], sc, 0.0f, qmax);
+                    if (u < units) qrow[u] = quantize8<kInt8, kClamp, true>(v[j], sc, 0.0f, 0.0f, qmax);
                 }
             }
         }
@@ -444,7 +485,7 @@ __global__ void div_selftest_kernel(const float* __restrict__ a, const float* __
         const float r = __frcp_rn(y);
         // the packed form the quantizers use; both lanes carry the same
         // quotient, the sign of a zero result is restored as the quantizers do
-        const float2 t = div2_rn_from_rcp_unsigned_zero(make_float2(x, x), make_float2(-y, -y), make_float2(r, r));
+        const float2 t = div2_rn_unsigned_zero(make_float2(x, x), y, r, rcp_low(y, r));
         ours[i] = copysignf(t.y, x);
         ieee[i] = __fdiv_rn(x, y);
     }

@@ -1,9 +1,13 @@
-"""The quantizers' branch-free division (Markstein's method from the row's
-correctly rounded reciprocal) against CUDA's IEEE division __fdiv_rn, bit
-for bit, through the tfq_selftest_div_rn self-check entry point: every
+"""The quantizers' branch-free division (a two-term reciprocal of the row
+scale and one Markstein correction) against CUDA's IEEE division __fdiv_rn,
+bit for bit, through the tfq_selftest_div_rn self-check entry point: every
 finite bf16 numerator against row scales s = fl32(amax / qmax) drawn over
-the whole range the quantizers produce (including the 1e-12 floor), plus
-scales next to powers of two and random fp32 numerators."""
+the whole range the quantizers take this path for (the 1e-12 floor up to
+2^64; larger scales use the IEEE division), plus scales next to powers of
+two and random fp32 numerators.  Quotients below 2^-58 in magnitude, far
+below every code's rounding threshold, need only be tiny with the sign of
+the numerator."""
+
 import numpy as np
 import pytest
 import torch
@@ -12,6 +16,9 @@ from int8_w8a8_quantized_b200 import _capi
 from tests import _gpu
 
 pytestmark = pytest.mark.gpu
+
+# Largest row scale the quantizers divide by without __fdiv_rn.
+DIV_MAX_SCALE = np.float32(2.0 ** 64)
 
 
 def _all_finite_bf16():
@@ -31,11 +38,11 @@ def _run(a: np.ndarray, b: np.ndarray):
     torch.cuda.synchronize()
     o = ours.cpu().numpy()
     r = ieee.cpu().numpy()
-    exact = np.abs(a) >= np.float32(2.0 ** -102)
+    exact = np.abs(a.astype(np.float64) / b.astype(np.float64)) >= 2.0 ** -58
     bad = np.nonzero(exact & (o.view(np.uint32) != r.view(np.uint32)))[0]
     assert bad.size == 0, (f"{bad.size} mismatches; first a={a[bad[0]]!r} b={b[bad[0]]!r} "
                            f"ours={o[bad[0]]!r} ieee={r[bad[0]]!r}")
-    # tiny numerators: both quotients tiny (so both encode to +-0) with the sign of a
+    # tiny quotients: both tiny (so both encode to +-0) with the sign of a
     tiny = ~exact
     assert np.all(np.abs(o[tiny]) < 2.0 ** -53) and np.all(np.abs(r[tiny]) < 2.0 ** -53)
     assert np.array_equal(np.signbit(o[tiny]), np.signbit(a[tiny]))
@@ -48,9 +55,9 @@ def _scales(rng, n):
     amax = np.exp(rng.uniform(np.log(1e-12), np.log(3e38), n)).astype(np.float32)
     amax[: n // 8] = np.float32(1e-12)                    # the floor
     s = (np.maximum(amax, np.float32(1e-12)) / qmax).astype(np.float32)
-    s = np.minimum(s, np.float32(2.0 ** 125))             # larger scales use the IEEE division
+    s = np.minimum(s, DIV_MAX_SCALE)                      # larger scales use the IEEE division
     # scales just around powers of two and their neighbours
-    p2 = (2.0 ** rng.integers(-40, 120, n // 4)).astype(np.float32)
+    p2 = (2.0 ** rng.integers(-40, 64, n // 4)).astype(np.float32)
     s2 = np.concatenate([p2, np.nextafter(p2, np.float32(0)), np.nextafter(p2, np.float32(np.inf))])
     return np.concatenate([s, s2]).astype(np.float32)
 

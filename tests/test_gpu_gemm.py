@@ -159,3 +159,28 @@ def test_pair_kernel_split_last_round(M, N, K):
     partial tile (72 valid columns: the second half is empty; 200: the second
     half holds 72), ragged M and K tails; full compare."""
     _run_case(M, N, K, True, seed=5 * M + N + K)
+
+
+def test_float8_views_accepted():
+    """The Python binding takes torch.float8_e4m3fn tensors wherever it takes
+    E4M3 codes as uint8 (the same bytes): outputs identical to the uint8 path."""
+    from int8_w8a8_quantized_b200 import tfq_quant_act_fp8_per_token, tfq_quant_weight_per_channel, \
+        tfq_scaled_fp8_linear
+    x = workloads.activations(600, 512, seed=21, device="cuda")
+    w = workloads.weights(264, 512, seed=22, std=0.02, device="cuda")
+    b = workloads.bias(264, seed=23, device="cuda")
+    Wq, sw = tfq_quant_weight_per_channel(w, "fp8")
+    Wq8 = torch.empty((264, 512), dtype=torch.float8_e4m3fn, device="cuda")
+    _, sw8 = tfq_quant_weight_per_channel(w, "fp8", q=Wq8)
+    A, sa = tfq_quant_act_fp8_per_token(x)
+    A8 = torch.empty((600, 512), dtype=torch.float8_e4m3fn, device="cuda")
+    tfq_quant_act_fp8_per_token(x, q=A8)
+    assert torch.equal(Wq8.view(torch.uint8), Wq) and torch.equal(sw8, sw)
+    assert torch.equal(A8.view(torch.uint8), A)
+    y = tfq_scaled_fp8_linear(A, sa, Wq, sw, b)
+    y8 = tfq_scaled_fp8_linear(A8, sa, Wq8, sw, b)
+    assert torch.equal(y, y8)
+    with pytest.raises(TypeError):
+        tfq_scaled_fp8_linear(A.view(torch.int8), sa, Wq, sw, b)
+    with pytest.raises(ValueError):
+        tfq_scaled_fp8_linear(A, sa.cpu(), Wq, sw, b)

@@ -127,7 +127,7 @@ def test_int8_tensor_wrappers():
 def test_int8_rounding_edges(K):
     """INT8 codes where x/s is an exact half-integer (round half to even
     decides), signed zeros, values that round to 0, rows below the 1e-12
-    floor and rows whose scale exceeds 2^125 (the IEEE-division branch), for
+    floor and rows whose scale exceeds 2^64 (the IEEE-division branch), for
     the grouped, one-warp-per-row and shared-memory-staged kernels."""
     halves = torch.arange(-127, 127, dtype=torch.float32) + 0.5
     row = torch.cat([torch.tensor([127.0, -127.0]), halves, torch.tensor([-0.0, 0.0, 0.25, -0.25, 0.75, 1e-30])])
@@ -140,7 +140,7 @@ def test_int8_rounding_edges(K):
     x[3] = -0.0
     x[4, :4] = torch.tensor([1e-13, -3e-13, 2e-13, -1e-14])   # below the floor
     x[5] = base * 3.0                  # a scale that is not a power of two
-    x[6] = base * (3.0e38 / 127.0)     # with qmax <= 2: s > 2^125
+    x[6] = base * (3.0e38 / 127.0)     # s > 2^64 for every qmax
     x[7] = -base
     x = x.to(torch.bfloat16).cuda()
     assert torch.isfinite(x.float()).all()

@@ -98,12 +98,15 @@ def test_rounding_edges():
 @pytest.mark.parametrize("K", [256, 5120, 16384])
 @pytest.mark.parametrize("qmax", [1.0, 2.0, 448.0])
 def test_huge_magnitude_rows(qmax, K):
-    """Rows near the bf16 maximum: with a small qmax the scale exceeds 2^125
-    and the kernel takes its IEEE-division branch for the row (grouped,
+    """Rows near the bf16 maximum and rows whose scale is near 2^64: above it
+    the kernel takes its IEEE-division branch for the row (grouped,
     one-warp-per-row and shared-memory-staged kernels)."""
-    x = workloads.activations(40, K, seed=3, device="cuda").float()
+    x = workloads.activations(48, K, seed=3, device="cuda").float()
     x[:20] *= 3.0e38 / x[:20].abs().amax(dim=1, keepdim=True)
     x[20:30] *= 1.0e30
+    # scales on both sides of 2^64, where the reciprocal-based division hands over to __fdiv_rn
+    near = torch.tensor([0.5, 0.99, 0.999, 1.0, 1.001, 1.01, 2.0, 1.0], device="cuda")[:, None]
+    x[40:48] *= near * (2.0 ** 64) * qmax / x[40:48].abs().amax(dim=1, keepdim=True)
     x = x.to(torch.bfloat16)
     assert torch.isfinite(x.float()).all()
     _assert_fp8_equal(x, qmax)
