@@ -221,11 +221,17 @@ class ClockSampler:
                 sm_max = float(pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM))
             except Exception:
                 sm_max = None
+            try:  # read only: the enforced board power limit sets the clock a power-bound kernel gets
+                limit_w = pynvml.nvmlDeviceGetEnforcedPowerLimit(h) / 1000.0
+            except Exception:
+                limit_w = None
             if not self.samples:
                 return None
             reasons = sorted(n for n, bit in self.REASON_BITS.items() if any(r & bit for _, _, r in self.samples))
             return {"sm_mhz": statistics.median(c for c, _, _ in self.samples), "sm_max_mhz": sm_max,
-                    "power_w_max": max(p for _, p, _ in self.samples), "samples": len(self.samples),
+                    "power_w_max": max(p for _, p, _ in self.samples),
+                    "power_w_median": statistics.median(p for _, p, _ in self.samples),
+                    "power_limit_w": limit_w, "samples": len(self.samples),
                     "source": "nvml, 10 ms", "reasons": reasons}
         if self.proc is None:
             return None

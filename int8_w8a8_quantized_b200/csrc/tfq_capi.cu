@@ -99,30 +99,12 @@ DeviceState* current_device_state(tfq_status* st) {
     return ds;
 }
 
-unsigned* take_round_counter(DeviceState* ds, uint32_t increments, uint32_t* base) {
-    *base = 0;
-    if (ds->round_ctrs == nullptr || ds->round_slots <= 0 || ds->round_slots > DeviceState::kMaxRoundSlots)
-        return nullptr;
+unsigned* take_round_counter(DeviceState* ds) {
+    if (ds->round_ctrs == nullptr || ds->round_slots <= 0) return nullptr;
     std::lock_guard<std::mutex> lock(g_mutex);
     const int slot = ds->next_round_slot;
     ds->next_round_slot = (slot + 1) % ds->round_slots;
-    *base = ds->round_issued[slot];
-    ds->round_issued[slot] += increments;  // wraps modulo 2^32, as the counter does
     return ds->round_ctrs + 32 * slot;
-}
-
-void restart_round_totals(DeviceState* ds) {
-    std::lock_guard<std::mutex> lock(g_mutex);
-    for (int i = 0; i < DeviceState::kMaxRoundSlots; ++i) ds->round_issued[i] = 0;
-}
-
-tfq_status reset_round_counters(DeviceState* ds) {
-    if (ds->round_ctrs == nullptr || ds->round_slots <= 0) return TFQ_OK;
-    std::lock_guard<std::mutex> lock(g_mutex);
-    const cudaError_t e = cudaMemset(ds->round_ctrs, 0, 128 * static_cast<size_t>(ds->round_slots));
-    if (e != cudaSuccess) return fail(TFQ_ECUDA, "resetting the round counters: %s", cudaGetErrorString(e));
-    for (int i = 0; i < DeviceState::kMaxRoundSlots; ++i) ds->round_issued[i] = 0;
-    return TFQ_OK;
 }
 
 tfq_status encode_tensor_map_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, uint64_t inner,
@@ -331,16 +313,7 @@ tfq_status tfq_device_error(void* stream) {
     e = cudaMemcpy(&word, ds->err_word, sizeof word, cudaMemcpyDeviceToHost);
     if (e == cudaSuccess && word != 0) e = cudaMemset(ds->err_word, 0, sizeof(uint32_t));
     if (e != cudaSuccess) return fail(TFQ_ECUDA, "reading the error word: %s", cudaGetErrorString(e));
-    if (word != 0) {
-        // a GEMM that gave up added fewer rounds than its slot's total assumes
-        if (word & (kErrGemmProducer | kErrGemmMma | kErrGemmEpilogue | kErrGemmDrain)) {
-            e = cudaDeviceSynchronize();  // no GEMM of any stream may still be counting
-            if (e != cudaSuccess) return fail(TFQ_ECUDA, "cudaDeviceSynchronize: %s", cudaGetErrorString(e));
-            const tfq_status rs = reset_round_counters(ds);
-            if (rs != TFQ_OK) return rs;
-        }
-        return fail(TFQ_ETIMEOUT, "a bounded device wait ran out (error bits 0x%x)", word);
-    }
+    if (word != 0) return fail(TFQ_ETIMEOUT, "a bounded device wait ran out (error bits 0x%x)", word);
     return TFQ_OK;
 }
 

@@ -297,7 +297,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             int round = 0, t, half;
             for (int w = cluster; ok && pair_work_item(w, total_tiles, n_clusters, p.tail_halves, t, half);
                  w += n_clusters, ++round) {
-                if (rank == 0) pace_round(p.round_ctr, p.round_base, round, total_tiles, n_clusters);
+                if (rank == 0) pace_round(p.round_ctr, round, total_tiles, n_clusters);
                 int tm, tn;
                 pair_tile_coords(t, m_tiles, p.n_tiles, p.group_m, p.band_n, tm, tn);
                 // a half tile: PBN / 2 columns, PBN / 4 B rows per CTA (tmBq's box)
@@ -330,6 +330,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                     if (issued_phase[i] >= 0 &&
                         !mbar_wait(&full[i], static_cast<uint32_t>(issued_phase[i]), nullptr))
                         atomicOr(p.err, kErrGemmDrain);
+                pacing_done(p.round_ctr, n_clusters);
             }
         }
     } else if (warp == 1) {
@@ -484,9 +485,7 @@ tfq_status launch_scaled_mm(const void* A, const float* s_a, const void* W, cons
         const int64_t pair_tiles = ((M + 255) / 256) * static_cast<int64_t>(a.n_tiles);
         const int clusters = static_cast<int>(std::min<int64_t>(pair_tiles, ds->sm_count / 2));
         a.tail_halves = choose_tail_halves(pair_tiles, clusters);
-        // one count per work item: the tiles, with the last round's counted twice when it is split
-        const int64_t items = a.tail_halves ? 2 * pair_tiles - pair_tiles / clusters * clusters : pair_tiles;
-        a.round_ctr = take_round_counter(ds, static_cast<uint32_t>(items), &a.round_base);
+        a.round_ctr = take_round_counter(ds);
         scaled_mm_pair_kernel<256, kAcc><<<2 * clusters, THREADS, PairCfg<256>::kSmem, stream>>>(tmA, tmBh, tmBq,
                                                                                               tmY, a);
     } else {

@@ -67,18 +67,18 @@ struct GemmArgs {
     int band_n;
     int group_m;
     uint32_t* err;
-    // Cluster pacing (CTA-pair kernel): a counter that holds round_base when
-    // the launch starts (it is never reset: the host keeps the running total
-    // of each counter, so no memset precedes the kernel in the stream); the
-    // even CTA's producer adds 1 after issuing each tile's loads and, before
-    // its round r, waits (up to TFQ_PACING_WAIT_NS, then goes on: a
-    // performance hint, not a dependency) until every cluster has issued its
-    // rounds before r.  Keeps the clusters within one tile of each other, so
-    // the N tiles of a band that share an activation panel read it from L2
-    // together instead of drifting apart and re-reading it from DRAM.  Null:
-    // no pacing.
+    // Cluster pacing (CTA-pair kernel): round_ctr[0] is zero when the launch
+    // starts; the even CTA's producer adds 1 after issuing each tile's loads
+    // and, before its round r, waits (up to TFQ_PACING_WAIT_NS, then goes on:
+    // a performance hint, not a dependency) until every cluster has issued
+    // its rounds before r.  Keeps the clusters within one tile of each other,
+    // so the N tiles of a band that share an activation panel read it from L2
+    // together instead of drifting apart and re-reading it from DRAM.
+    // round_ctr[1] counts the clusters that are done; the last one sets both
+    // words back to zero for the next launch given this slot (pacing_done),
+    // so no memset sits between kernels in the stream, and a CUDA graph
+    // replays the launch with the counter it expects.  Null: no pacing.
     unsigned* round_ctr;
-    unsigned round_base = 0;
     // CTA-pair kernel: when the last round has at most half as many tiles as
     // there are clusters, each of its tiles is split along N into two
     // half-width tiles (PBN / 2 columns, two clusters each), so that the
@@ -90,16 +90,29 @@ struct GemmArgs {
 #define TFQ_PACING_WAIT_NS 200000ull
 #endif
 
-__device__ __forceinline__ void pace_round(const unsigned* ctr, unsigned base, int round, int total_tiles,
-                                           int n_clusters) {
+__device__ __forceinline__ void pace_round(const unsigned* ctr, int round, int total_tiles, int n_clusters) {
     if (ctr == nullptr || round < 1) return;
-    const int need = min(total_tiles, round * n_clusters);
+    const unsigned need = static_cast<unsigned>(min(total_tiles, round * n_clusters));
     const uint64_t t0 = globaltimer_ns();
     for (uint32_t i = 0; i < TFQ_WAIT_LIMIT_POLLS; ++i) {
         unsigned v;
         asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ctr) : "memory");
-        if (static_cast<int>(v - base) >= need) return;  // modulo 2^32
+        if (v >= need) return;
         if (globaltimer_ns() - t0 > TFQ_PACING_WAIT_NS) return;
+    }
+}
+
+// Called once per cluster (the even CTA's producer thread) after its last
+// round-counter update: counts the cluster as done; the last one of the
+// launch sets the slot back to zero.  Every other cluster's round updates
+// precede its own done count (the fence), so nothing adds to the counter
+// after the reset.
+__device__ __forceinline__ void pacing_done(unsigned* ctr, int n_clusters) {
+    if (ctr == nullptr) return;
+    __threadfence();
+    if (atomicAdd(ctr + 1, 1u) == static_cast<unsigned>(n_clusters - 1)) {
+        atomicExch(ctr, 0u);
+        atomicExch(ctr + 1, 0u);
     }
 }
 

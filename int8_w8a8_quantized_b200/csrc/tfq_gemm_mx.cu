@@ -385,7 +385,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             bool ok = true;
             int round = 0;
             for (int t = cluster; t < total_tiles && ok; t += n_clusters, ++round) {
-                if (rank == 0) pace_round(p.round_ctr, p.round_base, round, total_tiles, n_clusters);
+                if (rank == 0) pace_round(p.round_ctr, round, total_tiles, n_clusters);
                 int tm, tn;
                 pair_tile_coords(t, m_tiles, p.n_tiles, p.group_m, p.band_n, tm, tn);
                 const int a_row = tm * 256 + static_cast<int>(rank) * 128;
@@ -419,6 +419,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                     if (issued_phase[i] >= 0 &&
                         !mbar_wait(&full[i], static_cast<uint32_t>(issued_phase[i]), nullptr))
                         atomicOr(p.err, kErrGemmDrain);
+                pacing_done(p.round_ctr, n_clusters);
             }
         }
     } else if (warp == 1) {
@@ -597,7 +598,7 @@ tfq_status launch_mxfp8_mm(const void* A, const uint8_t* sf_a, const void* W, co
         }
         const int64_t pair_tiles = ((M + 255) / 256) * static_cast<int64_t>(a.n_tiles);
         const int clusters = static_cast<int>(std::min<int64_t>(pair_tiles, ds->sm_count / 2));
-        a.round_ctr = take_round_counter(ds, static_cast<uint32_t>(pair_tiles), &a.round_base);  // one count per tile
+        a.round_ctr = take_round_counter(ds);
         mxfp8_mm_pair_kernel<<<2 * clusters, THREADS, MXP_SMEM_BYTES, stream>>>(tmA, tmBh, tmY, tmSA, tmSB, a, mx);
     } else {
         const int grid = static_cast<int>(std::min<int64_t>(tiles, ds->sm_count));

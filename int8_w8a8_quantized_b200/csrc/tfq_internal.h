@@ -26,16 +26,14 @@ struct DeviceState {
     int cc_major = 0, cc_minor = 0;
     size_t smem_optin = 0;          // max dynamic shared memory per block
     uint32_t* err_word = nullptr;   // device memory, one 32-bit word
-    // Round counters of the GEMM's cluster pacing (one 128-byte line each);
-    // launches take slots round-robin so that launches in flight at the same
-    // time on different streams do not share one.  A counter is never reset:
-    // round_issued[slot] is what it will read once every launch given that
-    // slot so far has finished, and a launch paces on the difference.
-    static constexpr int kMaxRoundSlots = 64;
+    // Round counters of the GEMM's cluster pacing (one 128-byte line each:
+    // the round count, then the count of clusters done); launches take slots
+    // round-robin so that launches in flight at the same time on different
+    // streams do not share one.  The last cluster of a launch to finish sets
+    // both back to zero, so no memset precedes a launch.
     unsigned* round_ctrs = nullptr;
     int round_slots = 0;
     int next_round_slot = 0;
-    uint32_t round_issued[kMaxRoundSlots] = {};
     bool gemm_attr_set[5] = {false, false, false, false, false};  // FP8, INT8, FP8/FP16 acc, MXFP8, MXFP8 pair
     bool quant_attr_set = false;   // dynamic shared memory limit of the staged-row quantizers
 };
@@ -73,18 +71,8 @@ tfq_status launch_div_selftest(const float* a, const float* b, int64_t n, float*
 // Self-check of the bounded wait: a wait on a barrier that never completes.
 tfq_status launch_wait_selftest(uint64_t limit_ns, cudaStream_t stream, DeviceState* ds);
 
-// Round-counter slot for the next GEMM launch on this device (thread safe):
-// the launch will add `increments` to it; *base receives the value the
-// counter holds once the slot's earlier launches have finished.
-unsigned* take_round_counter(DeviceState* ds, uint32_t increments, uint32_t* base);
-
-// Sets the host-side totals of the round counters to zero, for a caller
-// that has just cleared the counters on its stream (thread safe).
-void restart_round_totals(DeviceState* ds);
-
-// After a device-side wait gave up (the counts of that launch are short):
-// zeroes every round counter of the device and the host-side totals.
-tfq_status reset_round_counters(DeviceState* ds);
+// Round-counter slot for the next GEMM launch on this device (thread safe).
+unsigned* take_round_counter(DeviceState* ds);
 
 // Scaled FP8 GEMM with the fused scale/bias/BF16 epilogue.
 tfq_status launch_scaled_fp8_gemm(const void* A, const float* s_a, const void* W, const float* s_w,

@@ -118,10 +118,9 @@ extern "C" tfq_status tfq_scaled_fp8_linear_noalloc(const void* A_q, const float
     if (ds == nullptr) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     // The array keeps the previous call's contents: the error word must start
-    // at zero, and so does the round counter in the next 128-byte line (one
-    // clear for both; the host-side total of the counter restarts with it).
-    const cudaError_t e = cudaMemsetAsync(ds->err_word, 0, kGemmScratchBytes, s);
-    if (e != cudaSuccess) return fail(TFQ_ECUDA, "clearing the scratch words: %s", cudaGetErrorString(e));
-    restart_round_totals(ds);
+    // at zero (the round counter in the next line is left at zero by the
+    // kernel that used it last).
+    const cudaError_t e = cudaMemsetAsync(ds->err_word, 0, sizeof(uint32_t), s);
+    if (e != cudaSuccess) return fail(TFQ_ECUDA, "clearing the scratch word: %s", cudaGetErrorString(e));
     return launch_scaled_fp8_gemm(A_q, s_a, W_q, s_w, bias_bf16, M, N, K, out_bf16, s, ds);
 }
