@@ -127,3 +127,41 @@ def test_mxfp8_and_int8_concurrent_streams_match_serial():
         torch.cuda.synchronize()
         assert torch.equal(y_m, ref_m) and torch.equal(y_i, ref_i)
     _gpu.check_device_error()
+
+
+def test_pacing_slots_reused_eager_and_in_a_graph():
+    """A pair-kernel GEMM launched 70 times in a row (more launches than
+    pacing-counter slots, so slots are reused; each launch leaves its slot at
+    zero for the next) and replayed 5 times from a CUDA graph (the same slot
+    every replay): every result equals the first, no bounded wait runs out."""
+    lib = _gpu.lib()
+    g = torch.Generator().manual_seed(5)
+    M, N, K = 2048, 2048, 512  # 64 pair tiles on 64 clusters
+    A, W = _codes(g, (M, K)), _codes(g, (N, K))
+    sa = (torch.rand(M, generator=g) * 1e-2).cuda()
+    sw = (torch.rand(N, generator=g) * 1e-2).cuda()
+    b = torch.randn(N, generator=g).to(torch.bfloat16).cuda()
+    main = torch.cuda.current_stream()
+    ref = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    _gemm(lib, A, sa, W, sw, b, ref, main)
+    y = torch.empty_like(ref)
+    for _ in range(70):
+        y.fill_(0)
+        _gemm(lib, A, sa, W, sw, b, y, main)
+    torch.cuda.synchronize()
+    assert torch.equal(y, ref)
+    _gpu.check_device_error()
+    s = torch.cuda.Stream()
+    yg = torch.zeros_like(ref)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        _gemm(lib, A, sa, W, sw, b, yg, s)  # warm up on the capture stream
+        torch.cuda.synchronize()
+        with torch.cuda.graph(graph, stream=s):
+            _gemm(lib, A, sa, W, sw, b, yg, s)
+    for _ in range(5):
+        yg.fill_(0)
+        graph.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(yg, ref)
+    _gpu.check_device_error()
