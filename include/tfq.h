@@ -231,10 +231,10 @@ TFQ_API tfq_status tfq_mxfp8_linear(const void *A_q, const void *sf_a, const voi
  * of TFQ_NOALLOC_SCRATCH_BYTES bytes, and no call allocates (no cudaMalloc,
  * cudaFree or allocating library routine).
  *  - The caller still owns and passes every input and output.
- *  - A call needs 132 bytes of the array whatever M, N and K (the error
- *    word and, one 128-byte line further, a counter the kernel's clusters use
- *    to keep pace); a call needing more than the array holds is rejected with
- *    TFQ_EUNSUPPORTED.
+ *  - A call needs 136 bytes of the array whatever M, N and K (the error
+ *    word and, one 128-byte line further, two counters the kernel's clusters
+ *    use to keep pace, which the kernel leaves at zero); a call needing more
+ *    than the array holds is rejected with TFQ_EUNSUPPORTED.
  *  - The first call on a device does a one-time set-up with that device
  *    current (device checks, cudaGetSymbolAddress of the array, which may
  *    load the library's device code into the context); make that first call

@@ -33,7 +33,7 @@ static __device__ __align__(256) uint32_t g_noalloc_scratch[TFQ_NOALLOC_SCRATCH_
 
 // Scratch the GEMM needs per call: its error word (first 128-byte line) and
 // the round counter of its cluster pacing (second line).
-constexpr size_t kGemmScratchBytes = 128 + sizeof(unsigned);
+constexpr size_t kGemmScratchBytes = 128 + 2 * sizeof(unsigned);  // error word; pacing line: rounds, clusters done
 
 constexpr int kMaxDevices = 64;
 std::mutex g_noalloc_mutex;
