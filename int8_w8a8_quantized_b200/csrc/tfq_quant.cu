@@ -11,16 +11,16 @@
 // the symmetric INT8 formula of the TeleFuser page (section "Core ideas").
 // Rows are tokens (activations) or output channels (weights).
 //
-// Design (B200): no shared memory, no barriers, no waits.  Rows of
-// K <= 2048 go to a grouped kernel: a power-of-two group of lanes per row,
-// several rows per warp, each lane holding 1, 4 or 8 of the row's 16-byte
-// units, so that a warp keeps kilobytes in flight however short the row.
-// Longer rows: one warp per row, rows strided over a grid of two CTAs of
-// eight warps per SM.  Pass 1 loads
-// a whole segment of the row (16 x 16-byte loads per lane: 8 KiB per warp in
-// flight, a warp reads 512 contiguous bytes per load) and reduces |x| with
-// packed max.xorsign.abs.bf16x2 and shuffles.  Pass 2 quantizes: a row of
-// at most one segment (K <= 4096) is still in registers; a longer row is
+// Design (B200): rows of K <= 2048 go to a grouped kernel: a power-of-two
+// group of lanes per row, several rows per warp, each lane holding 1, 4 or 8
+// of the row's 16-byte units, so that a warp keeps kilobytes in flight
+// however short the row.  Longer rows: one warp per row, rows strided over a grid of two or three
+// CTAs of eight warps per SM (rows of 16384 <= K <= 32768 are staged in
+// shared memory instead, see below).  Pass 1 loads a whole segment of the
+// row (12, 16 or 20 16-byte loads per lane: 6-10 KiB per warp in flight, a
+// warp reads 512 contiguous bytes per load) and reduces |x| with packed
+// max.xorsign.abs.bf16x2 and shuffles.  Pass 2 quantizes: a row of at most
+// one segment is still in registers; a longer row is
 // read again, which hits L2 because pass 1 loaded it with an evict_last
 // cache policy (so HBM sees 2 bytes read and 1 written per element).  The
 // division is a branch-free correctly rounded one (a two-term reciprocal of
