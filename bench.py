@@ -787,6 +787,18 @@ def quantizer_cpu_baseline(x_cpu):
             "ms_per_pass": 1e3 * secs / n}
 
 
+def use_all_host_cores_for_oracle():
+    """The reference arm runs on rank 0 alone (the other ranks exit without
+    work), so the oracle gets every core this process may use, as in a plain
+    N = 1 run -- torchrun sets OMP_NUM_THREADS=1 for each rank otherwise."""
+    import oracle
+    try:
+        n = len(os.sched_getaffinity(0))
+    except AttributeError:
+        n = os.cpu_count() or 1
+    oracle.set_num_threads(max(1, n))
+
+
 # ------------------------------------------------------------------ main
 def quantizer_main(args, rank, world, local_rank):
     if args.impl == "reference":
@@ -794,6 +806,7 @@ def quantizer_main(args, rank, world, local_rank):
             return 0
         from int8_w8a8_quantized_b200 import workloads
         import oracle
+        use_all_host_cores_for_oracle()
         x = workloads.quantizer_input()
         cb = quantizer_cpu_baseline(x)
         line = {"metric": "activation quantizer GB/s (per-token FP8 qmax 448 + per-row INT8 127), algorithmic bytes",
@@ -840,6 +853,7 @@ def main():
     if args.impl == "reference":
         if rank != 0:
             return 0
+        use_all_host_cores_for_oracle()
         reference_arm(args, wl, cfg, world)
         return 0
 
