@@ -741,6 +741,9 @@ def quantizer_arm(args, rank, world, local_rank):
     t1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = t0.elapsed_time(t1) / args.e2e_steps
+    if world > 1:  # the slowest rank times the job
+        copy_ms = max_over_ranks(copy_ms, dev)
+        e2e_ms = max_over_ranks(e2e_ms, dev)
     if rank != 0:
         return
     line = {
@@ -865,6 +868,10 @@ def main():
                                 device_id=torch.device("cuda", local_rank))
     res, e2e = gpu_arm(args, wl, rank, world, local_rank)
     if world > 1:
+        if e2e is not None:  # every rank measured its own replica; the slowest one times the job
+            slowest = max_over_ranks(e2e["ms_per_step"], torch.device("cuda", local_rank))
+            e2e["value"] *= e2e["ms_per_step"] / slowest
+            e2e["ms_per_step"] = slowest
         dist.barrier()
         dist.destroy_process_group()
     if rank != 0:
