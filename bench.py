@@ -891,7 +891,7 @@ def main():
     pair = wl.M >= 512
     if args.dtype == "mxfp8":
         kname = "mxfp8_mm_pair_kernel" if pair else "mxfp8_mm_kernel"
-        qname = "quant_mxfp8_kernel"
+        qname = "quant_mxfp8_blocks_kernel"
     else:
         kname = ("scaled_mm_pair_kernel" if pair else "scaled_mm_kernel") + f"<{args.dtype}>"
         qname = "quant_rows_kernel<" + args.dtype + ">"
