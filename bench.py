@@ -291,11 +291,16 @@ def aggregate_throughput(world: int, flops_per_step: int, ms_per_step_max: float
 # ------------------------------------------------------------ GPU arm
 def act_qmaxes(wl, dtype):
     """Activation quantization passes per step: one per qmax; INT8 uses 127,
-    MXFP8 has no qmax (its scale comes from each block's exponent)."""
+    MXFP8 has no qmax (its scale comes from each block's exponent), and the
+    FP16-accumulator GEMM takes activations quantized with qmax 7 -- the DiT
+    setting the LightX2V page pairs with FP16 accumulation; at 448 (and at 14
+    on the FFN-out shape) its partial sums overflow FP16."""
     if dtype == "int8":
         return (127.0,)
     if dtype == "mxfp8":
         return (0.0,)
+    if dtype == "fp8_f16acc":
+        return (7.0,)
     return wl.act_qmax
 
 
@@ -431,6 +436,8 @@ def gpu_arm(args, wl, rank, world, local_rank):
         key = f"{m}x{n}x{k}"
         out["per_linear"].setdefault(key, []).append(a.elapsed_time(b))
 
+    # outputs of the last timed step that are not finite (an FP16 accumulator can overflow); outside the timing
+    out["nonfinite_outputs"] = int(sum(int((~torch.isfinite(y)).sum()) for y in ys.values()))
     out["context"] = torch_scaled_mm_context(args, wl, lins, aq, ys, qmaxes, stream) if not args.no_context else None
 
     # -------- end-to-end through the C ABI with host buffers
@@ -846,7 +853,7 @@ def main():
     wl = workloads.WORKLOADS[args.workload]
     cfg = {"workload": wl.name, "M": wl.M, "dtype": args.dtype,
            "linears": [f"{l.name}:{l.K}->{l.N}" for l in wl.linears],
-           "act_qmax": list(wl.act_qmax) if args.dtype != "mxfp8" else "none (E8M0 scale per 32 values)",
+           "act_qmax": list(act_qmaxes(wl, args.dtype)) if args.dtype != "mxfp8" else "none (E8M0 scale per 32 values)",
            "weight_qmax": 448.0 if args.dtype != "mxfp8" else "none (E8M0 scale per 32 values)",
            "bias": wl.has_bias,
            "l2": "inputs larger than L2 (126 MB)" if wl.M * min(l.K for l in wl.linears) * 2 > L2_BYTES
@@ -942,6 +949,7 @@ def main():
         "context": res.get("context"),
         "per_linear_ms": {k: round(statistics.median(v), 4) for k, v in res["per_linear"].items()},
         "gpu_launches": res["gpu_launches"],
+        "nonfinite_outputs": res["nonfinite_outputs"],
         "clocks": res["clocks"],
     }
     if e2e is not None:
