@@ -184,3 +184,11 @@ def test_float8_views_accepted():
         tfq_scaled_fp8_linear(A.view(torch.int8), sa, Wq, sw, b)
     with pytest.raises(ValueError):
         tfq_scaled_fp8_linear(A, sa.cpu(), Wq, sw, b)
+
+
+@pytest.mark.parametrize("M,N,K", [(100, 136, 65536), (600, 264, 65536), (2048, 1024, 32784)])
+def test_long_k_full_compare(M, N, K):
+    """Hundreds of K blocks per tile (512 at K = 65536): the stage ring's
+    phases wrap many times within one tile; K = 32784 leaves a 16-element
+    K tail; one-CTA and pair kernels; full compare."""
+    _run_case(M, N, K, True, seed=M + N + K)

@@ -180,3 +180,11 @@ def test_gemm_pair_several_tiles_per_cluster(M, N, K):
     accumulators are reused, so every tile's first MMA waits for the other
     buffer's shared columns to be read; full compare."""
     _gemm_case(M, N, K, True, seed=M + 7 * N + K)
+
+
+@pytest.mark.parametrize("M,N,K", [(130, 200, 32768), (700, 520, 16416)])
+def test_gemm_long_k(M, N, K):
+    """Hundreds of K blocks per tile (and 1024 scale blocks per row): the scale
+    atoms of late K steps, the stage ring wrapping many times; K = 16416 ends
+    in a partial scale atom; one-CTA and pair kernels."""
+    _gemm_case(M, N, K, True, seed=M + N + K)
