@@ -141,9 +141,11 @@ TFQ_API tfq_status tfq_quant_act_int8_per_token(const void *x_bf16, int64_t M, i
  *   fp32, bias bf16 [N] or NULL, out bf16 [M, N]:
  *   out[m,n] = bf16_rn(fp32(sum_k A_q[m,k] W_q[n,k]) * s_a[m] * s_w[n] + bias[n]),
  * the integer sum exact in s32 on the tensor cores (|sum| <= 128^2 K < 2^31
- * for K < 131072), converted to fp32 (round to nearest) in the epilogue.
- * Same preconditions, tolerance and errors as tfq_scaled_fp8_linear.
+ * for K < TFQ_INT8_MAX_K = 131072), converted to fp32 (round to nearest) in
+ * the epilogue.  Same preconditions, tolerance and errors as
+ * tfq_scaled_fp8_linear, and K >= TFQ_INT8_MAX_K returns TFQ_EUNSUPPORTED.
  */
+#define TFQ_INT8_MAX_K 131072
 TFQ_API tfq_status tfq_scaled_int8_linear(const void *A_q, const float *s_a, const void *W_q,
                                           const float *s_w, const void *bias_bf16, int64_t M, int64_t N,
                                           int64_t K, void *out_bf16, void *stream);

@@ -16,6 +16,7 @@ from ._capi import (  # noqa: F401
     TFQ_ETIMEOUT,
     TFQ_EUNSUPPORTED,
     TFQ_OK,
+    TFQ_INT8_MAX_K,
     TFQ_QUANT_MAX_K,
     TfqError,
     last_error_message,

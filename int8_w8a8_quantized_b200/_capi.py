@@ -25,6 +25,7 @@ LIB_PATH = os.path.join(PKG, "libtfq.so")
 TFQ_OK, TFQ_EINVAL, TFQ_EUNSUPPORTED, TFQ_ECUDA, TFQ_ETIMEOUT = range(5)
 TFQ_DTYPE_FP8_E4M3, TFQ_DTYPE_INT8 = 0, 1
 TFQ_QUANT_MAX_K = 1 << 24
+TFQ_INT8_MAX_K = 131072  # the INT8 GEMM takes K < this (its s32 sum stays exact)
 
 # name -> (restype, argtypes), in the order include/tfq.h declares them
 _P, _I64, _F, _I = ctypes.c_void_p, ctypes.c_int64, ctypes.c_float, ctypes.c_int

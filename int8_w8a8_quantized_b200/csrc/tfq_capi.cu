@@ -203,7 +203,11 @@ tfq_status tfq_scaled_int8_linear(const void* A_q, const float* s_a, const void*
                                   const void* bias_bf16, int64_t M, int64_t N, int64_t K, void* out_bf16,
                                   void* stream) {
     tfq_status st = check_gemm_args(A_q, s_a, W_q, s_w, bias_bf16, M, N, K, out_bf16);
-    if (st != TFQ_OK || M == 0 || N == 0) return st;
+    if (st != TFQ_OK) return st;
+    // |sum| <= 128^2 K must stay below 2^31 for the s32 accumulator to be exact
+    if (K >= TFQ_INT8_MAX_K) return fail(TFQ_EUNSUPPORTED, "K=%lld: the INT8 sum may exceed s32 (K < %d)",
+                                         (long long)K, TFQ_INT8_MAX_K);
+    if (M == 0 || N == 0) return st;
     DeviceState* ds = current_device_state(&st);
     if (ds == nullptr) return st;
     return launch_scaled_int8_gemm(A_q, s_a, W_q, s_w, bias_bf16, M, N, K, out_bf16,

@@ -37,6 +37,12 @@ def test_header_declarations_match_binding():
     assert set(names) == set(_capi.SIGNATURES)
 
 
+def test_header_limits_match_binding():
+    text = open(os.path.join(ROOT, "include", "tfq.h"), encoding="utf-8").read()
+    assert re.search(r"#define TFQ_INT8_MAX_K (\d+)", text).group(1) == str(_capi.TFQ_INT8_MAX_K)
+    assert re.search(r"#define TFQ_QUANT_MAX_K \(1 << (\d+)\)", text).group(1) == str(_capi.TFQ_QUANT_MAX_K.bit_length() - 1)
+
+
 def test_library_exports_every_declared_symbol(lib):
     out = subprocess.run(["nm", "-D", "--defined-only", _capi.LIB_PATH], capture_output=True, text=True,
                          check=True).stdout
@@ -93,6 +99,14 @@ def test_quant_weight_validation(lib):
 ])
 def test_gemm_validation(lib, M, N, K, status):
     assert lib.tfq_scaled_fp8_linear(ALIGNED, ALIGNED, ALIGNED, ALIGNED, None, M, N, K, ALIGNED, None) == status
+
+
+def test_int8_gemm_k_limit(lib):
+    """The INT8 GEMM's s32 sum is exact only for K < TFQ_INT8_MAX_K (128^2 K < 2^31)."""
+    f = lib.tfq_scaled_int8_linear
+    assert f(ALIGNED, ALIGNED, ALIGNED, ALIGNED, None, 4, 16, 131072, ALIGNED, None) == _capi.TFQ_EUNSUPPORTED
+    assert f(ALIGNED, ALIGNED, ALIGNED, ALIGNED, None, 0, 16, 131072, ALIGNED, None) == _capi.TFQ_EUNSUPPORTED
+    assert f(ALIGNED, ALIGNED, ALIGNED, ALIGNED, None, 0, 16, 131056, ALIGNED, None) == _capi.TFQ_OK  # empty
 
 
 def test_gemm_rejects_null_and_misaligned(lib):
