@@ -775,11 +775,11 @@ def quantizer_arm(args, rank, world, local_rank):
                 "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t in outs)},
     }
     if world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = quantizer_cpu_baseline(x.cpu())
+        line["cpu_baseline"] = quantizer_cpu_baseline(x.cpu(), args.cpu_seconds)
     print(json.dumps(line), flush=True)
 
 
-def quantizer_cpu_baseline(x_cpu):
+def quantizer_cpu_baseline(x_cpu, seconds: float = 10.0):
     import numpy as np
     import torch
     import oracle
@@ -787,7 +787,7 @@ def quantizer_cpu_baseline(x_cpu):
     M, K = bits.shape
     t0 = time.perf_counter()
     n = 0
-    while time.perf_counter() - t0 < 10.0 or n == 0:
+    while time.perf_counter() - t0 < seconds or n == 0:
         oracle.quant_rows_fp8(bits, 448.0)
         oracle.quant_rows_int8(bits, 127.0)
         n += 1
@@ -818,7 +818,7 @@ def quantizer_main(args, rank, world, local_rank):
         import oracle
         use_all_host_cores_for_oracle()
         x = workloads.quantizer_input()
-        cb = quantizer_cpu_baseline(x)
+        cb = quantizer_cpu_baseline(x, args.cpu_seconds)
         line = {"metric": "activation quantizer GB/s (per-token FP8 qmax 448 + per-row INT8 127), algorithmic bytes",
                 "impl": "reference", "value": cb["value"], "unit": "GB/s", "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": cb["ms_per_pass"], "higher_is_better": True, "scaling": "weak",

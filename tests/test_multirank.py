@@ -51,3 +51,29 @@ def test_max_over_ranks_and_weak_scaling(world):
 
 def test_single_rank_throughput():
     assert bench.aggregate_throughput(1, 2 * 10 ** 12, 1000.0) == pytest.approx(2.0)
+
+
+def test_bench_reference_arm_under_torchrun():
+    """`bench.py --impl reference` launched like the multi-GPU bench (torchrun,
+    two ranks, rendezvous on 127.0.0.1): rank 0 alone runs the oracle and
+    prints one JSON line with the contract's keys; the other rank exits 0
+    without work.  Runs on the CPU (the reference arm needs no GPU)."""
+    import json
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
+           "--master-addr", "127.0.0.1", "--master-port", str(29600 + os.getpid() % 300),
+           os.path.join(root, "bench.py"), "--impl", "reference", "--gpus", "2", "--workload",
+           "activation_quantizer", "--steps", "1", "--warmup", "1", "--cpu-seconds", "0.5"]
+    r = subprocess.run(cmd, capture_output=True, text=True, timeout=300, cwd=root)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1, r.stdout[-2000:]
+    line = json.loads(lines[0])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "impl", "cpu_baseline", "e2e"):
+        assert key in line, key
+    assert line["impl"] == "reference" and line["n_gpus"] == 2 and line["value"] > 0
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
