@@ -39,8 +39,11 @@
  *    element quotient x / s is an fp32 IEEE division, the FP8 cast rounds
  *    to nearest even and saturates, the INT8 rounding is half-to-even.
  *  - Thread safety: calls may come from several host threads; the library
- *    keeps per-device state (launch attributes, the error word, a small
- *    TMA-descriptor cache) behind a mutex.
+ *    keeps per-device state (launch attributes, the error word, the GEMM's
+ *    ring of cluster-pacing counters) behind a mutex.  TMA descriptors are
+ *    encoded on the host for every call and passed as kernel parameters.
+ *  - Non-finite inputs (inf, NaN) are outside the contract: the codes and
+ *    scales of a row holding one are unspecified.
  */
 #ifndef TFQ_H_
 #define TFQ_H_
