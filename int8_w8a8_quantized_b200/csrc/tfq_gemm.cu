@@ -34,7 +34,8 @@
 // sweeping every M tile, so that the CTAs running at the same time share the
 // band's weight panels (kept in L2) and each activation panel; the pair
 // kernel also keeps its clusters within one tile of each other (pacing,
-// see tfq_gemm_common.cuh).  M and N tails are handled by
+// see tfq_gemm_common.cuh) and runs a last round of at most half as many
+// tiles as clusters as half-width (256 x 128) tiles.  M and N tails are handled by
 // TMA (zero fill on load, clipping on store); K tails by zero fill.
 // Every wait is bounded (see tfq_ptx.cuh); a CTA that gives up records it in
 // the error word, drains its own outstanding copies and MMAs, frees TMEM and

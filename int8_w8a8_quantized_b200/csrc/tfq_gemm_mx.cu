@@ -284,8 +284,8 @@ __global__ void __launch_bounds__(THREADS, 1)
 }
 
 // ---------------------------------------------------------------------------
-// MXFP8 CTA-pair kernel: a cluster of two CTAs computes a 256 x 192 tile with
-// tcgen05.mma.cta_group::2.kind::mxf8f6f4.block_scale (M = 256, N = 192).  As
+// MXFP8 CTA-pair kernel: a cluster of two CTAs computes a 256 x 256 tile with
+// tcgen05.mma.cta_group::2.kind::mxf8f6f4.block_scale (M = 256, N = 256).  As
 // in scaled_mm_pair_kernel, CTA r loads rows [128 r, 128 r + 128) of the A
 // panel and rows [128 r, 128 r + 128) of the B panel; in addition each CTA
 // loads the scale atom of its own 128 A rows and the two atoms of the tile's
