@@ -364,16 +364,23 @@ def gpu_arm(args, wl, rank, world, local_rank):
         if st != 0:
             raise RuntimeError(f"{what}: {_capi.status_string(st)}: {_capi.last_error_message()}")
 
-    def step(record):
+    n_kernels = len(qmaxes) * (len(xs) + len(lins))
+
+    def step(record, which=None):
+        """One block step; with `record`, CUDA events bracket kernel `which` of
+        the step (every kernel when which is None)."""
+        k = -1
         for q in qmaxes:
             for name, x in xs.items():
                 A, sa = aq[(name, q)]
-                if record:
+                k += 1
+                rec = record and (which is None or k == which)
+                if rec:
                     e0 = torch.cuda.Event(enable_timing=True); e0.record(stream)
                 check(quant_fn(x.data_ptr(), x.shape[0], x.shape[1], float(q), A.data_ptr(), sa.data_ptr(), sh),
                       "quant")
                 launches[0] += 1
-                if record:
+                if rec:
                     e1 = torch.cuda.Event(enable_timing=True); e1.record(stream)
                     # algorithmic bytes: read bf16, write 8-bit codes, 4 B of scale per row
                     # (MXFP8: 1 B of scale per 32 values)
@@ -381,12 +388,14 @@ def gpu_arm(args, wl, rank, world, local_rank):
             for lin, Wq, sw, b in lins:
                 A, sa = aq[(lin.x, q)]
                 y = ys[(lin.name, q)]
-                if record:
+                k += 1
+                rec = record and (which is None or k == which)
+                if rec:
                     e0 = torch.cuda.Event(enable_timing=True); e0.record(stream)
                 check(gemm_fn(A.data_ptr(), sa.data_ptr(), Wq.data_ptr(), sw.data_ptr(),
                               None if b is None else b.data_ptr(), wl.M, lin.N, lin.K, y.data_ptr(), sh), "gemm")
                 launches[0] += 1
-                if record:
+                if rec:
                     e1 = torch.cuda.Event(enable_timing=True); e1.record(stream)
                     ev["gemm"].append((e0, e1, (wl.M, lin.N, lin.K)))
 
@@ -404,8 +413,13 @@ def gpu_arm(args, wl, rank, world, local_rank):
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
     t0.record(stream)
-    for _ in range(args.steps):
-        step(True)
+    # Per-kernel events: step i brackets kernel i mod n_kernels only, so that every kernel is timed
+    # in steps / n_kernels of the steps and the other kernel boundaries run as they would without a
+    # profiler (an event between two kernels serialises their launches).  Fewer steps than kernels:
+    # events around every kernel of every step.
+    sample_one = args.steps >= n_kernels
+    for i in range(args.steps):
+        step(True, (i % n_kernels) if sample_one else None)
     t1.record(stream)
     torch.cuda.synchronize()
     clk = clocks.stop()
@@ -415,6 +429,9 @@ def gpu_arm(args, wl, rank, world, local_rank):
     ms = max_over_ranks(t0.elapsed_time(t1), dev) if world > 1 else t0.elapsed_time(t1)
     ms_per_step = ms / args.steps
 
+    # one step's kernels (for the path floor), independent of which launches had events
+    step_shapes = [(wl.M, lin.N, lin.K) for q in qmaxes for lin, _, _, _ in lins]
+    step_quant_bytes = [3 * x.numel() + (x.numel() // 32 if mx else 4 * x.shape[0]) for q in qmaxes for x in xs.values()]
     gemm_ms = [a.elapsed_time(b) for a, b, _ in ev["gemm"]]
     quant_ms = [a.elapsed_time(b) for a, b, _ in ev["quant"]]
     gemm_flops = [2 * m * n * k for _, _, (m, n, k) in ev["gemm"]]
@@ -423,12 +440,20 @@ def gpu_arm(args, wl, rank, world, local_rank):
     else:
         gemm_bytes = [m * k + n * k + 2 * m * n + 4 * m + 6 * n for _, _, (m, n, k) in ev["gemm"]]
     quant_bytes = [nbytes for _, _, nbytes in ev["quant"]]
+    def gemm_step_bytes(m, n, k):
+        return m * k + n * k + ((m + n) * k // 32 + 2 * m * n + 2 * n if mx else 2 * m * n + 4 * m + 6 * n)
     out = {
         "ms_per_step": ms_per_step,
-        "gemm_flops_each": gemm_flops, "gemm_bytes_each": gemm_bytes,
+        "step_gemm_flops": [2 * m * n * k for m, n, k in step_shapes],
+        "step_gemm_bytes": [gemm_step_bytes(m, n, k) for m, n, k in step_shapes],
+        "step_quant_bytes": step_quant_bytes,
         "gemm_ms_total": sum(gemm_ms), "gemm_flops_total": sum(gemm_flops), "gemm_bytes_total": sum(gemm_bytes),
         "quant_ms_total": sum(quant_ms), "quant_bytes_total": sum(quant_bytes),
         "gemm_launches": len(gemm_ms), "quant_launches": len(quant_ms),
+        "quant_launches_per_step": len(qmaxes) * len(xs),
+        "kernel_events": (f"each kernel bracketed in {args.steps // n_kernels}-{-(-args.steps // n_kernels)} of "
+                          f"the {args.steps} timed steps (one kernel per step)") if sample_one
+        else "every kernel of every timed step",
         "gpu_launches": launches[0], "clocks": clk,
         "per_linear": {},
     }
@@ -640,12 +665,12 @@ def path_roofline(res, steps, peaks, fp8_peak):
     measured step time; with the measured sustained 8-bit peak and with the
     4.5 PFLOP/s spec."""
     hbm = peaks.get("hbm_gbs", FALLBACK_HBM_GBS) * 1e9
-    q_s = res["quant_bytes_total"] / hbm
-    per_launch = [(f, b) for f, b in zip(res["gemm_flops_each"], res["gemm_bytes_each"])]
+    q_s = sum(res["step_quant_bytes"]) / hbm
+    per_launch = list(zip(res["step_gemm_flops"], res["step_gemm_bytes"]))
 
     def floor_ms(peak_tflops):
         g_s = sum(max(f / (peak_tflops * 1e12), b / hbm) for f, b in per_launch)
-        return 1e3 * (q_s + g_s) / steps
+        return 1e3 * (q_s + g_s)
 
     measured = res["ms_per_step"]
     f_meas, f_spec = floor_ms(fp8_peak), floor_ms(FP8_SPEC_TFLOPS)
@@ -941,7 +966,8 @@ def main():
             "unit": "GB/s",
             "frac": None if quant_gbs is None else round(quant_gbs / peaks.get("hbm_gbs", FALLBACK_HBM_GBS), 4),
             "frac_of_nominal_8tbs": None if quant_gbs is None else round(quant_gbs / 8000.0, 4),
-            "share_of_step": round(res["quant_ms_total"] / (res["ms_per_step"] * args.steps), 4),
+            "share_of_step": round(res["quant_ms_total"] / max(1, res["quant_launches"]) *
+                                   res["quant_launches_per_step"] / res["ms_per_step"], 4),
             "traffic": recorded_traffic("quant", wl.name, args.dtype),
             "algorithmic_bytes_per_launch": round(res["quant_bytes_total"] / max(1, res["quant_launches"])),
         },
@@ -949,6 +975,7 @@ def main():
         "context": res.get("context"),
         "per_linear_ms": {k: round(statistics.median(v), 4) for k, v in res["per_linear"].items()},
         "gpu_launches": res["gpu_launches"],
+        "kernel_events": res["kernel_events"],
         "nonfinite_outputs": res["nonfinite_outputs"],
         "clocks": res["clocks"],
     }

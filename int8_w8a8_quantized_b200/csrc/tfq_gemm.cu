@@ -90,6 +90,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    pdl_allow_next();
+    pdl_wait();  // the set-up above may overlap the previous kernel; global memory only from here
 
     if (warp == 0) {
         // ---------------------------------------------------- TMA producer
@@ -285,6 +287,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     cluster_sync_all();  // barriers of both CTAs initialised, TMEM allocated
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    pdl_allow_next();
+    pdl_wait();  // the set-up above may overlap the previous kernel; global memory only from here
 
     if (warp == 0) {
         // ---------------------------------------------------- TMA producer
@@ -487,15 +491,18 @@ tfq_status launch_scaled_mm(const void* A, const float* s_a, const void* W, cons
         const int clusters = static_cast<int>(std::min<int64_t>(pair_tiles, ds->sm_count / 2));
         a.tail_halves = choose_tail_halves(pair_tiles, clusters);
         a.round_ctr = take_round_counter(ds);
-        scaled_mm_pair_kernel<256, kAcc><<<2 * clusters, THREADS, PairCfg<256>::kSmem, stream>>>(tmA, tmBh, tmBq,
-                                                                                              tmY, a);
+        const cudaError_t el = launch_kernel(scaled_mm_pair_kernel<256, kAcc>, dim3(2 * clusters), dim3(THREADS),
+                                             PairCfg<256>::kSmem, stream, tmA, tmBh, tmBq, tmY, a);
+        if (el != cudaSuccess) return fail(TFQ_ECUDA, "GEMM launch: %s", cudaGetErrorString(el));
     } else {
         CUtensorMap tmB;
         st = encode_tensor_map_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, W, K, N, K, BK, BN,
                                   CU_TENSOR_MAP_SWIZZLE_128B);
         if (st != TFQ_OK) return st;
         const int grid = static_cast<int>(std::min<int64_t>(tiles, ds->sm_count));
-        scaled_mm_kernel<kAcc><<<grid, THREADS, SMEM_BYTES, stream>>>(tmA, tmB, tmY, a);
+        const cudaError_t el = launch_kernel(scaled_mm_kernel<kAcc>, dim3(grid), dim3(THREADS), SMEM_BYTES, stream,
+                                             tmA, tmB, tmY, a);
+        if (el != cudaSuccess) return fail(TFQ_ECUDA, "GEMM launch: %s", cudaGetErrorString(el));
     }
     const cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? TFQ_OK : fail(TFQ_ECUDA, "GEMM launch: %s", cudaGetErrorString(e));

@@ -157,6 +157,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    pdl_allow_next();
+    pdl_wait();  // the set-up above may overlap the previous kernel; global memory only from here
 
     if (warp == 0) {
         // ---------------------------------------------------- TMA producer
@@ -372,6 +374,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     cluster_sync_all();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    pdl_allow_next();
+    pdl_wait();  // the set-up above may overlap the previous kernel; global memory only from here
 
     if (warp == 0) {
         // ---------------------------------------------------- TMA producer
@@ -599,10 +603,14 @@ tfq_status launch_mxfp8_mm(const void* A, const uint8_t* sf_a, const void* W, co
         const int64_t pair_tiles = ((M + 255) / 256) * static_cast<int64_t>(a.n_tiles);
         const int clusters = static_cast<int>(std::min<int64_t>(pair_tiles, ds->sm_count / 2));
         a.round_ctr = take_round_counter(ds);
-        mxfp8_mm_pair_kernel<<<2 * clusters, THREADS, MXP_SMEM_BYTES, stream>>>(tmA, tmBh, tmY, tmSA, tmSB, a, mx);
+        const cudaError_t el = launch_kernel(mxfp8_mm_pair_kernel, dim3(2 * clusters), dim3(THREADS), MXP_SMEM_BYTES,
+                                             stream, tmA, tmBh, tmY, tmSA, tmSB, a, mx);
+        if (el != cudaSuccess) return fail(TFQ_ECUDA, "GEMM launch: %s", cudaGetErrorString(el));
     } else {
         const int grid = static_cast<int>(std::min<int64_t>(tiles, ds->sm_count));
-        mxfp8_mm_kernel<<<grid, THREADS, MX_SMEM_BYTES, stream>>>(tmA, tmB, tmY, a, mx);
+        const cudaError_t el = launch_kernel(mxfp8_mm_kernel, dim3(grid), dim3(THREADS), MX_SMEM_BYTES, stream, tmA,
+                                             tmB, tmY, a, mx);
+        if (el != cudaSuccess) return fail(TFQ_ECUDA, "GEMM launch: %s", cudaGetErrorString(el));
     }
     const cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? TFQ_OK : fail(TFQ_ECUDA, "GEMM launch: %s", cudaGetErrorString(e));

@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <utility>
 
 #include "tfq.h"
 
@@ -37,6 +38,29 @@ struct DeviceState {
     bool gemm_attr_set[5] = {false, false, false, false, false};  // FP8, INT8, FP8/FP16 acc, MXFP8, MXFP8 pair
     bool quant_attr_set = false;   // dynamic shared memory limit of the staged-row quantizers
 };
+
+#ifndef TFQ_PDL
+#define TFQ_PDL 1  // launch the hot-path kernels with programmatic stream serialization
+#endif
+
+// Launches `kernel` on `stream`; with TFQ_PDL the launch may overlap the
+// tail of the stream's previous kernel (the kernel calls pdl_wait() before
+// touching global memory).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_kernel(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                          Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = TFQ_PDL;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 // Per-device state of the current device, created on first use.  Returns
 // nullptr and sets *st on failure.

@@ -109,6 +109,16 @@ __device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, v
     return __all_sync(0xFFFFFFFFu, ok) != 0;
 }
 
+// ------------------------------------------------- programmatic dependent launch
+// A kernel launched with programmatic stream serialization may start while
+// the previous kernel of its stream is still running.  pdl_wait() blocks
+// until that kernel has completed and its memory is visible (it returns at
+// once when there is no such kernel), so every read of an input and every
+// write of an output must follow it; pdl_allow_next() lets the next kernel of
+// the stream start its own launch and set-up as this one's CTAs drain.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_allow_next() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ------------------------------------------------------- bulk / TMA copies
 // 1-D bulk copy global -> shared, completion counted on `bar` in bytes.
 // Both addresses 16-byte aligned, bytes a multiple of 16.

@@ -248,6 +248,8 @@ __global__ void __launch_bounds__(256, rows_ctas_per_sm<SEG>()) quant_rows_kerne
                                                                                  int64_t M, int K, float qmax,
                                                                                  uint8_t* __restrict__ q,
                                                                                  float* __restrict__ s) {
+    pdl_allow_next();
+    pdl_wait();
     const int lane = threadIdx.x & 31;
     const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
     const int units = K >> 3;  // 16-byte units of 8 bf16 per row
@@ -324,6 +326,8 @@ __global__ void __launch_bounds__(kStagedThreads) quant_rows_staged_kernel(const
                                                                            int K, int slots, float qmax,
                                                                            uint8_t* __restrict__ q,
                                                                            float* __restrict__ s, uint32_t* err) {
+    pdl_allow_next();
+    pdl_wait();
     extern __shared__ __align__(128) uint8_t staged_smem[];
     __shared__ uint64_t bar[kStagedMaxSlots];
     __shared__ float wmax[kStagedThreads / 32];
@@ -432,6 +436,8 @@ template <bool kInt8, bool kClamp, int LPR, int J>
 __global__ void __launch_bounds__(256, grouped_ctas_per_sm<J>()) quant_grouped_rows_kernel(const uint4* __restrict__ x, int64_t M, int K,
                                                                  float qmax, uint8_t* __restrict__ q,
                                                                  float* __restrict__ s) {
+    pdl_allow_next();
+    pdl_wait();
     constexpr int RPW = 32 / LPR;  // rows per warp
     const int lane = threadIdx.x & 31;
     const int sub = lane % LPR;
@@ -511,8 +517,9 @@ void launch_grouped_lpr(const void* x, int64_t rows, int64_t K, float qmax, bool
     auto kernel = out_int8 ? quant_grouped_rows_kernel<true, false, LPR, J>
                            : (clamp ? quant_grouped_rows_kernel<false, true, LPR, J>
                                     : quant_grouped_rows_kernel<false, false, LPR, J>);
-    kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(static_cast<const uint4*>(x), rows, static_cast<int>(K),
-                                                               qmax, static_cast<uint8_t*>(q), s);
+    // a launch error is also the runtime's last error, which the caller reads
+    (void)launch_kernel(kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, stream, static_cast<const uint4*>(x),
+                        rows, static_cast<int>(K), qmax, static_cast<uint8_t*>(q), s);
 }
 
 template <int J>
@@ -606,10 +613,9 @@ tfq_status launch_staged_rows(const void* x, int64_t rows, int64_t K, float qmax
     const cudaError_t eo = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kStagedThreads, smem);
     if (eo != cudaSuccess || per_sm < 1) return fail(TFQ_ECUDA, "staged quantizer occupancy: %s", cudaGetErrorString(eo));
     const int64_t blocks = std::min<int64_t>(rows, static_cast<int64_t>(ds->sm_count) * per_sm);
-    kernel<<<static_cast<unsigned>(blocks), kStagedThreads, smem, stream>>>(
-        static_cast<const uint4*>(x), rows, static_cast<int>(K), slots, qmax, static_cast<uint8_t*>(q), s,
-        ds->err_word);
-    const cudaError_t e = cudaGetLastError();
+    const cudaError_t e = launch_kernel(kernel, dim3(static_cast<unsigned>(blocks)), dim3(kStagedThreads), smem,
+                                        stream, static_cast<const uint4*>(x), rows, static_cast<int>(K), slots, qmax,
+                                        static_cast<uint8_t*>(q), s, ds->err_word);
     return e == cudaSuccess ? TFQ_OK : fail(TFQ_ECUDA, "quantizer launch: %s", cudaGetErrorString(e));
 }
 
@@ -654,10 +660,9 @@ tfq_status launch_quant_rows(const void* x, int64_t rows, int64_t K, float qmax,
     const int ctas_per_sm = short_seg ? rows_ctas_per_sm<kShort>()
                                       : (wide ? rows_ctas_per_sm<kWide>() : rows_ctas_per_sm<kLong>());
     const int64_t blocks = std::min<int64_t>((rows + 7) / 8, static_cast<int64_t>(ds->sm_count) * ctas_per_sm);
-    kernel<<<static_cast<unsigned>(blocks), threads, 0, stream>>>(static_cast<const uint4*>(x), rows,
-                                                                 static_cast<int>(K), qmax,
-                                                                 static_cast<uint8_t*>(q), s);
-    const cudaError_t e = cudaGetLastError();
+    const cudaError_t e = launch_kernel(kernel, dim3(static_cast<unsigned>(blocks)), dim3(threads), 0, stream,
+                                        static_cast<const uint4*>(x), rows, static_cast<int>(K), qmax,
+                                        static_cast<uint8_t*>(q), s);
     return e == cudaSuccess ? TFQ_OK : fail(TFQ_ECUDA, "quantizer launch: %s", cudaGetErrorString(e));
 }
 

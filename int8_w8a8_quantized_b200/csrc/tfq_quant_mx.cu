@@ -7,6 +7,7 @@
 #include <algorithm>
 
 #include "tfq_internal.h"
+#include "tfq_ptx.cuh"
 #include "tfq_quant_common.cuh"
 
 namespace tfq {
@@ -106,6 +107,8 @@ __global__ void __launch_bounds__(256, TFQ_MX_CTAS) quant_mxfp8_blocks_kernel(co
                                                                                     int64_t rows, int nb,
                                                                                     uint8_t* __restrict__ q,
                                                                                     uint8_t* __restrict__ sf) {
+    pdl_allow_next();
+    pdl_wait();
     const int64_t ra = (rows + 127) >> 7;
     const int ka4 = ((nb + 3) >> 2) << 2;
     const int64_t total = rows * nb;
@@ -152,10 +155,9 @@ tfq_status launch_quant_mxfp8(const void* x, int64_t rows, int64_t K, void* q, v
     // enough threads to take every block in one step of two, at most TFQ_MX_CTAS CTAs per SM
     const int64_t nblocks = rows * (K / 32);
     const int64_t grid = std::min<int64_t>((nblocks + 511) / 512, static_cast<int64_t>(ds->sm_count) * TFQ_MX_CTAS);
-    quant_mxfp8_blocks_kernel<<<static_cast<unsigned>(std::max<int64_t>(grid, 1)), 256, 0, stream>>>(
-        static_cast<const uint4*>(x), rows, static_cast<int>(K / 32), static_cast<uint8_t*>(q),
-        static_cast<uint8_t*>(sf));
-    const cudaError_t e = cudaGetLastError();
+    const cudaError_t e = launch_kernel(quant_mxfp8_blocks_kernel, dim3(static_cast<unsigned>(std::max<int64_t>(grid, 1))),
+                                        dim3(256), 0, stream, static_cast<const uint4*>(x), rows,
+                                        static_cast<int>(K / 32), static_cast<uint8_t*>(q), static_cast<uint8_t*>(sf));
     return e == cudaSuccess ? TFQ_OK : fail(TFQ_ECUDA, "quantizer launch: %s", cudaGetErrorString(e));
 }
 
