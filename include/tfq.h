@@ -26,6 +26,10 @@
  *  - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
  *    stream of the current device).  Work is enqueued asynchronously on it
  *    on the CURRENT device; the call returns once the launch is enqueued.
+ *    Kernels are launched with programmatic stream serialization: a kernel
+ *    may be scheduled and set itself up while the stream's previous kernel
+ *    finishes, but reads and writes memory only after that kernel has
+ *    completed, so stream order is kept.
  *  - Return value: TFQ_OK, or an error detected before any launch
  *    (TFQ_EINVAL for bad arguments, TFQ_EUNSUPPORTED for a device that is
  *    not sm_100 or a size beyond a stated limit), or TFQ_ECUDA when the CUDA
