@@ -78,14 +78,14 @@ def parse_args():
 _CSRC = "int8_w8a8_quantized_b200/csrc/"
 # Sources of the kernels a traffic record was captured on, per dtype and kind.
 KERNEL_SOURCES = {
-    ("fp8", "gemm"): ("tfq_gemm.cu", "tfq_gemm_common.cuh", "tfq_ptx.cuh"),
-    ("fp8", "quant"): ("tfq_quant.cu", "tfq_quant_common.cuh", "tfq_ptx.cuh"),
-    ("int8", "gemm"): ("tfq_gemm.cu", "tfq_gemm_common.cuh", "tfq_ptx.cuh"),
-    ("int8", "quant"): ("tfq_quant.cu", "tfq_quant_common.cuh", "tfq_ptx.cuh"),
-    ("fp8_f16acc", "gemm"): ("tfq_gemm.cu", "tfq_gemm_common.cuh", "tfq_ptx.cuh"),
-    ("fp8_f16acc", "quant"): ("tfq_quant.cu", "tfq_quant_common.cuh", "tfq_ptx.cuh"),
-    ("mxfp8", "gemm"): ("tfq_gemm_mx.cu", "tfq_gemm_common.cuh", "tfq_ptx.cuh"),
-    ("mxfp8", "quant"): ("tfq_quant_mx.cu", "tfq_quant_common.cuh"),
+    ("fp8", "gemm"): ("tfq_gemm.cu", "tfq_gemm_common.cuh", "tfq_ptx.cuh", "tfq_internal.h"),
+    ("fp8", "quant"): ("tfq_quant.cu", "tfq_quant_common.cuh", "tfq_ptx.cuh", "tfq_internal.h"),
+    ("int8", "gemm"): ("tfq_gemm.cu", "tfq_gemm_common.cuh", "tfq_ptx.cuh", "tfq_internal.h"),
+    ("int8", "quant"): ("tfq_quant.cu", "tfq_quant_common.cuh", "tfq_ptx.cuh", "tfq_internal.h"),
+    ("fp8_f16acc", "gemm"): ("tfq_gemm.cu", "tfq_gemm_common.cuh", "tfq_ptx.cuh", "tfq_internal.h"),
+    ("fp8_f16acc", "quant"): ("tfq_quant.cu", "tfq_quant_common.cuh", "tfq_ptx.cuh", "tfq_internal.h"),
+    ("mxfp8", "gemm"): ("tfq_gemm_mx.cu", "tfq_gemm_common.cuh", "tfq_ptx.cuh", "tfq_internal.h"),
+    ("mxfp8", "quant"): ("tfq_quant_mx.cu", "tfq_quant_common.cuh", "tfq_ptx.cuh", "tfq_internal.h"),
 }
 
 
