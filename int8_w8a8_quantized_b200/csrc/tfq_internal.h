@@ -108,9 +108,12 @@ tfq_status launch_scaled_fp8_gemm_f16acc(const void* A, const float* s_a, const 
                                          const void* bias, int64_t M, int64_t N, int64_t K, void* out,
                                          cudaStream_t stream, DeviceState* ds);
 
-// Scaled INT8 GEMM (S8 x S8 -> S32 on the tensor cores) with the same epilogue.
+// MXFP8 GEMM (E4M3 x E4M3 with one E8M0 scale per 32 values of K on both
+// operands, block-scaled on the tensor cores) with the bias/BF16 epilogue.
 tfq_status launch_mxfp8_gemm(const void* A, const uint8_t* sf_a, const void* W, const uint8_t* sf_w, const void* bias,
                              int64_t M, int64_t N, int64_t K, void* out, cudaStream_t stream, DeviceState* ds);
+
+// Scaled INT8 GEMM (S8 x S8 -> S32 on the tensor cores) with the same epilogue.
 tfq_status launch_scaled_int8_gemm(const void* A, const float* s_a, const void* W, const float* s_w,
                                    const void* bias, int64_t M, int64_t N, int64_t K, void* out,
                                    cudaStream_t stream, DeviceState* ds);
