@@ -67,7 +67,11 @@ def _load():
     global _lib
     with _lock:
         if _lib is None:
-            lib = ctypes.CDLL(build())
+            # TFQ_ORACLE_LIB names another build of tfq_oracle.c to load
+            # instead (the mutation test runs the pins against copies of the
+            # source with a planted mistake this way).
+            override = os.environ.get("TFQ_ORACLE_LIB")
+            lib = ctypes.CDLL(override if override else build())
             P = ctypes.c_void_p
             I64 = ctypes.c_int64
             lib.tfq_oracle_e4m3_decode.restype = ctypes.c_double

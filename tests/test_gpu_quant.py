@@ -1,12 +1,17 @@
 """GPU parity of the row quantizers against the oracle: codes and scales
 bit-exact, on the workloads' shapes and distributions, ragged sizes and the
 degenerate cases (zero rows, K = 0, M = 0, tiny magnitudes, rounding ties)."""
+import os
+
 import numpy as np
 import pytest
 import torch
 
 from int8_w8a8_quantized_b200 import _capi, workloads
 from tests import _gpu
+from tests._pins import load_hand_rows
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "hand_rows.txt")
 
 pytestmark = pytest.mark.gpu
 
@@ -93,6 +98,31 @@ def test_rounding_edges():
     x = x.to(torch.bfloat16).cuda()
     for qmax in (448.0, 14.0, 7.0, 21.0, 100.0):
         _assert_fp8_equal(x, qmax)
+
+
+@pytest.mark.parametrize("K", [16, 5120, 16384])
+def test_hand_rows(K):
+    """The hand-worked rows of tests/golden/hand_rows.txt (codes derived by
+    hand from the formulas and the E4M3FN format), zero-padded to K: the
+    padding changes neither the row maximum nor the codes of the given
+    values.  K picks the grouped, warp-per-row and staged kernels."""
+    for kind, qmax, xs, codes in load_hand_rows(GOLDEN):
+        n = len(xs)
+        x = torch.zeros(1, K, dtype=torch.float64)
+        x[0, :n] = torch.tensor(xs, dtype=torch.float64)
+        xb = x.to(torch.bfloat16)
+        assert torch.equal(xb[0, :n].double(), x[0, :n]), "hand rows are exact bf16 numbers"
+        xd = xb.cuda()
+        if kind == "fp8":
+            q, s = _gpu.quant_act_fp8(xd, qmax)
+            got = [int(c) for c in q[0, :n].cpu()]
+        else:
+            q, s = _gpu.quant_weight(xd, _capi.TFQ_DTYPE_INT8, qmax)
+            got = [int(c) for c in q[0, :n].cpu().view(torch.int8)]
+        assert got == codes, (kind, qmax, xs)
+        assert torch.all(q[0, n:] == 0)
+        amax = max(abs(v) for v in xs)
+        assert s.cpu().numpy()[0] == np.float32(max(amax, 1e-12)) / np.float32(qmax)
 
 
 @pytest.mark.parametrize("K", [256, 5120, 16384])
