@@ -155,8 +155,6 @@ class ClockSampler:
     QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
-    REASON_BITS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
-                   "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80}
 
     def __init__(self, gpu_index: int):
         self.gpu = gpu_index
@@ -225,14 +223,7 @@ class ClockSampler:
                 limit_w = pynvml.nvmlDeviceGetEnforcedPowerLimit(h) / 1000.0
             except Exception:
                 limit_w = None
-            if not self.samples:
-                return None
-            reasons = sorted(n for n, bit in self.REASON_BITS.items() if any(r & bit for _, _, r in self.samples))
-            return {"sm_mhz": statistics.median(c for c, _, _ in self.samples), "sm_max_mhz": sm_max,
-                    "power_w_max": max(p for _, p, _ in self.samples),
-                    "power_w_median": statistics.median(p for _, p, _ in self.samples),
-                    "power_limit_w": limit_w, "samples": len(self.samples),
-                    "source": "nvml, 10 ms", "reasons": reasons}
+            return summarize_nvml_samples(self.samples, sm_max, limit_w)
         if self.proc is None:
             return None
         self.proc.terminate()
@@ -241,34 +232,58 @@ class ClockSampler:
         except subprocess.TimeoutExpired:
             self.proc.kill()
         self.fh.close()
-        rows = []
         with open(self.path) as fh:
-            for line in fh:
-                parts = [p.strip() for p in line.split(",")]
-                if len(parts) >= 9:
-                    rows.append(parts)
+            lines = fh.readlines()
         os.unlink(self.path)
-        if not rows:
+        return summarize_smi_lines(lines)
+
+
+# NVML clock-event reason bits (nvmlClocksEventReason*) reported by name.
+CLOCK_REASON_BITS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
+                     "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80}
+
+
+def summarize_nvml_samples(samples, sm_max, limit_w):
+    """Clock record from NVML samples (SM MHz, board watts, reason bit mask):
+    median SM clock and power, the peak power, and every reason that was
+    active in any sample.  None without samples."""
+    if not samples:
+        return None
+    reasons = sorted(n for n, bit in CLOCK_REASON_BITS.items() if any(r & bit for _, _, r in samples))
+    return {"sm_mhz": statistics.median(c for c, _, _ in samples), "sm_max_mhz": sm_max,
+            "power_w_max": max(p for _, p, _ in samples),
+            "power_w_median": statistics.median(p for _, p, _ in samples),
+            "power_limit_w": limit_w, "samples": len(samples),
+            "source": "nvml, 10 ms", "reasons": reasons}
+
+
+def summarize_smi_lines(lines):
+    """Clock record from `nvidia-smi --query-gpu=ClockSampler.QUERY
+    --format=csv,noheader,nounits` lines; a reason counts when any sample
+    shows it "Active".  None without a complete line."""
+    rows = [parts for parts in ([p.strip() for p in line.split(",")] for line in lines) if len(parts) >= 9]
+    if not rows:
+        return None
+
+    def num(v):
+        try:
+            return float(v)
+        except ValueError:
             return None
-        def num(v):
-            try:
-                return float(v)
-            except ValueError:
-                return None
-        sm = [num(r[1]) for r in rows if num(r[1]) is not None]
-        pw = [num(r[3]) for r in rows if num(r[3]) is not None]
-        reasons = set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for r in rows:
-            for name, v in zip(names, r[5:9]):
-                if v.strip().lower() == "active":
-                    reasons.add(name)
-        return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": num(rows[0][2]),
-                "power_w_max": max(pw) if pw else None,
-                "samples": len(rows),
-                "source": "nvidia-smi, 200 ms",
-                "reasons": sorted(reasons)}
+    sm = [num(r[1]) for r in rows if num(r[1]) is not None]
+    pw = [num(r[3]) for r in rows if num(r[3]) is not None]
+    reasons = set()
+    names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    for r in rows:
+        for name, v in zip(names, r[5:9]):
+            if v.strip().lower() == "active":
+                reasons.add(name)
+    return {"sm_mhz": statistics.median(sm) if sm else None,
+            "sm_max_mhz": num(rows[0][2]),
+            "power_w_max": max(pw) if pw else None,
+            "samples": len(rows),
+            "source": "nvidia-smi, 200 ms",
+            "reasons": sorted(reasons)}
 
 
 # --------------------------------------------------------- multi-rank
