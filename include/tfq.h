@@ -46,6 +46,10 @@
  *    keeps per-device state (launch attributes, the error word, the GEMM's
  *    ring of cluster-pacing counters) behind a mutex.  TMA descriptors are
  *    encoded on the host for every call and passed as kernel parameters.
+ *    The pacing ring has 64 slots taken in turn: more GEMMs than that in
+ *    flight at once on one device (on many streams) can share a slot, which
+ *    only loosens or delays the pacing (each wait gives up after 200 us);
+ *    results never depend on it.
  *  - Non-finite inputs (inf, NaN) are outside the contract: the codes and
  *    scales of a row holding one are unspecified.
  */

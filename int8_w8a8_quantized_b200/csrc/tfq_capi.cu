@@ -71,6 +71,11 @@ DeviceState* current_device_state(tfq_status* st) {
                        prop.minor);
             return nullptr;
         }
+        tfq_status rs = resolve_encode();
+        if (rs != TFQ_OK) {
+            *st = rs;
+            return nullptr;
+        }
         // One allocation: the error word in the first 128-byte line, then
         // kRoundSlots round counters, one line each.
         constexpr int kRoundSlots = 64;
@@ -78,16 +83,12 @@ DeviceState* current_device_state(tfq_status* st) {
         e = cudaMalloc(&err_word, 128 * (1 + kRoundSlots));
         if (e == cudaSuccess) e = cudaMemset(err_word, 0, 128 * (1 + kRoundSlots));
         if (e != cudaSuccess) {
+            if (err_word != nullptr) cudaFree(err_word);
             *st = fail(TFQ_ECUDA, "allocating the device error word: %s", cudaGetErrorString(e));
             return nullptr;
         }
         ds->round_ctrs = err_word + 32;
         ds->round_slots = kRoundSlots;
-        tfq_status rs = resolve_encode();
-        if (rs != TFQ_OK) {
-            *st = rs;
-            return nullptr;
-        }
         ds->sm_count = prop.multiProcessorCount;
         ds->cc_major = prop.major;
         ds->cc_minor = prop.minor;
