@@ -19,6 +19,7 @@
 
 #include <mutex>
 
+#include "tfq_args.h"
 #include "tfq_internal.h"
 
 namespace tfq {
@@ -99,21 +100,12 @@ using namespace tfq;
 extern "C" tfq_status tfq_scaled_fp8_linear_noalloc(const void* A_q, const float* s_a, const void* W_q,
                                                     const float* s_w, const void* bias_bf16, int64_t M, int64_t N,
                                                     int64_t K, void* out_bf16, void* stream) {
-    if (M < 0 || N < 0 || K < 0) return fail(TFQ_EINVAL, "negative size");
-    if (K == 0 || K % 16 != 0) return fail(TFQ_EINVAL, "K=%lld must be a positive multiple of 16", (long long)K);
-    if (N % 8 != 0) return fail(TFQ_EINVAL, "N=%lld is not a multiple of 8", (long long)N);
-    const int64_t lim = int64_t(1) << 31;
-    if (M >= lim || N >= lim || K >= lim) return fail(TFQ_EUNSUPPORTED, "size too large");
+    tfq_status st = check_gemm_args(A_q, s_a, W_q, s_w, bias_bf16, M, N, K, out_bf16);
+    if (st != TFQ_OK) return st;
     if (kGemmScratchBytes > TFQ_NOALLOC_SCRATCH_BYTES)
         return fail(TFQ_EUNSUPPORTED, "call needs %zu bytes of scratch, the static array holds %d",
                     kGemmScratchBytes, TFQ_NOALLOC_SCRATCH_BYTES);
     if (M == 0 || N == 0) return TFQ_OK;
-    if (A_q == nullptr || s_a == nullptr || W_q == nullptr || s_w == nullptr || out_bf16 == nullptr)
-        return fail(TFQ_EINVAL, "null pointer");
-    if (!aligned16(A_q) || !aligned16(s_a) || !aligned16(W_q) || !aligned16(s_w) || !aligned16(out_bf16) ||
-        (bias_bf16 != nullptr && !aligned16(bias_bf16)))
-        return fail(TFQ_EINVAL, "pointer not 16-byte aligned");
-    tfq_status st;
     DeviceState* ds = noalloc_state(&st);
     if (ds == nullptr) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);

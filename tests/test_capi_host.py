@@ -97,8 +97,10 @@ def test_quant_weight_validation(lib):
     (0, 16, 32, _capi.TFQ_OK),         # empty: no-op
     (4, 0, 32, _capi.TFQ_OK),
 ])
-def test_gemm_validation(lib, M, N, K, status):
-    assert lib.tfq_scaled_fp8_linear(ALIGNED, ALIGNED, ALIGNED, ALIGNED, None, M, N, K, ALIGNED, None) == status
+@pytest.mark.parametrize("entry", ["tfq_scaled_fp8_linear", "tfq_scaled_fp8_linear_noalloc"])
+def test_gemm_validation(lib, entry, M, N, K, status):
+    f = getattr(lib, entry)
+    assert f(ALIGNED, ALIGNED, ALIGNED, ALIGNED, None, M, N, K, ALIGNED, None) == status
 
 
 def test_int8_gemm_k_limit(lib):
@@ -109,8 +111,9 @@ def test_int8_gemm_k_limit(lib):
     assert f(ALIGNED, ALIGNED, ALIGNED, ALIGNED, None, 0, 16, 131056, ALIGNED, None) == _capi.TFQ_OK  # empty
 
 
-def test_gemm_rejects_null_and_misaligned(lib):
-    f = lib.tfq_scaled_fp8_linear
+@pytest.mark.parametrize("entry", ["tfq_scaled_fp8_linear", "tfq_scaled_fp8_linear_noalloc"])
+def test_gemm_rejects_null_and_misaligned(lib, entry):
+    f = getattr(lib, entry)
     assert f(None, ALIGNED, ALIGNED, ALIGNED, None, 4, 16, 32, ALIGNED, None) == _capi.TFQ_EINVAL
     assert f(ALIGNED, ALIGNED, ALIGNED, ALIGNED, ALIGNED + 2, 4, 16, 32, ALIGNED, None) == _capi.TFQ_EINVAL
     assert f(ALIGNED, ALIGNED, ALIGNED, ALIGNED, None, 4, 16, 32, ALIGNED + 4, None) == _capi.TFQ_EINVAL
@@ -121,6 +124,8 @@ def test_valid_call_without_gpu_fails_loudly(lib):
     st = lib.tfq_quant_act_fp8_per_token(ALIGNED, 4, 32, 448.0, ALIGNED, ALIGNED, None)
     assert st in (_capi.TFQ_ECUDA, _capi.TFQ_EUNSUPPORTED)
     assert lib.tfq_scaled_fp8_linear(ALIGNED, ALIGNED, ALIGNED, ALIGNED, None, 4, 16, 32, ALIGNED, None) \
+        in (_capi.TFQ_ECUDA, _capi.TFQ_EUNSUPPORTED)
+    assert lib.tfq_scaled_fp8_linear_noalloc(ALIGNED, ALIGNED, ALIGNED, ALIGNED, None, 4, 16, 32, ALIGNED, None) \
         in (_capi.TFQ_ECUDA, _capi.TFQ_EUNSUPPORTED)
 
 
