@@ -32,6 +32,8 @@ from ._capi import (  # noqa: F401
     tfq_quant_mxfp8,
     tfq_quant_weight_per_channel,
     tfq_scaled_fp8_linear,
+    tfq_scaled_fp8_linear_f16acc,
+    tfq_scaled_fp8_linear_noalloc,
     tfq_scaled_int8_linear,
     w8a8_int8_linear,
     w8a8_linear,
@@ -41,6 +43,8 @@ __all__ = [
     "tfq_quant_act_fp8_per_token",
     "tfq_quant_weight_per_channel",
     "tfq_scaled_fp8_linear",
+    "tfq_scaled_fp8_linear_f16acc",
+    "tfq_scaled_fp8_linear_noalloc",
     "tfq_quant_act_int8_per_token",
     "tfq_scaled_int8_linear",
     "w8a8_int8_linear",

@@ -183,6 +183,23 @@ def tfq_quant_weight_per_channel(w, dtype: str = "fp8", qmax: float | None = Non
 def tfq_scaled_fp8_linear(A_q, s_a, W_q, s_w, bias=None, out=None, stream=None):
     """A_q uint8 [M, K], s_a fp32 [M], W_q uint8 [N, K], s_w fp32 [N], bias bf16 [N] or None
     -> out bf16 [M, N]."""
+    return _scaled_fp8_gemm("tfq_scaled_fp8_linear", A_q, s_a, W_q, s_w, bias, out, stream)
+
+
+def tfq_scaled_fp8_linear_f16acc(A_q, s_a, W_q, s_w, bias=None, out=None, stream=None):
+    """tfq_scaled_fp8_linear with FP16 partial sums on the tensor cores: the
+    result is defined only while every partial sum fits in FP16, i.e. for
+    activations quantized with a reduced qmax (7, 14)."""
+    return _scaled_fp8_gemm("tfq_scaled_fp8_linear_f16acc", A_q, s_a, W_q, s_w, bias, out, stream)
+
+
+def tfq_scaled_fp8_linear_noalloc(A_q, s_a, W_q, s_w, bias=None, out=None, stream=None):
+    """tfq_scaled_fp8_linear that never allocates device memory (its kernel's
+    scratch words live in a static array of the library)."""
+    return _scaled_fp8_gemm("tfq_scaled_fp8_linear_noalloc", A_q, s_a, W_q, s_w, bias, out, stream)
+
+
+def _scaled_fp8_gemm(entry, A_q, s_a, W_q, s_w, bias, out, stream):
     import torch
     _require(A_q, torch.uint8, 2, "A_q")
     dev = A_q.device
@@ -203,10 +220,10 @@ def tfq_scaled_fp8_linear(A_q, s_a, W_q, s_w, bias=None, out=None, stream=None):
     if tuple(out.shape) != (M, N):
         raise ValueError("out shape")
     with torch.cuda.device(A_q.device):
-        st = raw.tfq_scaled_fp8_linear(A_q.data_ptr(), s_a.data_ptr(), W_q.data_ptr(), s_w.data_ptr(),
-                                       None if bias is None else bias.data_ptr(), M, N, K, out.data_ptr(),
-                                       _stream_handle(stream))
-    _check(st, "tfq_scaled_fp8_linear")
+        st = getattr(raw, entry)(A_q.data_ptr(), s_a.data_ptr(), W_q.data_ptr(), s_w.data_ptr(),
+                                 None if bias is None else bias.data_ptr(), M, N, K, out.data_ptr(),
+                                 _stream_handle(stream))
+    _check(st, entry)
     return out
 
 

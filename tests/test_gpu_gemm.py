@@ -143,6 +143,32 @@ def test_tensor_wrapper_linear():
     _gpu.gemm_tolerance_check(y, y_ref, "wrapper")
 
 
+@pytest.mark.parametrize("entry", ["tfq_scaled_fp8_linear", "tfq_scaled_fp8_linear_f16acc",
+                                   "tfq_scaled_fp8_linear_noalloc"])
+def test_gemm_tensor_wrappers_match_raw(entry):
+    """The tensor-level wrappers pass their operands to the C entry point of
+    the same name unchanged: same bits as the raw call (activations at qmax
+    7, where the FP16-accumulator GEMM is defined too)."""
+    import int8_w8a8_quantized_b200 as pkg
+    M, N, K = 300, 264, 512
+    x = workloads.activations(M, K, seed=12, device="cuda")
+    w = workloads.weights(N, K, seed=13, std=0.02, device="cuda")
+    b = workloads.bias(N, seed=14, device="cuda")
+    A, sa = _gpu.quant_act_fp8(x, 7.0)
+    Wq, sw = pkg.tfq_quant_weight_per_channel(w, "fp8")
+    y = getattr(pkg, entry)(A, sa, Wq, sw, b)
+    out = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+    st = getattr(_capi.raw, entry)(A.data_ptr(), sa.data_ptr(), Wq.data_ptr(), sw.data_ptr(), b.data_ptr(),
+                                   M, N, K, out.data_ptr(), _gpu.stream_handle())
+    assert st == _capi.TFQ_OK, _capi.last_error_message()
+    _gpu.check_device_error()
+    assert torch.equal(y.view(torch.int16), out.view(torch.int16))
+    if entry != "tfq_scaled_fp8_linear_f16acc":
+        y_ref = oracle.scaled_fp8_linear(A.cpu().numpy(), sa.cpu().numpy(), Wq.cpu().numpy(), sw.cpu().numpy(),
+                                         _gpu.bf16_bits_np(b))
+        _gpu.gemm_tolerance_check(y, y_ref, entry)
+
+
 @pytest.mark.parametrize("M,N,K", [(4096, 4096, 256), (3000, 5120, 384)])
 def test_pair_kernel_several_tiles_per_cluster(M, N, K):
     """256 / 240 pair tiles over the 74 clusters: every cluster runs 3-4
