@@ -49,6 +49,46 @@ def test_max_over_ranks_and_weak_scaling(world):
         assert value == pytest.approx(world * 1.0 / (expect_ms * 1e-3))
 
 
+def _dying_worker(rank, world, port, q):
+    import datetime
+    import time
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=5))
+    if rank == 1:
+        os._exit(3)  # leaves between steps: before the reduction of the step timer
+    t0 = time.time()
+    try:
+        bench.max_over_ranks(1.0, torch.device("cpu"))
+        q.put(("no error", time.time() - t0))
+    except Exception as e:  # noqa: BLE001 -- any error type: what matters is that the wait ends
+        q.put((type(e).__name__, time.time() - t0))
+    q.close()
+    q.join_thread()
+    os._exit(0)  # no destroy_process_group: its peer is gone
+
+
+def test_rank_that_leaves_ends_the_others_with_an_error():
+    """A rank that exits before the timer's reduction: the remaining rank's
+    collective ends with an error within the process group's timeout (5 s
+    here) instead of waiting for good."""
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_dying_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    try:
+        what, seconds = q.get(timeout=120)
+    finally:
+        for p in procs:
+            p.join(timeout=30)
+            if p.is_alive():
+                p.kill()
+    assert what != "no error"
+    assert seconds < 60
+    assert procs[1].exitcode == 3
+
+
 def test_single_rank_throughput():
     assert bench.aggregate_throughput(1, 2 * 10 ** 12, 1000.0) == pytest.approx(2.0)
 
