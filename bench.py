@@ -598,10 +598,36 @@ def e2e_arm(args, wl, qmaxes, quant_fn, gemm_fn, xs, lins, aq, ys, stream, sh, c
     t1.record(stream)
     torch.cuda.synchronize()
     ms = t0.elapsed_time(t1) / args.e2e_steps
+
+    # Floor of the step over PCIe: the same copies with no kernels, both
+    # directions at once on the same two copy streams (same buffers, same
+    # bytes; the contents written are the ones already there).
+    def copies_only():
+        copy_in.wait_stream(stream)
+        copy_out.wait_stream(stream)
+        with torch.cuda.stream(copy_in):
+            for n in order:
+                xs[n].copy_(hx[n], non_blocking=True)
+        with torch.cuda.stream(copy_out):
+            for key, y in ys.items():
+                hy[key].copy_(y, non_blocking=True)
+        stream.wait_stream(copy_in)
+        stream.wait_stream(copy_out)
+
+    copies_only()
+    torch.cuda.synchronize()
+    t0.record(stream)
+    for _ in range(args.e2e_steps):
+        copies_only()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    copy_ms = t0.elapsed_time(t1) / args.e2e_steps
     flops = wl.flops() // len(wl.act_qmax) * len(qmaxes)
     return {"value": flops / (ms * 1e-3) / 1e12, "unit": unit_name(args.dtype), "ms_per_step": ms,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": args.e2e_steps,
-            "host_buffers": "pinned", "overlap": "H2D and D2H on two copy streams, overlapping compute"}
+            "host_buffers": "pinned", "overlap": "H2D and D2H on two copy streams, overlapping compute",
+            "copies_alone_ms": round(copy_ms, 3), "frac_of_copy_floor": round(copy_ms / ms, 4),
+            "floor": "the step's H2D and D2H copies alone, both directions at once, no kernels"}
 
 
 # ------------------------------------------------------------ CPU oracle
