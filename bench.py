@@ -803,35 +803,43 @@ def quantizer_arm(args, rank, world, local_rank):
     hbm = peaks.get("hbm_gbs", FALLBACK_HBM_GBS)
     # end to end: X from pinned host memory, codes and scales back, every
     # step; H2D and D2H on two copy streams, so that the next step's input
-    # crosses PCIe while this step's outputs go back (events keep each copy
-    # after the kernels that read or write its buffer, also across steps)
+    # crosses PCIe while this step's outputs go back.  The device input and
+    # outputs are double-buffered (steps alternate between two sets), and
+    # events keep each copy after the kernels that read or write its buffer.
     hx = torch.empty(x.shape, dtype=x.dtype, pin_memory=True)
     hx.copy_(x)
     outs = [q8, s8, qi, si]
     hout = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in outs]
+    xbuf = [x, torch.empty_like(x)]
+    obuf = [outs, [torch.empty_like(t) for t in outs]]
     copy_in, copy_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
-    pending = {}
+    x_read, outs_read, counter = {}, {}, [0]
 
     def e2e_step():
-        if "x_read" in pending:
-            copy_in.wait_event(pending["x_read"])
+        k = counter[0] % 2
+        counter[0] += 1
+        xk, (q8k, s8k, qik, sik) = xbuf[k], obuf[k]
+        if k in x_read:
+            copy_in.wait_event(x_read[k])
         with torch.cuda.stream(copy_in):
-            x.copy_(hx, non_blocking=True)
+            xk.copy_(hx, non_blocking=True)
         landed = torch.cuda.Event()
         landed.record(copy_in)
         stream.wait_event(landed)
-        if "outs_read" in pending:
-            stream.wait_event(pending["outs_read"])
-        step()
-        done = torch.cuda.Event()
-        done.record(stream)
-        pending["x_read"] = done
-        copy_out.wait_event(done)
+        if k in outs_read:
+            stream.wait_event(outs_read[k])
+        check(lib.tfq_quant_act_fp8_per_token(xk.data_ptr(), M, K, 448.0, q8k.data_ptr(), s8k.data_ptr(), sh),
+              "fp8")
+        check(lib.tfq_quant_weight_per_channel(xk.data_ptr(), M, K, _capi.TFQ_DTYPE_INT8, 127.0, qik.data_ptr(),
+                                               sik.data_ptr(), sh), "int8")
+        x_read[k] = torch.cuda.Event()
+        x_read[k].record(stream)
+        copy_out.wait_event(x_read[k])
         with torch.cuda.stream(copy_out):
-            for h, t in zip(hout, outs):
+            for h, t in zip(hout, obuf[k]):
                 h.copy_(t, non_blocking=True)
-        pending["outs_read"] = torch.cuda.Event()
-        pending["outs_read"].record(copy_out)
+        outs_read[k] = torch.cuda.Event()
+        outs_read[k].record(copy_out)
 
     def copies_alone():
         copy_in.wait_stream(stream)
@@ -844,20 +852,25 @@ def quantizer_arm(args, rank, world, local_rank):
         stream.wait_stream(copy_in)
         stream.wait_stream(copy_out)
 
+    # a step is ~1 ms: enough steps that filling and draining the copy
+    # pipeline are a small part of the timed region
+    n_e2e = max(args.e2e_steps, 30)
+
     def timed(fn):
+        fn()
         fn()
         torch.cuda.synchronize()
         t0 = torch.cuda.Event(enable_timing=True); t1 = torch.cuda.Event(enable_timing=True)
         t0.record(stream)
         copy_in.wait_stream(stream)  # no copy of the timed steps starts before t0
         copy_out.wait_stream(stream)
-        for _ in range(args.e2e_steps):
+        for _ in range(n_e2e):
             fn()
         stream.wait_stream(copy_out)
         stream.wait_stream(copy_in)
         t1.record(stream)
         torch.cuda.synchronize()
-        return t0.elapsed_time(t1) / args.e2e_steps
+        return t0.elapsed_time(t1) / n_e2e
 
     e2e_ms = timed(e2e_step)
     e2e_copy_ms = timed(copies_alone)
@@ -887,8 +900,9 @@ def quantizer_arm(args, rank, world, local_rank):
         "e2e": {"value": round(world * nbytes / (e2e_ms * 1e-3) / 1e9, 1), "unit": "GB/s", "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": x.numel() * 2,
                 "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t in outs),
-                "steps": args.e2e_steps, "host_buffers": "pinned",
-                "overlap": "H2D and D2H on two copy streams, overlapping the quantizers and each other",
+                "steps": n_e2e, "host_buffers": "pinned",
+                "overlap": "H2D and D2H on two copy streams, overlapping the quantizers and each other; "
+                           "device input and outputs double-buffered",
                 "copies_alone_ms": round(e2e_copy_ms, 4), "frac_of_copy_floor": round(e2e_copy_ms / e2e_ms, 4),
                 "floor": "the step's H2D and D2H copies alone, both directions at once, no kernels"},
     }
