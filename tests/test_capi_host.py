@@ -164,3 +164,19 @@ def test_mxfp8_valid_call_without_gpu_fails_loudly(lib):
     assert lib.tfq_quant_mxfp8(ALIGNED, 4, 64, ALIGNED, ALIGNED, None) in (_capi.TFQ_ECUDA, _capi.TFQ_EUNSUPPORTED)
     assert lib.tfq_mxfp8_linear(ALIGNED, ALIGNED, ALIGNED, ALIGNED, None, 4, 16, 64, ALIGNED, None) \
         in (_capi.TFQ_ECUDA, _capi.TFQ_EUNSUPPORTED)
+
+
+def test_missing_library_raises_no_fallback():
+    """Without libtfq.so every call raises: there is no other implementation
+    to fall back to.  Run in a fresh process (the loaded library is cached)."""
+    import sys
+    code = ("from int8_w8a8_quantized_b200 import _capi\n"
+            "_capi.LIB_PATH = '/nonexistent/libtfq.so'\n"
+            "import int8_w8a8_quantized_b200 as p\n"
+            "try:\n"
+            "    p.raw.tfq_version()\n"
+            "except RuntimeError as e:\n"
+            "    print('raised:', e)\n")
+    r = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, timeout=120, cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-2000:]
+    assert r.stdout.startswith("raised:") and "not built" in r.stdout
