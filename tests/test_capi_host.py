@@ -180,3 +180,46 @@ def test_missing_library_raises_no_fallback():
     r = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, timeout=120, cwd=ROOT)
     assert r.returncode == 0, r.stderr[-2000:]
     assert r.stdout.startswith("raised:") and "not built" in r.stdout
+
+
+C_PROGRAM = r"""
+#include <stdio.h>
+#include <string.h>
+#include "tfq.h"
+
+int main(void)
+{
+    const void *p = (const void *)0x10000; /* aligned, never dereferenced: every call below is rejected */
+    if (tfq_version() != 100)
+        return 1;
+    if (strcmp(tfq_status_string(TFQ_EINVAL), "TFQ_EINVAL") != 0)
+        return 2;
+    if (tfq_quant_act_fp8_per_token(p, 4, 24, 448.0f, (void *)p, (float *)p, NULL) != TFQ_EINVAL)
+        return 3;
+    if (tfq_last_error_message()[0] == '\0')
+        return 4;
+    if (tfq_scaled_fp8_linear(p, (const float *)p, p, (const float *)p, NULL, 4, 12, 32, (void *)p, NULL)
+        != TFQ_EINVAL)
+        return 5;
+    if (tfq_mxfp8_scale_bytes(129, 160) != 2 * 2 * 512)
+        return 6;
+    if (tfq_selftest_wait_timeout(0, NULL) != TFQ_EINVAL)
+        return 7;
+    printf("ok\n");
+    return 0;
+}
+"""
+
+
+def test_header_is_plain_c_and_links(lib, tmp_path):
+    """include/tfq.h compiles as strict C99 (warnings as errors) and a C
+    program links libtfq.so and gets the documented host-side answers."""
+    src = tmp_path / "use_tfq.c"
+    src.write_text(C_PROGRAM)
+    exe = tmp_path / "use_tfq"
+    pkg = os.path.dirname(_capi.LIB_PATH)
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-Werror", "-pedantic", "-I", os.path.join(ROOT, "include"),
+                    str(src), "-L", pkg, "-ltfq", f"-Wl,-rpath,{pkg}", "-o", str(exe)], check=True,
+                   capture_output=True, text=True)
+    r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert r.returncode == 0 and r.stdout.strip() == "ok", (r.returncode, r.stdout, r.stderr)
