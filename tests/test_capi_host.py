@@ -223,3 +223,10 @@ def test_header_is_plain_c_and_links(lib, tmp_path):
                    capture_output=True, text=True)
     r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
     assert r.returncode == 0 and r.stdout.strip() == "ok", (r.returncode, r.stdout, r.stderr)
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU behaviour")
+def test_smoke_without_gpu_raises(lib):
+    import __graft_entry__
+    with pytest.raises(RuntimeError, match="CUDA device"):
+        __graft_entry__.smoke()
