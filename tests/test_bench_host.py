@@ -166,3 +166,26 @@ def test_path_roofline_floor():
     assert out["frac_measured_peaks"] == pytest.approx(0.7)
     # at the 4.5 PFLOP/s spec GEMM 1 takes 4e12 / 4.5e15 s, still above its 0.25 ms of bytes
     assert out["floor_ms_spec"] == pytest.approx(0.5 + 1e3 * 4e12 / (bench.FP8_SPEC_TFLOPS * 1e12) + 1.0, rel=1e-4)
+
+
+def test_profile_commands_still_run_with_this_bench(monkeypatch):
+    """Every profile summary names the command that produced it: each
+    `python bench.py ...` there parses with the bench's current options, and
+    each ncu command leaves the GPU clocks alone (--clock-control none)."""
+    import glob
+    import os
+    import shlex
+    files = sorted(glob.glob(os.path.join(bench.ROOT, "profiles", "*.md")))
+    assert files
+    for f in files:
+        text = open(f, encoding="utf-8").read().replace("\\\n", " ")
+        cmds = [line.strip() for line in text.splitlines() if line.strip().startswith(("python bench.py", "ncu "))]
+        assert any(c.startswith("ncu ") for c in cmds), f
+        for c in cmds:
+            if c.startswith("ncu ") and " -i " not in c:  # `ncu -i` reads a saved report: no GPU
+                assert "--clock-control none" in c, (f, c)
+            words = shlex.split(c)
+            argv = words[words.index("bench.py"):] if "bench.py" in words else None
+            if argv is not None:
+                monkeypatch.setattr(sys, "argv", argv)
+                bench.parse_args()  # exits (SystemExit) on an option the bench no longer has
