@@ -470,6 +470,7 @@ def gpu_arm(args, wl, rank, world, local_rank):
                           f"the {args.steps} timed steps (one kernel per step)") if sample_one
         else "every kernel of every timed step",
         "gpu_launches": launches[0], "clocks": clk,
+        "sm_count": torch.cuda.get_device_properties(dev).multi_processor_count,
         "per_linear": {},
     }
     for (a, b, (m, n, k)) in ev["gemm"]:
@@ -695,11 +696,40 @@ def _x_rows(wl, lin, n, seed):
     return x.contiguous().view(torch.int16).numpy().view(np.uint16)
 
 
-def cpu_baseline(wl, seconds, dtype="fp8"):
+def cpu_baseline(wl, seconds, dtype="fp8", single_thread_seconds=None):
+    """The oracle on every host core (OpenMP over rows), then on one core
+    (a smaller sample of the same kind), both as FLOPs of the sample / time."""
     import oracle
     flops, secs, desc = oracle_sample(wl, seconds, dtype=dtype)
-    return {"value": flops / secs / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
-            "sample": desc, "seconds": secs}
+    out = {"value": flops / secs / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
+           "sample": desc, "seconds": secs}
+    if single_thread_seconds:
+        threads = oracle.num_threads()
+        oracle.set_num_threads(1)
+        try:
+            f1, s1, d1 = oracle_sample(wl, single_thread_seconds, seed=1, dtype=dtype)
+        finally:
+            oracle.set_num_threads(threads)
+        out["single_thread"] = {"value": f1 / s1 / 1e12, "unit": "TFLOP/s", "cores": 1, "sample": d1,
+                                "seconds": s1}
+    return out
+
+
+# Dense 8-bit tensor-core rate of one B200 SM per clock (E4M3 or S8 operands):
+# twice the 8192 bf16 FLOP/clk/SM behind the 2.25 PFLOP/s dense bf16 figure.
+FP8_FLOP_PER_CLK_PER_SM = 16384
+
+
+def clock_normalised(achieved_tflops, clocks, sm_count):
+    """The GEMM's rate against the tensor-core peak at the SM clock sampled
+    during the timed region (SMs x 16384 FLOP/clk x median MHz): comparable
+    between boxes whose power-capped clocks differ."""
+    mhz = (clocks or {}).get("sm_mhz")
+    if not mhz or not sm_count:
+        return None
+    peak = sm_count * FP8_FLOP_PER_CLK_PER_SM * mhz * 1e6 / 1e12
+    return {"frac": round(achieved_tflops / peak, 4), "peak_at_clock": round(peak, 1), "sm_mhz": mhz,
+            "sm_count": sm_count, "flop_per_clk_per_sm": FP8_FLOP_PER_CLK_PER_SM}
 
 
 def path_roofline(res, steps, peaks, fp8_peak):
@@ -907,26 +937,44 @@ def quantizer_arm(args, rank, world, local_rank):
                 "floor": "the step's H2D and D2H copies alone, both directions at once, no kernels"},
     }
     if world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = quantizer_cpu_baseline(x.cpu(), args.cpu_seconds)
+        line["cpu_baseline"] = quantizer_cpu_baseline(x.cpu(), args.cpu_seconds,
+                                                      single_thread_seconds=max(2.0, args.cpu_seconds / 2))
     print(json.dumps(line), flush=True)
 
 
-def quantizer_cpu_baseline(x_cpu, seconds: float = 10.0):
+def quantizer_cpu_baseline(x_cpu, seconds: float = 10.0, single_thread_seconds=None):
+    """The oracle's FP8 and INT8 quantizers over the whole input, on every
+    host core; then (optionally) on one core."""
     import numpy as np
     import torch
     import oracle
     bits = x_cpu.contiguous().view(torch.int16).numpy().view(np.uint16)
     M, K = bits.shape
-    t0 = time.perf_counter()
-    n = 0
-    while time.perf_counter() - t0 < seconds or n == 0:
-        oracle.quant_rows_fp8(bits, 448.0)
-        oracle.quant_rows_int8(bits, 127.0)
-        n += 1
-    secs = time.perf_counter() - t0
-    return {"value": n * 2 * (3 * M * K + 4 * M) / secs / 1e9, "unit": "GB/s", "cores": oracle.num_threads(),
-            "kind": "oracle", "sample": f"{n} passes over the full [{M}, {K}] input (FP8 and INT8)", "seconds": secs,
-            "ms_per_pass": 1e3 * secs / n}
+
+    def passes(limit):
+        t0 = time.perf_counter()
+        n = 0
+        while time.perf_counter() - t0 < limit or n == 0:
+            oracle.quant_rows_fp8(bits, 448.0)
+            oracle.quant_rows_int8(bits, 127.0)
+            n += 1
+        return n, time.perf_counter() - t0
+
+    n, secs = passes(seconds)
+    out = {"value": n * 2 * (3 * M * K + 4 * M) / secs / 1e9, "unit": "GB/s", "cores": oracle.num_threads(),
+           "kind": "oracle", "sample": f"{n} passes over the full [{M}, {K}] input (FP8 and INT8)", "seconds": secs,
+           "ms_per_pass": 1e3 * secs / n}
+    if single_thread_seconds:
+        threads = oracle.num_threads()
+        oracle.set_num_threads(1)
+        try:
+            n1, s1 = passes(single_thread_seconds)
+        finally:
+            oracle.set_num_threads(threads)
+        out["single_thread"] = {"value": n1 * 2 * (3 * M * K + 4 * M) / s1 / 1e9, "unit": "GB/s", "cores": 1,
+                                "sample": f"{n1} passes over the full [{M}, {K}] input (FP8 and INT8)",
+                                "seconds": s1}
+    return out
 
 
 def use_all_host_cores_for_oracle():
@@ -1064,6 +1112,7 @@ def main():
             "frac_of_burst_peak": round(gemm_tflops / (bf16_burst * FP8_OVER_BF16), 4),
             "avg_launch_ms": round(gemm_avg_ms, 4),
             "frac_of_fp8_spec": round(gemm_tflops / FP8_SPEC_TFLOPS, 4),
+            "clock_normalised": clock_normalised(gemm_tflops, res["clocks"], res.get("sm_count")),
         },
         "quantizer": {
             "kernel": qname,
@@ -1090,7 +1139,8 @@ def main():
         e2e["value"] = round(world * e2e["value"], 3)
         line["e2e"] = e2e
     if world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(wl, args.cpu_seconds, args.dtype)
+        line["cpu_baseline"] = cpu_baseline(wl, args.cpu_seconds, args.dtype,
+                                            single_thread_seconds=max(2.0, args.cpu_seconds / 2))
     print(json.dumps(line), flush=True)
     return 0
 

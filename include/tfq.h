@@ -235,27 +235,30 @@ TFQ_API tfq_status tfq_mxfp8_linear(const void *A_q, const void *sf_a, const voi
  * library for callers that cannot allocate; the pages have no counterpart.)
  *
  * Same arguments, preconditions, result and errors as tfq_scaled_fp8_linear.
- * The regular entry points cudaMalloc one device word per device on their
- * first call (where a kernel records a bounded wait that ran out).  Callers
- * that must not allocate device memory -- a framework that owns all device
- * memory through its own pool, a process that has reserved nearly all of
- * HBM, code running where a possibly synchronizing CUDA call is not allowed
- * -- call this one instead: that word lives in a file-scope __device__ array
+ * The regular entry points cudaMalloc one small device buffer per device on
+ * their first call (the word where a kernel records a bounded wait that ran
+ * out, and the counters the GEMM's clusters keep pace with).  Callers that
+ * must not allocate device memory -- a framework that owns all device memory
+ * through its own pool, a process that has reserved nearly all of HBM --
+ * call this one instead: those words live in a file-scope __device__ array
  * of TFQ_NOALLOC_SCRATCH_BYTES bytes, and no call allocates (no cudaMalloc,
  * cudaFree or allocating library routine).
  *  - The caller still owns and passes every input and output.
  *  - A call needs 136 bytes of the array whatever M, N and K (the error
  *    word and, one 128-byte line further, two counters the kernel's clusters
- *    use to keep pace, which the kernel leaves at zero); a call needing more
- *    than the array holds is rejected with TFQ_EUNSUPPORTED.
+ *    use to keep pace); a call needing more than the array holds is rejected
+ *    with TFQ_EUNSUPPORTED.
  *  - The first call on a device does a one-time set-up with that device
  *    current (device checks, cudaGetSymbolAddress of the array, which may
  *    load the library's device code into the context); make that first call
  *    before any stream capture.
+ *  - Every call issues stream-ordered CUDA calls (a memset and a kernel
+ *    launch), so it cannot be made where CUDA calls are not allowed, such as
+ *    inside a host callback enqueued on a stream.
  *  - Every call on a device shares the array, which keeps the last call's
- *    contents; each call clears the error word and the counter on `stream`
- *    before its kernel.  Calls that overlap on the GPU (on different
- *    streams) race on both (the counter only paces; results stay correct).
+ *    contents; each call clears those 136 bytes on `stream` before its
+ *    kernel.  Calls that overlap on the GPU (on different streams) race on
+ *    them (the counters only pace the clusters; results stay correct).
  *  - A bounded wait that runs out is recorded in the array's word only:
  *    this entry point does not read it back (that would need a host
  *    synchronization), and tfq_device_error() does not see it.

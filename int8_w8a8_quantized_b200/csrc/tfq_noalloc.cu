@@ -6,12 +6,18 @@
 // out, and the counters the GEMM's clusters use to keep pace) with
 // cudaMalloc on their first call on a device.  Some callers cannot allow
 // that: a host framework that owns every byte of device memory through its
-// own pool and forbids libraries from calling cudaMalloc, a serving process
-// that reserved nearly all of HBM up front, or code running where a CUDA API
-// call that may synchronize the device is not allowed (for example inside a
-// host callback enqueued on a stream).  This entry point runs the same GEMM
-// kernel, but the words the kernel writes live in a file-scope __device__
-// array, so no call allocates anything.
+// own pool and forbids libraries from calling cudaMalloc, or a serving
+// process that reserved nearly all of HBM up front.  This entry point runs
+// the same GEMM kernel, but the words the kernel writes live in a
+// file-scope __device__ array, so no call allocates anything.
+//
+// What it guarantees: no cudaMalloc, cudaFree or other allocating call, on
+// any call.  Every call still issues stream-ordered CUDA calls (a memset of
+// the scratch words and the kernel launch), and the first call on a device
+// also queries the device and looks up the array's address; so, like any
+// call that launches work, it cannot be made from inside a host callback
+// enqueued on a stream, and its first call on a device belongs outside
+// stream capture.
 //
 // The array is part of the library image: every GPU that loads the library
 // holds it until the process exits.
@@ -57,10 +63,12 @@ DeviceState* noalloc_state(tfq_status* st) {
     std::lock_guard<std::mutex> lock(g_noalloc_mutex);
     DeviceState* ds = &g_noalloc_states[dev];
     if (ds->device < 0) {
-        int major = 0, minor = 0, sms = 0;
+        int major = 0, minor = 0, sms = 0, smem_optin = 0;
         e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
         if (e == cudaSuccess) e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
         if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        if (e == cudaSuccess)
+            e = cudaDeviceGetAttribute(&smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
         if (e != cudaSuccess) {
             *st = fail(TFQ_ECUDA, "cudaDeviceGetAttribute: %s", cudaGetErrorString(e));
             return nullptr;
@@ -83,6 +91,7 @@ DeviceState* noalloc_state(tfq_status* st) {
         ds->sm_count = sms;
         ds->cc_major = major;
         ds->cc_minor = minor;
+        ds->smem_optin = static_cast<size_t>(smem_optin);
         ds->err_word = ptr;
         ds->round_ctrs = ptr + 32;  // one slot: calls overlapping on the GPU share it
         ds->round_slots = 1;
@@ -109,10 +118,11 @@ extern "C" tfq_status tfq_scaled_fp8_linear_noalloc(const void* A_q, const float
     DeviceState* ds = noalloc_state(&st);
     if (ds == nullptr) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    // The array keeps the previous call's contents: the error word must start
-    // at zero (the round counter in the next line is left at zero by the
-    // kernel that used it last).
-    const cudaError_t e = cudaMemsetAsync(ds->err_word, 0, sizeof(uint32_t), s);
+    // The array keeps the previous call's contents: the error word and both
+    // pacing words must start at zero.  (The kernel's last cluster leaves the
+    // pacing words at zero, but a call that overlapped another one on the
+    // GPU, or whose waits gave up, may not have.)
+    const cudaError_t e = cudaMemsetAsync(ds->err_word, 0, kGemmScratchBytes, s);
     if (e != cudaSuccess) return fail(TFQ_ECUDA, "clearing the scratch word: %s", cudaGetErrorString(e));
     return launch_scaled_fp8_gemm(A_q, s_a, W_q, s_w, bias_bf16, M, N, K, out_bf16, s, ds);
 }

@@ -37,6 +37,7 @@ from __future__ import annotations
 import ctypes
 import os
 import subprocess
+import sys
 import threading
 
 import numpy as np
@@ -68,9 +69,15 @@ def _load():
     with _lock:
         if _lib is None:
             # TFQ_ORACLE_LIB names another build of tfq_oracle.c to load
-            # instead (the mutation test runs the pins against copies of the
-            # source with a planted mistake this way).
+            # instead: the mutation test runs the pins against copies of the
+            # source with a planted mistake this way.  Taking it is announced
+            # on stderr, and the GPU parity tests refuse to run under it
+            # (tests/conftest.py), so a stray variable cannot swap the checker
+            # silently.
             override = os.environ.get("TFQ_ORACLE_LIB")
+            if override:
+                sys.stderr.write(f"oracle: loading {override} (named by TFQ_ORACLE_LIB) "
+                                 "instead of the built oracle\n")
             lib = ctypes.CDLL(override if override else build())
             P = ctypes.c_void_p
             I64 = ctypes.c_int64

@@ -110,6 +110,32 @@ def sample_rows(M: int, n: int, seed: int, tail: int = 128) -> np.ndarray:
     return np.unique(np.concatenate([pick, last, [0]])).astype(np.int64)
 
 
+# Rows a GEMM CTA owns: 128 (one CTA of a pair holds 128 rows of a 256-row
+# tile; the one-CTA kernel's tiles are 128 rows).
+CTA_ROWS = 128
+
+
+def tile_sample_rows(M: int, seed: int, n_random: int = 512, block: int = CTA_ROWS) -> np.ndarray:
+    """Rows of a full-size GEMM to recompute with the oracle: one seeded row
+    inside every `block`-row slice of M (so every CTA's share of every M tile
+    is compared), n_random more seeded rows, and every row of the last,
+    ragged slice.  Checks that every slice is hit."""
+    rng = np.random.default_rng(seed)
+    starts = np.arange(0, M, block, dtype=np.int64)
+    per_block = starts + rng.integers(0, np.minimum(block, M - starts))
+    rows = np.unique(np.concatenate([per_block, sample_rows(M, n_random, seed + 1, tail=block)]))
+    assert_covers_blocks(rows, M, block)
+    return rows
+
+
+def assert_covers_blocks(rows: np.ndarray, M: int, block: int = CTA_ROWS) -> None:
+    """Every `block`-row slice of [0, M) holds at least one of `rows`."""
+    hit = np.zeros((M + block - 1) // block, dtype=bool)
+    hit[np.asarray(rows) // block] = True
+    missing = np.flatnonzero(~hit)
+    assert missing.size == 0, f"row slices never compared: {missing[:10]} ..."
+
+
 # MXFP8 scale-factor layout (include/tfq.h): 512-byte atoms of 128 rows x 4
 # K blocks, atom (b // 4) * RA + r // 128; inside it row r % 32 owns 16 bytes,
 # (r % 128) // 32 picks the 4-byte word, b % 4 the byte.

@@ -17,3 +17,19 @@ if ROOT not in sys.path:
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs an NVIDIA B200 (sm_100a) and the built libtfq.so")
     config.addinivalue_line("markers", "slow: full-size parity cases (minutes)")
+
+
+def pytest_report_header(config):
+    override = os.environ.get("TFQ_ORACLE_LIB")
+    if override:
+        return f"oracle library override (TFQ_ORACLE_LIB): {override}"
+    return None
+
+
+@pytest.fixture(autouse=True)
+def _no_oracle_override_under_gpu_parity(request):
+    """The GPU parity tests compare against the built oracle only: with
+    TFQ_ORACLE_LIB set (the mutation test's way of loading a planted
+    mistake) they fail instead of checking against another library."""
+    if request.node.get_closest_marker("gpu") is not None and os.environ.get("TFQ_ORACLE_LIB"):
+        pytest.fail("TFQ_ORACLE_LIB is set: GPU parity tests run only against the built oracle")

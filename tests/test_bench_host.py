@@ -189,3 +189,28 @@ def test_profile_commands_still_run_with_this_bench(monkeypatch):
             if argv is not None:
                 monkeypatch.setattr(sys, "argv", argv)
                 bench.parse_args()  # exits (SystemExit) on an option the bench no longer has
+
+
+def test_clock_normalised_fraction():
+    """achieved / (SMs x 16384 FLOP/clk x sampled MHz); absent without a clock."""
+    import bench
+    r = bench.clock_normalised(2900.0, {"sm_mhz": 1230}, 148)
+    peak = 148 * 16384 * 1230e6 / 1e12
+    assert abs(r["peak_at_clock"] - round(peak, 1)) < 1e-9
+    assert abs(r["frac"] - round(2900.0 / peak, 4)) < 1e-12
+    assert bench.clock_normalised(2900.0, {}, 148) is None
+    assert bench.clock_normalised(2900.0, {"sm_mhz": 1230}, None) is None
+
+
+@pytest.mark.parametrize("M", [75600, 6889, 32760, 512, 129, 1])
+def test_tile_sample_rows_hit_every_cta_share(M):
+    """The full-size parity sample holds a row of every 128-row CTA share of
+    M, the whole ragged last share, and the random rows."""
+    import numpy as np
+    from tests import _gpu
+    rows = _gpu.tile_sample_rows(M, seed=3)
+    assert rows.min() >= 0 and rows.max() < M and np.all(np.diff(rows) > 0)
+    assert set(range(M - (M % 128 or min(M, 128)), M)) <= set(rows.tolist())
+    assert len(rows) >= min(M, (M + 127) // 128 + 512) * 0.9
+    with pytest.raises(AssertionError):
+        _gpu.assert_covers_blocks(rows[rows >= 128], M) if M > 128 else _gpu.assert_covers_blocks(rows[:0], M)

@@ -95,7 +95,9 @@ def test_int8_linear_end_to_end():
 
 
 def test_int8_full_size_sampled():
-    """Video-DiT FFN-down at full size (75600 x 13824 -> 5120) through the INT8 path."""
+    """Video-DiT FFN-down at full size (75600 x 13824 -> 5120) through the
+    INT8 path; one row of every 128-row CTA share of every M tile, 512 more
+    seeded rows and the ragged tail, all N columns."""
     wl = workloads.VIDEO_DIT
     lin = [l for l in wl.linears if l.name == "ffn_down"][0]
     x = wl.make_x(lin.x, device="cuda")
@@ -104,7 +106,7 @@ def test_int8_full_size_sampled():
     A, sa = _quant_act_int8(x)
     Wq, sw = _gpu.quant_weight(w, _capi.TFQ_DTYPE_INT8, 127.0)
     y = _int8_linear(A, sa, Wq.view(torch.int8), sw, b)
-    rows = _gpu.sample_rows(wl.M, 64, seed=5)
+    rows = _gpu.tile_sample_rows(wl.M, seed=5)
     A_ref, sa_ref = _gpu.oracle_quant_int8(x, 127.0, rows)
     np.testing.assert_array_equal(A[torch.as_tensor(rows, device="cuda")].cpu().numpy(), A_ref)
     y_ref = oracle.scaled_int8_linear(A.cpu().numpy(), sa.cpu().numpy(), Wq.view(torch.int8).cpu().numpy(),

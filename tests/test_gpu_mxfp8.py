@@ -130,7 +130,8 @@ def test_quant_then_gemm_tiny_linear():
 def test_full_size_video_linears_sampled():
     """The video-DiT block's Linears in MXFP8 at full size: GPU quantizer
     (sampled rows checked bit-exact) and GPU GEMM (sampled rows within the
-    tolerance)."""
+    tolerance): one row of every 128-row CTA share of every M tile, 512 more
+    seeded rows and the ragged tail, all N columns."""
     wl = workloads.WORKLOADS["video_dit_block"]
     xs = {}
     for lin in wl.linears:
@@ -146,7 +147,7 @@ def test_full_size_video_linears_sampled():
         y = _capi.tfq_mxfp8_linear(A, sfa, W, sfw, b)
         torch.cuda.synchronize()
         _gpu.check_device_error()
-        rows = _gpu.sample_rows(M, 64, seed=lin.N + lin.K)
+        rows = _gpu.tile_sample_rows(M, seed=lin.N + lin.K)
         ridx = torch.as_tensor(rows, device="cuda")
         xr = x[ridx]
         q_ref, sf_ref = oracle.quant_mxfp8(_gpu.bf16_bits_np(xr))
