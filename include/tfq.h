@@ -56,6 +56,7 @@
 #ifndef TFQ_H_
 #define TFQ_H_
 
+#include <stddef.h>
 #include <stdint.h>
 
 #if defined(__GNUC__)
@@ -130,6 +131,45 @@ TFQ_API tfq_status tfq_quant_weight_per_channel(const void *w_bf16, int64_t N, i
 TFQ_API tfq_status tfq_scaled_fp8_linear(const void *A_q, const float *s_a, const void *W_q,
                                  const float *s_w, const void *bias_bf16, int64_t M, int64_t N,
                                  int64_t K, void *out_bf16, void *stream);
+
+/*
+ * Per-token FP8 quantization and the scaled FP8 Linear in one call: the
+ * LinearFP8 forward of the TeleFuser "Quantization" page (section "Scaled
+ * FP8 checkpoints: W8A8": quantize each input row dynamically, then run the
+ * scaled GEMM), with the per-token activation / per-output-channel weight
+ * scheme of its section "tf-kernel FP8: online W8A8".
+ *   x_bf16 : [M, K] bf16 activations, read only; qmax as in
+ *            tfq_quant_act_fp8_per_token.
+ *   W_q, s_w, bias_bf16, N : as in tfq_scaled_fp8_linear.
+ *   A_q : [M, K] bytes, written: the E4M3FN codes tfq_quant_act_fp8_per_token
+ *         writes (bit for bit); s_a : [M] fp32, written: its scales.
+ *   out_bf16 : [M, N] bf16, written: as tfq_scaled_fp8_linear(A_q, s_a, ...).
+ *   workspace : device memory of
+ *         tfq_quant_scaled_fp8_linear_workspace_bytes(M) bytes, owned by the
+ *         caller, 16-byte aligned; cleared by the call on `stream` (so calls
+ *         that overlap on the GPU need workspaces of their own).
+ * From M = 512 rows up one kernel does both: besides the GEMM's roles every
+ * CTA runs quantizer warps that quantize rows in increasing order ahead of
+ * the tiles that read them (each 128-row share is published through a
+ * counter in the workspace, and a CTA waits, bounded, for the shares it
+ * loads), so the HBM-bound quantization overlaps the tensor-bound GEMM.
+ * Below 512 rows it runs the row quantizer, then the GEMM.  A_q and s_a stay
+ * valid after the call (the other Linears of a shared input, such as K and V
+ * beside Q, can take them to tfq_scaled_fp8_linear).
+ * Measured on B200 the one-kernel form is not faster than the two calls
+ * tfq_quant_act_fp8_per_token + tfq_scaled_fp8_linear (the GEMM slows down by
+ * about the quantizer's time); those remain the recommended path, and this
+ * entry point is the measured alternative (same results, bit for bit).
+ * M == 0 is a no-op; N == 0 quantizes only.
+ * Errors: those of tfq_quant_act_fp8_per_token and tfq_scaled_fp8_linear,
+ * TFQ_EINVAL for a null or misaligned workspace; a bounded wait that runs
+ * out is reported by tfq_device_error() (TFQ_ETIMEOUT).
+ */
+TFQ_API size_t tfq_quant_scaled_fp8_linear_workspace_bytes(int64_t M);
+TFQ_API tfq_status tfq_quant_scaled_fp8_linear(const void *x_bf16, int64_t M, int64_t K, float qmax,
+                                               const void *W_q, const float *s_w, const void *bias_bf16,
+                                               int64_t N, void *A_q, float *s_a, void *out_bf16,
+                                               void *workspace, void *stream);
 
 /*
  * INT8 W8A8 (the int8 modes of the LightX2V "模型量化技术" page, quantization-

@@ -30,6 +30,8 @@ from ._capi import (  # noqa: F401
     tfq_quant_act_fp8_per_token,
     tfq_quant_act_int8_per_token,
     tfq_quant_mxfp8,
+    tfq_quant_scaled_fp8_linear,
+    tfq_quant_scaled_fp8_linear_workspace_bytes,
     tfq_quant_weight_per_channel,
     tfq_scaled_fp8_linear,
     tfq_scaled_fp8_linear_f16acc,
@@ -43,6 +45,8 @@ __all__ = [
     "tfq_quant_act_fp8_per_token",
     "tfq_quant_weight_per_channel",
     "tfq_scaled_fp8_linear",
+    "tfq_quant_scaled_fp8_linear",
+    "tfq_quant_scaled_fp8_linear_workspace_bytes",
     "tfq_scaled_fp8_linear_f16acc",
     "tfq_scaled_fp8_linear_noalloc",
     "tfq_quant_act_int8_per_token",

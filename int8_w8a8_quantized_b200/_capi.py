@@ -33,6 +33,8 @@ SIGNATURES = {
     "tfq_quant_act_fp8_per_token": (_I, [_P, _I64, _I64, _F, _P, _P, _P]),
     "tfq_quant_weight_per_channel": (_I, [_P, _I64, _I64, _I, _F, _P, _P, _P]),
     "tfq_scaled_fp8_linear": (_I, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _P]),
+    "tfq_quant_scaled_fp8_linear_workspace_bytes": (ctypes.c_size_t, [_I64]),
+    "tfq_quant_scaled_fp8_linear": (_I, [_P, _I64, _I64, _F, _P, _P, _P, _I64, _P, _P, _P, _P, _P]),
     "tfq_quant_act_int8_per_token": (_I, [_P, _I64, _I64, _F, _P, _P, _P]),
     "tfq_scaled_int8_linear": (_I, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _P]),
     "tfq_scaled_fp8_linear_f16acc": (_I, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _P]),
@@ -356,3 +358,53 @@ def w8a8_linear(x, W_q, s_w, bias=None, qmax: float = 448.0, stream=None):
     """The whole Linear: per-token FP8 quantization of x, then the scaled GEMM."""
     A_q, s_a = tfq_quant_act_fp8_per_token(x, qmax, stream=stream)
     return tfq_scaled_fp8_linear(A_q, s_a, W_q, s_w, bias, stream=stream)
+
+
+def tfq_quant_scaled_fp8_linear_workspace_bytes(M: int) -> int:
+    """Bytes of the workspace tfq_quant_scaled_fp8_linear needs for M rows."""
+    return int(load_library().tfq_quant_scaled_fp8_linear_workspace_bytes(int(M)))
+
+
+def tfq_quant_scaled_fp8_linear(x, W_q, s_w, bias=None, qmax: float = 448.0, A_q=None, s_a=None, out=None,
+                                workspace=None, stream=None):
+    """x bf16 [M, K], W_q uint8 [N, K], s_w fp32 [N], bias bf16 [N] or None ->
+    (out bf16 [M, N], A_q uint8 [M, K], s_a fp32 [M]): per-token FP8
+    quantization of x and the scaled GEMM in one call (one kernel from 512
+    rows up)."""
+    import torch
+    _require(x, torch.bfloat16, 2, "x")
+    dev = x.device
+    _require(W_q, torch.uint8, 2, "W_q", dev)
+    _require(s_w, torch.float32, 1, "s_w", dev)
+    M, K = x.shape
+    N, K2 = W_q.shape
+    if K2 != K or s_w.shape[0] != N:
+        raise ValueError("shape mismatch")
+    if bias is not None:
+        _require(bias, torch.bfloat16, 1, "bias", dev)
+        if bias.shape[0] != N:
+            raise ValueError("bias shape")
+    if A_q is None:
+        A_q = torch.empty((M, K), dtype=torch.uint8, device=dev)
+    if s_a is None:
+        s_a = torch.empty((M,), dtype=torch.float32, device=dev)
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    nws = tfq_quant_scaled_fp8_linear_workspace_bytes(M)
+    if workspace is None:
+        workspace = torch.empty((max(nws, 16),), dtype=torch.uint8, device=dev)
+    _require(A_q, torch.uint8, 2, "A_q", dev)
+    _require(s_a, torch.float32, 1, "s_a", dev)
+    _require(out, torch.bfloat16, 2, "out", dev)
+    _require(workspace, torch.uint8, 1, "workspace", dev)
+    if tuple(A_q.shape) != (M, K) or tuple(s_a.shape) != (M,) or tuple(out.shape) != (M, N):
+        raise ValueError("output shapes do not match x and W_q")
+    if workspace.numel() < nws:
+        raise ValueError(f"workspace holds {workspace.numel()} bytes, {nws} needed")
+    with torch.cuda.device(dev):
+        st = raw.tfq_quant_scaled_fp8_linear(x.data_ptr(), M, K, float(qmax), W_q.data_ptr(), s_w.data_ptr(),
+                                             None if bias is None else bias.data_ptr(), N, A_q.data_ptr(),
+                                             s_a.data_ptr(), out.data_ptr(), workspace.data_ptr(),
+                                             _stream_handle(stream))
+    _check(st, "tfq_quant_scaled_fp8_linear")
+    return out, A_q, s_a

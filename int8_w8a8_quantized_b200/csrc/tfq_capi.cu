@@ -280,6 +280,25 @@ tfq_status tfq_scaled_fp8_linear(const void* A_q, const float* s_a, const void* 
                                   static_cast<cudaStream_t>(stream), ds);
 }
 
+size_t tfq_quant_scaled_fp8_linear_workspace_bytes(int64_t M) {
+    return M < 0 ? 0 : quant_gemm_workspace_bytes(M);
+}
+
+tfq_status tfq_quant_scaled_fp8_linear(const void* x_bf16, int64_t M, int64_t K, float qmax, const void* W_q,
+                                       const float* s_w, const void* bias_bf16, int64_t N, void* A_q, float* s_a,
+                                       void* out_bf16, void* workspace, void* stream) {
+    tfq_status st = check_quant_args(x_bf16, M, K, A_q, s_a, qmax, 448.0f);
+    if (st != TFQ_OK) return st;
+    st = check_gemm_args(A_q, s_a, W_q, s_w, bias_bf16, M, N, K, out_bf16);
+    if (st != TFQ_OK || M == 0) return st;
+    if (workspace == nullptr || !aligned16(workspace))
+        return fail(TFQ_EINVAL, "workspace null or not 16-byte aligned");
+    DeviceState* ds = current_device_state(&st);
+    if (ds == nullptr) return st;
+    return launch_quant_scaled_fp8_gemm(x_bf16, M, K, qmax, !is_e4m3_value(qmax), W_q, s_w, bias_bf16, N, A_q, s_a,
+                                        out_bf16, workspace, static_cast<cudaStream_t>(stream), ds);
+}
+
 tfq_status tfq_selftest_div_rn(const float* a, const float* b, int64_t n, float* ours, float* ieee,
                                void* stream) {
     if (n < 0) return fail(TFQ_EINVAL, "negative n");

@@ -84,6 +84,18 @@ struct GemmArgs {
     // half-width tiles (PBN / 2 columns, two clusters each), so that the
     // round takes about half a tile's time instead of a whole one.
     int tail_halves = 0;
+    // The CTA-pair kernel that quantizes its own activations (null qx
+    // otherwise): its quantizer warps turn bf16 rows of qx [M, K] into E4M3
+    // codes qa [M, K] (the A operand its TMA loads read) and scales qs [M]
+    // (= s_a), taking rows in increasing order from *q_next_row; each row
+    // done adds one to q_share_rows[row / 128].  A CTA loads rows of A, and
+    // reads their scales, only once their 128-row share is complete.
+    const uint4* qx = nullptr;
+    uint8_t* qa = nullptr;
+    float* qs = nullptr;
+    unsigned* q_next_row = nullptr;
+    unsigned* q_share_rows = nullptr;
+    float qmax = 0.0f;
 };
 
 #ifndef TFQ_PACING_WAIT_NS

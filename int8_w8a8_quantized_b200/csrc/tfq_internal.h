@@ -35,7 +35,8 @@ struct DeviceState {
     unsigned* round_ctrs = nullptr;
     int round_slots = 0;
     int next_round_slot = 0;
-    bool gemm_attr_set[5] = {false, false, false, false, false};  // FP8, INT8, FP8/FP16 acc, MXFP8, MXFP8 pair
+    // FP8, INT8, FP8/FP16 acc, MXFP8, MXFP8 pair, FP8 pair quantizing its activations
+    bool gemm_attr_set[6] = {false, false, false, false, false, false};
     bool quant_attr_set = false;   // dynamic shared memory limit of the staged-row quantizers
 };
 
@@ -80,6 +81,12 @@ tfq_status encode_tensor_map_2d(CUtensorMap* map, CUtensorMapDataType dtype, con
                                 uint64_t outer, uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer,
                                 CUtensorMapSwizzle swizzle);
 
+// True when v is exactly representable in E4M3FN (at most 4 significant bits,
+// within the normal range used for qmax): then an FP8 quantizer needs no
+// clamp to +-qmax (x / s exceeds qmax by at most one rounding, which encodes
+// like qmax).
+bool is_e4m3_value(float v);
+
 // Row quantizer: out_int8 == false -> E4M3FN codes, true -> INT8 codes.
 tfq_status launch_quant_rows(const void* x, int64_t rows, int64_t K, float qmax, bool out_int8, void* q, float* s,
                              cudaStream_t stream, DeviceState* ds);
@@ -102,6 +109,19 @@ unsigned* take_round_counter(DeviceState* ds);
 tfq_status launch_scaled_fp8_gemm(const void* A, const float* s_a, const void* W, const float* s_w,
                                   const void* bias, int64_t M, int64_t N, int64_t K, void* out,
                                   cudaStream_t stream, DeviceState* ds);
+
+// Bytes of the workspace of launch_quant_scaled_fp8_gemm for M rows.
+size_t quant_gemm_workspace_bytes(int64_t M);
+
+// Per-token FP8 quantization of x [M, K] into A (codes) and s_a (scales)
+// and the scaled FP8 GEMM on them, in one kernel from M = 512 rows up (its
+// quantizer warps overlap the quantization with the MMAs; `workspace`
+// holds its row counters and is cleared on `stream` first), as the row
+// quantizer followed by the GEMM below that.  clamp: qmax is not an E4M3
+// value.
+tfq_status launch_quant_scaled_fp8_gemm(const void* x, int64_t M, int64_t K, float qmax, bool clamp, const void* W,
+                                        const float* s_w, const void* bias, int64_t N, void* A, float* s_a,
+                                        void* out, void* workspace, cudaStream_t stream, DeviceState* ds);
 
 // Scaled FP8 GEMM with a half-precision (FP16) accumulator.
 tfq_status launch_scaled_fp8_gemm_f16acc(const void* A, const float* s_a, const void* W, const float* s_w,

@@ -230,3 +230,42 @@ def test_smoke_without_gpu_raises(lib):
     import __graft_entry__
     with pytest.raises(RuntimeError, match="CUDA device"):
         __graft_entry__.smoke()
+
+
+def test_quant_scaled_linear_workspace_bytes(lib):
+    """Two 128-byte lines of counters (the next row to quantize) plus one word
+    per 128-row share of M, in whole 256-byte blocks."""
+    f = lib.tfq_quant_scaled_fp8_linear_workspace_bytes
+    for M in (1, 128, 129, 512, 6889, 75600, (1 << 31) - 1):
+        n = f(M)
+        assert n % 256 == 0 and n >= 4 * (32 + (M + 127) // 128) and n < 4 * (32 + (M + 127) // 128) + 256
+    assert f(0) == 256 and f(-1) == 0
+
+
+def _fused(lib, x=ALIGNED, M=1024, K=256, qmax=448.0, W=ALIGNED, sw=ALIGNED, b=None, N=256, A=ALIGNED,
+           sa=ALIGNED, out=ALIGNED, ws=ALIGNED):
+    return lib.tfq_quant_scaled_fp8_linear(x, M, K, qmax, W, sw, b, N, A, sa, out, ws, None)
+
+
+def test_quant_scaled_linear_validation(lib):
+    """The fused entry point checks the quantizer's and the GEMM's arguments
+    and its workspace on the host, before any device work."""
+    assert _fused(lib, K=24) == _capi.TFQ_EINVAL                      # K % 16
+    assert _fused(lib, qmax=449.0) == _capi.TFQ_EINVAL
+    assert _fused(lib, qmax=0.5) == _capi.TFQ_EINVAL
+    assert _fused(lib, N=12) == _capi.TFQ_EINVAL                      # N % 8
+    assert _fused(lib, x=None) == _capi.TFQ_EINVAL
+    assert _fused(lib, W=None) == _capi.TFQ_EINVAL
+    assert _fused(lib, sa=ALIGNED + 4) == _capi.TFQ_EINVAL
+    assert _fused(lib, out=ALIGNED + 2) == _capi.TFQ_EINVAL
+    assert _fused(lib, b=ALIGNED + 8) == _capi.TFQ_EINVAL
+    assert _fused(lib, ws=None) == _capi.TFQ_EINVAL
+    assert _fused(lib, ws=ALIGNED + 4) == _capi.TFQ_EINVAL
+    assert _fused(lib, M=-1) == _capi.TFQ_EINVAL
+    assert _fused(lib, M=1 << 31) == _capi.TFQ_EUNSUPPORTED
+    assert _fused(lib, M=0, x=None, W=None, sw=None, A=None, sa=None, out=None, ws=None) == _capi.TFQ_OK
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU behaviour")
+def test_quant_scaled_linear_without_gpu_fails_loudly(lib):
+    assert _fused(lib) in (_capi.TFQ_ECUDA, _capi.TFQ_EUNSUPPORTED)
