@@ -70,6 +70,9 @@ def parse_args():
     ap.add_argument("--fused", action="store_true",
                     help="fp8 only: the first Linear of each activation quantizes it inside its GEMM "
                          "(tfq_quant_scaled_fp8_linear: one kernel); the other Linears of that input take its codes")
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="run the workload's Linears over this many tokens instead of its M (for ncu captures on "
+                         "a reduced case; never a benchmark figure)")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -1089,6 +1092,9 @@ def main():
     if args.workload == "activation_quantizer":
         return quantizer_main(args, rank, world, local_rank)
     wl = workloads.WORKLOADS[args.workload]
+    if args.tokens:
+        import dataclasses
+        wl = dataclasses.replace(wl, M=args.tokens)
     if args.fused and args.dtype != "fp8":
         raise SystemExit("--fused takes --dtype fp8")
     cfg = {"workload": wl.name, "M": wl.M, "dtype": args.dtype,
@@ -1101,6 +1107,8 @@ def main():
            "parallelism": f"replicas x{world}"}
     if args.fused:
         cfg["quantization"] = "inside the first GEMM of each activation (one kernel per Linear)"
+    if args.tokens:
+        cfg["reduced_tokens"] = f"M = {args.tokens} instead of the workload's M (a profiling case, not a benchmark)"
 
     if args.impl == "reference":
         if rank != 0:

@@ -24,6 +24,10 @@ What each function follows (page titles and sections of the source pages):
 * ``scaled_int8_linear``: the INT8 W8A8 modes of LightX2V "模型量化技术",
   quantization-mode table (INT8 per-channel weights, dynamic per-token INT8
   activations), exact int64 sums.
+* ``fp8_block_prefix_sums``: the running sums of the FP8 GEMM at every
+  32-element block of K (their final value and largest magnitude), for the
+  FP16-accumulator study of LightX2V "模型量化技术", "MiniMax-H3 FP8 FP16
+  累加" (FP16 partial sums overflow at qmax 14 and 12, not at 7).
 * ``quant_mxfp8`` / ``mxfp8_linear``: MXFP8 as named on the TeleFuser
   "Quantization" page, "Offline conversion" (32-value blocks, E8M0 scales),
   with the conversion of the OCP Microscaling (MX) v1.0 specification; the
@@ -93,6 +97,8 @@ def _load():
                 fn = getattr(lib, name)
                 fn.restype = None
                 fn.argtypes = [P, P, P, P, P, I64, I64, I64, P, I64, P]
+            lib.tfq_oracle_fp8_block_prefix_sums.restype = None
+            lib.tfq_oracle_fp8_block_prefix_sums.argtypes = [P, P, I64, I64, I64, I64, P, I64, P, P]
             lib.tfq_oracle_quant_mxfp8.restype = None
             lib.tfq_oracle_quant_mxfp8.argtypes = [P, I64, I64, P, P]
             lib.tfq_oracle_mxfp8_linear.restype = None
@@ -204,6 +210,32 @@ def scaled_int8_linear(A, s_a, W, s_w, bias_bits=None, rows=None) -> np.ndarray:
     """y[i,n] = sum_k A[m,k] W[n,k] * s_a[m] * s_w[n] + bias[n] (double)."""
     return _linear(_load().tfq_oracle_scaled_int8_linear, A, s_a, W, s_w,
                    bias_bits, rows, np.int8)
+
+
+def fp8_block_prefix_sums(A, W, block: int = 32, rows=None):
+    """The FP8 GEMM's running sums at every `block`-element boundary of K:
+    (final [rows, N] = sum_k dec(A) dec(W), prefix_max [rows, N] = the largest
+    |running sum| at a block boundary), exact, no scales or bias.  For the
+    FP16-accumulator study of LightX2V "模型量化技术", "MiniMax-H3 FP8 FP16
+    累加"."""
+    A = np.ascontiguousarray(A, dtype=np.uint8)
+    W = np.ascontiguousarray(W, dtype=np.uint8)
+    M, K = A.shape
+    N, K2 = W.shape
+    if K2 != K or block < 1:
+        raise ValueError("shape mismatch")
+    r = None
+    nrows = M
+    if rows is not None:
+        r = np.ascontiguousarray(rows, dtype=np.int64)
+        if r.size and (r.min() < 0 or r.max() >= M):
+            raise ValueError("row index out of range")
+        nrows = r.size
+    final = np.empty((nrows, N), dtype=np.float64)
+    pmax = np.empty((nrows, N), dtype=np.float64)
+    _load().tfq_oracle_fp8_block_prefix_sums(_ptr(A), _ptr(W), M, N, K, int(block), _ptr(r), nrows, _ptr(final),
+                                             _ptr(pmax))
+    return final, pmax
 
 
 def quant_mxfp8(x_bits):

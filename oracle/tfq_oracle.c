@@ -277,6 +277,53 @@ void tfq_oracle_scaled_int8_linear(const int8_t *A, const float *s_a,
     }
 }
 
+/*
+ * Block prefix sums of the FP8 GEMM's accumulation, for the FP16-accumulator
+ * study (LightX2V "模型量化技术" page, section "MiniMax-H3 FP8 FP16 累加":
+ * with FP16 accumulation the partial sums of the FFN-out Linear overflow at
+ * qmax 14 and 12; qmax 7 keeps them in range).  For m = rows[i] (or i) and
+ * every n, with P_j = sum_{k < j * block} dec(A[m,k]) dec(W[n,k]) (exact in
+ * double, see above) and P_last the whole sum:
+ *   final[i, n]      = P_last,
+ *   prefix_max[i, n] = max |P_j| over j = 1 .. ceil(K / block) (the last
+ *                      block may be partial), i.e. the largest magnitude the
+ *                      running sum reaches at a block boundary.
+ * No scales, no bias: these are the accumulator's values.
+ */
+void tfq_oracle_fp8_block_prefix_sums(const uint8_t *A, const uint8_t *W,
+                                      int64_t M, int64_t N, int64_t K,
+                                      int64_t block, const int64_t *rows,
+                                      int64_t nrows, double *final_sum,
+                                      double *prefix_max)
+{
+    double dec[256];
+    int64_t i;
+    int c;
+    (void)M;
+    for (c = 0; c < 256; ++c)
+        dec[c] = tfq_oracle_e4m3_decode((uint8_t)c);
+#pragma omp parallel for schedule(dynamic, 1)
+    for (i = 0; i < nrows; ++i) {
+        int64_t m = rows ? rows[i] : i;
+        const uint8_t *a = A + m * K;
+        int64_t n;
+        for (n = 0; n < N; ++n) {
+            const uint8_t *w = W + n * K;
+            double acc = 0.0, pmax = 0.0;
+            int64_t k;
+            for (k = 0; k < K; ++k) {
+                acc = acc + dec[a[k]] * dec[w[k]];
+                if ((k + 1) % block == 0 || k + 1 == K) {
+                    if (fabs(acc) > pmax)
+                        pmax = fabs(acc);
+                }
+            }
+            final_sum[i * N + n] = acc;
+            prefix_max[i * N + n] = pmax;
+        }
+    }
+}
+
 /* ------------------------------------------------------------------ */
 /* MXFP8: E4M3 elements with one E8M0 (power-of-two) scale per block of */
 /* 32 consecutive values of a row.                                     */

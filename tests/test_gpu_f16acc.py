@@ -67,25 +67,62 @@ def test_error_within_fp16_accumulation_bound():
     assert np.all(np.abs(y - y_ref) <= bound)
 
 
+# The FP16 accumulator's reading (the pages do not fix the tensor cores'
+# accumulation granularity): the running sum is rounded to FP16 once per
+# 32-deep MMA step (the K of one kind::f8f6f4 instruction), the step's own
+# products summed without FP16 rounding.  FP16_EPS_PER_STEP is twice that
+# rounding's relative bound (2^-11), a margin for a step sum rounded to fp32
+# first.
+FP16_MAX = 65504.0
+FP16_EPS_PER_STEP = 2.0 ** -10
+
+
+def _overflow_verdicts(A, Wq, rows):
+    """For sampled rows: which outputs must stay finite and which must
+    overflow with an FP16 accumulator, from the oracle's exact running sums
+    at every 32-element block of K.  With n steps and eps = n *
+    FP16_EPS_PER_STEP, every accumulator value stays within |P_max| (1 + eps) /
+    (1 - eps) when no step overflowed (P_max the largest exact running sum
+    at a step boundary), so it cannot overflow if that is below FP16_MAX;
+    and a final exact sum beyond FP16_MAX (1 + eps) cannot be reached without
+    an overflow, after which the sum stays infinite (or NaN)."""
+    K = A.shape[1]
+    final, pmax = oracle.fp8_block_prefix_sums(A.cpu().numpy(), Wq.cpu().numpy(), 32, rows=rows)
+    eps = -(-K // 32) * FP16_EPS_PER_STEP
+    must_finite = pmax * (1 + eps) / (1 - eps) < FP16_MAX
+    must_overflow = np.abs(final) > FP16_MAX * (1 + eps)
+    return must_finite, must_overflow
+
+
 def test_reduced_qmax_overflow_study(capsys):
     """FFN-out-like Linear (K = 13824 -> N = 5120, X = 4 Student-t(3), FP8
     weights at qmax 448): the fraction of non-finite outputs with an FP16
     accumulator as the activation qmax goes down.  It must fall to zero by
     qmax 7, never rise as qmax decreases, and the FP32-accumulator path must
-    stay finite throughout."""
+    stay finite throughout.  On 48 sampled rows (all N) every output the
+    oracle's running sums say must stay finite is finite, and every output
+    they say must overflow is not (see _overflow_verdicts)."""
     M, K, N = 2048, 13824, 5120
     x = workloads.activations(M, K, seed=41, nu=3, amplitude=4.0, device="cuda")
     w = workloads.weights(N, K, seed=42, std=0.015, device="cuda")
     Wq, sw = _gpu.quant_weight(w, _capi.TFQ_DTYPE_FP8_E4M3, 448.0)
-    fracs = {}
+    rows = _gpu.sample_rows(M, 47, seed=43)
+    ridx = torch.as_tensor(rows, device="cuda")
+    fracs, decided = {}, {}
     for qmax in (448.0, 64.0, 21.0, 14.0, 12.0, 7.0):
         A, sa = _gpu.quant_act_fp8(x, qmax)
         y16 = _f16acc(A, sa, Wq, sw, None)
         fracs[qmax] = float((~torch.isfinite(y16.float())).float().mean())
         y32 = _gpu.scaled_linear(A, sa, Wq, sw, None)
         assert torch.isfinite(y32.float()).all()
+        must_finite, must_overflow = _overflow_verdicts(A, Wq, rows)
+        finite = torch.isfinite(y16[ridx].float()).cpu().numpy()
+        assert finite[must_finite].all(), f"qmax {qmax}: an output that cannot overflow is not finite"
+        assert not finite[must_overflow].any(), f"qmax {qmax}: an output that must overflow is finite"
+        decided[qmax] = (int(must_finite.sum()), int(must_overflow.sum()), int(finite.size))
     with capsys.disabled():
         print("\nFP16-accumulator non-finite fraction by activation qmax:", fracs)
+        print("sampled outputs (must stay finite, must overflow, total):", decided)
     qs = sorted(fracs, reverse=True)
     assert all(fracs[a] >= fracs[b] for a, b in zip(qs, qs[1:]))
     assert fracs[7.0] == 0.0 and fracs[448.0] > 0.0

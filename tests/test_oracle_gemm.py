@@ -119,3 +119,45 @@ def test_int8_bruteforce(M, N, K):
             exact = Fraction(acc) * Fraction(float(sa[m])) * Fraction(float(sw[n])) + _bf16_value(int(b[n]))
             mag = abs(acc * float(sa[m]) * float(sw[n])) + abs(float(_bf16_value(int(b[n]))))
             assert abs(Fraction(y[m, n]) - exact) <= Fraction(4 * 2.0 ** -53 * mag)
+
+
+@pytest.mark.parametrize("M,N,K,block", [(3, 4, 70, 32), (2, 5, 64, 32), (4, 3, 33, 16), (2, 2, 31, 32), (3, 3, 9, 1)])
+def test_block_prefix_sums_bruteforce(M, N, K, block):
+    """The FP16-accumulator study's oracle: the exact running sum at every
+    block boundary (a partial last block included), by exact rational
+    arithmetic over the independent E4M3 grid; the final sum and the largest
+    |running sum| at a boundary.  The codes are mostly large and of one
+    sign per row, so intermediate maxima exceed the final sum."""
+    rng = np.random.default_rng(M + 10 * N + 100 * K + block)
+    A = _rand_codes(rng, (M, K))
+    W = _rand_codes(rng, (N, K))
+    A[0, : K // 2] = 0x70          # a long positive run, then mixed: the peak lies inside
+    W[:, : K // 2] = 0x68
+    final, pmax = oracle.fp8_block_prefix_sums(A, W, block)
+    assert final.shape == (M, N) and pmax.shape == (M, N)
+    for m in range(M):
+        for n in range(N):
+            acc, peak = Fraction(0), Fraction(0)
+            for k in range(K):
+                acc += _e4m3_value(int(A[m, k])) * _e4m3_value(int(W[n, k]))
+                if (k + 1) % block == 0 or k + 1 == K:
+                    peak = max(peak, abs(acc))
+            assert Fraction(final[m, n]) == acc
+            assert Fraction(pmax[m, n]) == peak
+    rows = np.array([M - 1, 0])
+    f2, p2 = oracle.fp8_block_prefix_sums(A, W, block, rows=rows)
+    np.testing.assert_array_equal(f2, final[rows])
+    np.testing.assert_array_equal(p2, pmax[rows])
+
+
+def test_block_prefix_max_is_not_the_final_sum():
+    """A sum that climbs to 16 * 448^2 and comes back to zero: the running
+    maximum at block boundaries (block 16) is the peak, the final sum 0."""
+    K = 32
+    A = np.full((1, K), 0x7E, dtype=np.uint8)           # 448
+    W = np.full((1, K), 0x7E, dtype=np.uint8)
+    W[0, 16:] = 0xFE                                     # -448
+    final, pmax = oracle.fp8_block_prefix_sums(A, W, 16)
+    assert final[0, 0] == 0.0 and pmax[0, 0] == 16 * 448.0 ** 2
+    final, pmax = oracle.fp8_block_prefix_sums(A, W, 32)
+    assert final[0, 0] == 0.0 and pmax[0, 0] == 0.0

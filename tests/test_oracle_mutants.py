@@ -30,6 +30,13 @@ PIN_FILES = ["tests/test_oracle_e4m3.py", "tests/test_oracle_quant.py",
 
 # name -> [(text in tfq_oracle.c, replacement)]; each text occurs exactly once.
 MUTANTS = {
+    # block prefix sums (FP16-accumulator study)
+    "block_prefix_signed_max": [("if (fabs(acc) > pmax)\n                        pmax = fabs(acc);",
+                                 "if (acc > pmax)\n                        pmax = acc;")],
+    "block_prefix_boundary_off_by_one": [("if ((k + 1) % block == 0 || k + 1 == K) {",
+                                          "if (k % block == 0 || k + 1 == K) {")],
+    "block_prefix_no_partial_last_block": [("if ((k + 1) % block == 0 || k + 1 == K) {",
+                                            "if ((k + 1) % block == 0) {")],
     # E4M3FN decoding
     "decode_subnormal_exponent": [("mag = ldexp((double)m, -9);", "mag = ldexp((double)m, -10);")],
     "decode_exponent_bias": [("ldexp((double)(8 + m), e - 10)", "ldexp((double)(8 + m), e - 9)")],
