@@ -30,11 +30,12 @@ def _lib():
     _gpu.lib()
 
 
-@pytest.mark.parametrize("M,N,K", [(130, 264, 2048), (777, 520, 1024), (2523, 1992, 256)])
+@pytest.mark.parametrize("M,N,K", [(130, 264, 2048), (777, 520, 1024), (2523, 1992, 256), (9400, 1000, 400)])
 def test_integer_sums_are_exact(M, N, K):
     """Codes of +-1 and 0: every partial sum is an integer of magnitude <= K <=
     2048, exact in FP16, so the result matches the oracle to bf16 rounding
-    (the last shape runs the pair kernel with its last round split)."""
+    (the third shape runs the pair kernel with its last round split, the
+    last two full rounds of pair tiles with ragged M, N and K)."""
     g = torch.Generator().manual_seed(M + N)
     choice = torch.tensor([0x38, 0xB8, 0x00], dtype=torch.uint8)
     A = choice[torch.randint(0, 3, (M, K), generator=g)]

@@ -220,3 +220,27 @@ def test_long_k_full_compare(M, N, K):
     phases wrap many times within one tile; K = 32784 leaves a 16-element
     K tail; one-CTA and pair kernels; full compare."""
     _run_case(M, N, K, True, seed=M + N + K)
+
+
+# Large pair-kernel shapes, one row of every 128-row CTA share compared: 148
+# tiles (two rounds) with 2 K blocks; ragged M, N (the last N tile 232
+# columns wide) and K; 444 tiles (six rounds) with a single K block; 592
+# tiles (eight rounds) with 8 K blocks.
+LARGE_SHAPES = [(9472, 1024, 256), (9400, 1000, 400), (18944, 1536, 128), (9472, 4096, 1024)]
+
+
+@pytest.mark.parametrize("M,N,K", LARGE_SHAPES)
+def test_pair_kernel_large_sampled(M, N, K):
+    """One row of every 128-row CTA share, 512 more seeded rows and the
+    ragged tail, all N columns, against the oracle."""
+    g = torch.Generator().manual_seed(M + N + K)
+    A = _rand_codes(g, (M, K))
+    W = _rand_codes(g, (N, K))
+    sa = (torch.rand(M, generator=g) * 0.01 + 1e-4).float()
+    sw = (torch.rand(N, generator=g) * 0.01 + 1e-4).float()
+    bias = (torch.randn(N, generator=g) * 0.5).to(torch.bfloat16)
+    y = _gpu.scaled_linear(A.cuda(), sa.cuda(), W.cuda(), sw.cuda(), bias.cuda())
+    rows = _gpu.tile_sample_rows(M, seed=M + K)
+    y_ref = oracle.scaled_fp8_linear(A.numpy(), sa.numpy(), W.numpy(), sw.numpy(), _gpu.bf16_bits_np(bias),
+                                     rows=rows)
+    _gpu.gemm_tolerance_check(y[torch.as_tensor(rows, device="cuda")], y_ref, f"M={M} N={N} K={K}")

@@ -157,3 +157,9 @@ def test_int8_rounding_edges(K):
 def test_int8_split_last_round(M, N, K):
     """The INT8 pair kernel with its last round split into half-width tiles."""
     _case(M, N, K, True, seed=M + 5 * N + K)
+
+
+@pytest.mark.parametrize("M,N,K", [(9400, 1000, 400), (18944, 1536, 128)])
+def test_int8_pair_kernel_large(M, N, K):
+    """The INT8 pair kernel on a ragged 148-tile shape and a 444-tile one (six rounds)."""
+    _case(M, N, K, True, seed=M + 3 * N + K)
