@@ -214,3 +214,21 @@ def test_tile_sample_rows_hit_every_cta_share(M):
     assert len(rows) >= min(M, (M + 127) // 128 + 512) * 0.9
     with pytest.raises(AssertionError):
         _gpu.assert_covers_blocks(rows[rows >= 128], M) if M > 128 else _gpu.assert_covers_blocks(rows[:0], M)
+
+
+def test_path_roofline_overlapped_floor():
+    """A launch that quantizes inside its GEMM is floored at max(FLOPs / peak,
+    (GEMM + quantizer bytes) / HBM); the serialized floor adds the quantizer's
+    bytes / HBM to the GEMM's floor."""
+    import bench
+    hbm = 6543.1
+    peaks = {"hbm_gbs": hbm}
+    F, G, Q = 4e12, 1.2e9, 1.16e9
+    res = {"ms_per_step": 2.0, "step_quant_bytes": [Q], "step_gemm_flops": [F, F], "step_gemm_bytes": [G, G],
+           "step_ops": [("fused", F, G, Q), ("gemm", F, G, 0)]}
+    out = bench.path_roofline(res, 1, peaks, 2800.0)
+    t = lambda f, b: max(f / 2800e12, b / (hbm * 1e9))
+    assert abs(out["floor_ms_measured_peaks"] - round(1e3 * (Q / (hbm * 1e9) + 2 * t(F, G)), 4)) < 1e-9
+    assert abs(out["overlapped"]["floor_ms_measured_peaks"] - round(1e3 * (t(F, G + Q) + t(F, G)), 4)) < 1e-9
+    res["step_ops"] = [("quant", 0, 0, Q), ("gemm", F, G, 0), ("gemm", F, G, 0)]
+    assert "overlapped" not in bench.path_roofline(res, 1, peaks, 2800.0)
