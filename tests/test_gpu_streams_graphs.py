@@ -165,3 +165,69 @@ def test_pacing_slots_reused_eager_and_in_a_graph():
         torch.cuda.synchronize()
         assert torch.equal(yg, ref)
     _gpu.check_device_error()
+
+
+def test_one_call_quant_linear_graph_and_concurrent_streams():
+    """The one-call quantization + GEMM (its workspace clear and its kernel)
+    captured into a CUDA graph replays to the eager result on new inputs; two
+    calls with workspaces of their own run concurrently on two streams and give
+    the results of the same calls run one after the other."""
+    lib = _gpu.lib()
+    cases = []
+    for i, (M, K, N) in enumerate([(2600, 1024, 1032), (1800, 3072, 776)]):
+        x = workloads.activations(M, K, seed=30 + i, outlier_cols=8, outlier_mult=20.0, device="cuda")
+        w = workloads.weights(N, K, seed=40 + i, std=0.02, device="cuda")
+        b = workloads.bias(N, seed=50 + i, device="cuda")
+        Wq, sw = _gpu.quant_weight(w, _capi.TFQ_DTYPE_FP8_E4M3, 448.0)
+        A = torch.empty((M, K), dtype=torch.uint8, device="cuda")
+        sa = torch.empty(M, device="cuda")
+        y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+        ws = torch.empty(lib.tfq_quant_scaled_fp8_linear_workspace_bytes(M), dtype=torch.uint8, device="cuda")
+        cases.append((x, Wq, sw, b, A, sa, y, ws))
+
+    def call(c, stream):
+        x, Wq, sw, b, A, sa, y, ws = c
+        M, K = x.shape
+        st = lib.tfq_quant_scaled_fp8_linear(x.data_ptr(), M, K, 448.0, Wq.data_ptr(), sw.data_ptr(), b.data_ptr(),
+                                             Wq.shape[0], A.data_ptr(), sa.data_ptr(), y.data_ptr(), ws.data_ptr(),
+                                             int(stream.cuda_stream))
+        assert st == _capi.TFQ_OK, _capi.last_error_message()
+
+    main = torch.cuda.current_stream()
+    for c in cases:
+        call(c, main)
+    torch.cuda.synchronize()
+    serial = [c[6].clone() for c in cases]
+    # concurrent streams, a workspace each
+    streams = [torch.cuda.Stream() for _ in cases]
+    for _ in range(3):
+        for c in cases:
+            c[6].zero_()
+        for c, s in zip(cases, streams):
+            s.wait_stream(main)
+            call(c, s)
+        for s in streams:
+            main.wait_stream(s)
+        torch.cuda.synchronize()
+        for c, ref in zip(cases, serial):
+            assert torch.equal(c[6], ref)
+    # graph capture of the first call, replayed on new inputs
+    c = cases[0]
+    graph = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream()
+    side.wait_stream(main)
+    with torch.cuda.stream(side):
+        with torch.cuda.graph(graph, stream=side):
+            call(c, side)
+    main.wait_stream(side)
+    M, K = c[0].shape
+    for seed in (60, 61):
+        c[0].copy_(workloads.activations(M, K, seed=seed, nu=4, device="cuda"))
+        graph.replay()
+        torch.cuda.synchronize()
+        y_graph = c[6].clone()
+        call(c, main)
+        torch.cuda.synchronize()
+        assert torch.equal(y_graph, c[6])
+    del graph
+    _gpu.check_device_error()
