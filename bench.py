@@ -768,16 +768,28 @@ def cpu_baseline(wl, seconds, dtype="fp8", single_thread_seconds=None):
 FP8_FLOP_PER_CLK_PER_SM = 16384
 
 
-def clock_normalised(achieved_tflops, clocks, sm_count):
+# Below this many milliseconds of timed region the sampled clock is not the
+# clock the kernels ran at: the power limiter acts on a comparable time scale
+# and the 10 ms sampler takes only a few samples.
+SHORT_REGION_MS = 250.0
+
+
+def clock_normalised(achieved_tflops, clocks, sm_count, region_ms=None):
     """The GEMM's rate against the tensor-core peak at the SM clock sampled
     during the timed region (SMs x 16384 FLOP/clk x median MHz): comparable
-    between boxes whose power-capped clocks differ."""
+    between boxes whose power-capped clocks differ.  Flagged unreliable when
+    the timed region is shorter than SHORT_REGION_MS."""
     mhz = (clocks or {}).get("sm_mhz")
     if not mhz or not sm_count:
         return None
     peak = sm_count * FP8_FLOP_PER_CLK_PER_SM * mhz * 1e6 / 1e12
-    return {"frac": round(achieved_tflops / peak, 4), "peak_at_clock": round(peak, 1), "sm_mhz": mhz,
-            "sm_count": sm_count, "flop_per_clk_per_sm": FP8_FLOP_PER_CLK_PER_SM}
+    out = {"frac": round(achieved_tflops / peak, 4), "peak_at_clock": round(peak, 1), "sm_mhz": mhz,
+           "sm_count": sm_count, "flop_per_clk_per_sm": FP8_FLOP_PER_CLK_PER_SM}
+    if region_ms is not None and region_ms < SHORT_REGION_MS:
+        out["reliable"] = False
+        out["note"] = (f"timed region {region_ms:.0f} ms: too short for the sampled clock to be the clock the "
+                       f"kernels ran at; run more --steps")
+    return out
 
 
 def path_roofline(res, steps, peaks, fp8_peak):
@@ -1191,7 +1203,8 @@ def main():
             "frac_of_burst_peak": round(gemm_tflops / (bf16_burst * FP8_OVER_BF16), 4),
             "avg_launch_ms": round(gemm_avg_ms, 4),
             "frac_of_fp8_spec": round(gemm_tflops / FP8_SPEC_TFLOPS, 4),
-            "clock_normalised": clock_normalised(gemm_tflops, res["clocks"], res.get("sm_count")),
+            "clock_normalised": clock_normalised(gemm_tflops, res["clocks"], res.get("sm_count"),
+                                                 res["ms_per_step"] * args.steps),
         },
         "quantizer": {"inside": "the fused launches quantize their activations (quantizer warps of the GEMM "
                                 "kernel); no quantizer launch of its own"} if fused else {

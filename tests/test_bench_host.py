@@ -232,3 +232,10 @@ def test_path_roofline_overlapped_floor():
     assert abs(out["overlapped"]["floor_ms_measured_peaks"] - round(1e3 * (t(F, G + Q) + t(F, G)), 4)) < 1e-9
     res["step_ops"] = [("quant", 0, 0, Q), ("gemm", F, G, 0), ("gemm", F, G, 0)]
     assert "overlapped" not in bench.path_roofline(res, 1, peaks, 2800.0)
+
+
+def test_clock_normalised_flags_short_regions():
+    import bench
+    r = bench.clock_normalised(2900.0, {"sm_mhz": 1965}, 148, region_ms=20.0)
+    assert r["reliable"] is False and "too short" in r["note"]
+    assert "reliable" not in bench.clock_normalised(2900.0, {"sm_mhz": 1230}, 148, region_ms=450.0)
