@@ -399,21 +399,21 @@ def gpu_arm(args, wl, rank, world, local_rank):
     wss = {name: torch.empty(lib.tfq_quant_scaled_fp8_linear_workspace_bytes(x.shape[0]), dtype=torch.uint8,
                              device=dev) for name, x in xs.items()} if fused else {}
     ops = []
+    # Block order, as a LinearFP8 forward runs: each activation is quantized
+    # directly before the first Linear that reads it (Q, K and V share theirs).
     for q in qmaxes:
-        if not fused:
-            for name, x in xs.items():
-                A, sa = aq[(name, q)]
-                ops.append(("quant",
-                            lambda x=x, q=q, A=A, sa=sa: quant_fn(x.data_ptr(), x.shape[0], x.shape[1], float(q),
-                                                                  A.data_ptr(), sa.data_ptr(), sh),
-                            3 * x.numel() + (x.numel() // 32 if mx else 4 * x.shape[0])))
         seen = set()
         for lin, Wq, sw, b in lins:
             A, sa = aq[(lin.x, q)]
             y = ys[(lin.name, q)]
             bp = None if b is None else b.data_ptr()
+            if not fused and lin.x not in seen:
+                x = xs[lin.x]
+                ops.append(("quant",
+                            lambda x=x, q=q, A=A, sa=sa: quant_fn(x.data_ptr(), x.shape[0], x.shape[1], float(q),
+                                                                  A.data_ptr(), sa.data_ptr(), sh),
+                            3 * x.numel() + (x.numel() // 32 if mx else 4 * x.shape[0])))
             if fused and lin.x not in seen:
-                seen.add(lin.x)
                 x = xs[lin.x]
                 ops.append(("fused",
                             lambda x=x, q=q, Wq=Wq, sw=sw, bp=bp, lin=lin, A=A, sa=sa, y=y, ws=wss[lin.x]:
@@ -427,6 +427,7 @@ def gpu_arm(args, wl, rank, world, local_rank):
                             gemm_fn(A.data_ptr(), sa.data_ptr(), Wq.data_ptr(), sw.data_ptr(), bp, wl.M, lin.N,
                                     lin.K, y.data_ptr(), sh),
                             (wl.M, lin.N, lin.K)))
+            seen.add(lin.x)
     n_kernels = len(ops)
 
     def step(record, which=None):
