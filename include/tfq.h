@@ -132,6 +132,29 @@ TFQ_API tfq_status tfq_scaled_fp8_linear(const void *A_q, const float *s_a, cons
                                  const float *s_w, const void *bias_bf16, int64_t M, int64_t N,
                                  int64_t K, void *out_bf16, void *stream);
 
+/* Most Linears tfq_scaled_fp8_linear_multi takes in one call. */
+#define TFQ_MULTI_MAX_LINEARS 4
+
+/*
+ * Scaled FP8 Linears that share their input: out[i] = the result of
+ * tfq_scaled_fp8_linear(A_q, s_a, W_q[i], s_w[i], bias_bf16[i], M, N[i], K,
+ * out[i]) for i < n, 1 <= n <= TFQ_MULTI_MAX_LINEARS -- such as the Q, K and
+ * V projections of a DiT block, which read one normed input (the per-token
+ * quantized activations A_q, s_a).  The arrays are host arrays of n entries;
+ * bias_bf16 may be NULL (no bias for any Linear), and so may any
+ * bias_bf16[i].  From M = 512 rows up the n GEMMs run as one launch of the
+ * CTA-pair kernel, their N tiles concatenated, which saves the fixed costs
+ * of n - 1 launches (ramp-up, drain, a partial last round); the results are
+ * the same, bit for bit, as those of the n separate calls.  Each N[i] follows
+ * the rules of tfq_scaled_fp8_linear (N[i] == 0 skips that Linear).
+ * Errors: those of tfq_scaled_fp8_linear for any Linear, TFQ_EINVAL for n out
+ * of range or a null array.
+ */
+TFQ_API tfq_status tfq_scaled_fp8_linear_multi(const void *A_q, const float *s_a, int64_t M, int64_t K, int n,
+                                               const void *const *W_q, const float *const *s_w,
+                                               const void *const *bias_bf16, const int64_t *N,
+                                               void *const *out_bf16, void *stream);
+
 /*
  * Per-token FP8 quantization and the scaled FP8 Linear in one call: the
  * LinearFP8 forward of the TeleFuser "Quantization" page (section "Scaled

@@ -35,6 +35,7 @@ from ._capi import (  # noqa: F401
     tfq_quant_weight_per_channel,
     tfq_scaled_fp8_linear,
     tfq_scaled_fp8_linear_f16acc,
+    tfq_scaled_fp8_linear_multi,
     tfq_scaled_fp8_linear_noalloc,
     tfq_scaled_int8_linear,
     w8a8_int8_linear,
@@ -48,6 +49,7 @@ __all__ = [
     "tfq_quant_scaled_fp8_linear",
     "tfq_quant_scaled_fp8_linear_workspace_bytes",
     "tfq_scaled_fp8_linear_f16acc",
+    "tfq_scaled_fp8_linear_multi",
     "tfq_scaled_fp8_linear_noalloc",
     "tfq_quant_act_int8_per_token",
     "tfq_scaled_int8_linear",

@@ -26,6 +26,7 @@ TFQ_OK, TFQ_EINVAL, TFQ_EUNSUPPORTED, TFQ_ECUDA, TFQ_ETIMEOUT = range(5)
 TFQ_DTYPE_FP8_E4M3, TFQ_DTYPE_INT8 = 0, 1
 TFQ_QUANT_MAX_K = 1 << 24
 TFQ_INT8_MAX_K = 131072  # the INT8 GEMM takes K < this (its s32 sum stays exact)
+TFQ_MULTI_MAX_LINEARS = 4
 
 # name -> (restype, argtypes), in the order include/tfq.h declares them
 _P, _I64, _F, _I = ctypes.c_void_p, ctypes.c_int64, ctypes.c_float, ctypes.c_int
@@ -33,6 +34,7 @@ SIGNATURES = {
     "tfq_quant_act_fp8_per_token": (_I, [_P, _I64, _I64, _F, _P, _P, _P]),
     "tfq_quant_weight_per_channel": (_I, [_P, _I64, _I64, _I, _F, _P, _P, _P]),
     "tfq_scaled_fp8_linear": (_I, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _P]),
+    "tfq_scaled_fp8_linear_multi": (_I, [_P, _P, _I64, _I64, _I, _P, _P, _P, _P, _P, _P]),
     "tfq_quant_scaled_fp8_linear_workspace_bytes": (ctypes.c_size_t, [_I64]),
     "tfq_quant_scaled_fp8_linear": (_I, [_P, _I64, _I64, _F, _P, _P, _P, _I64, _P, _P, _P, _P, _P]),
     "tfq_quant_act_int8_per_token": (_I, [_P, _I64, _I64, _F, _P, _P, _P]),
@@ -358,6 +360,54 @@ def w8a8_linear(x, W_q, s_w, bias=None, qmax: float = 448.0, stream=None):
     """The whole Linear: per-token FP8 quantization of x, then the scaled GEMM."""
     A_q, s_a = tfq_quant_act_fp8_per_token(x, qmax, stream=stream)
     return tfq_scaled_fp8_linear(A_q, s_a, W_q, s_w, bias, stream=stream)
+
+
+def pointer_array(ptrs):
+    """A C array of void* (None for NULL entries) for the multi-Linear call."""
+    return (ctypes.c_void_p * len(ptrs))(*ptrs)
+
+
+def tfq_scaled_fp8_linear_multi(A_q, s_a, W_qs, s_ws, biases=None, outs=None, stream=None):
+    """The Linears that share A_q, s_a: W_qs / s_ws / biases (lists, biases or
+    any entry None) -> [out bf16 [M, N_i]], as one launch of the CTA-pair
+    kernel from 512 rows up (same bits as separate tfq_scaled_fp8_linear calls)."""
+    import torch
+    n = len(W_qs)
+    if not 1 <= n <= TFQ_MULTI_MAX_LINEARS or len(s_ws) != n or (biases is not None and len(biases) != n):
+        raise ValueError(f"1 to {TFQ_MULTI_MAX_LINEARS} Linears with one weight, scale and bias entry each")
+    _require(A_q, torch.uint8, 2, "A_q")
+    dev = A_q.device
+    _require(s_a, torch.float32, 1, "s_a", dev)
+    M, K = A_q.shape
+    if s_a.shape[0] != M:
+        raise ValueError("shape mismatch")
+    biases = [None] * n if biases is None else list(biases)
+    outs = [None] * n if outs is None else list(outs)
+    Ns = []
+    for i in range(n):
+        _require(W_qs[i], torch.uint8, 2, "W_q", dev)
+        _require(s_ws[i], torch.float32, 1, "s_w", dev)
+        N, K2 = W_qs[i].shape
+        if K2 != K or s_ws[i].shape[0] != N:
+            raise ValueError("shape mismatch")
+        if biases[i] is not None:
+            _require(biases[i], torch.bfloat16, 1, "bias", dev)
+            if biases[i].shape[0] != N:
+                raise ValueError("bias shape")
+        if outs[i] is None:
+            outs[i] = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        _require(outs[i], torch.bfloat16, 2, "out", dev)
+        if tuple(outs[i].shape) != (M, N):
+            raise ValueError("out shape")
+        Ns.append(N)
+    with torch.cuda.device(dev):
+        st = raw.tfq_scaled_fp8_linear_multi(
+            A_q.data_ptr(), s_a.data_ptr(), M, K, n, pointer_array([w.data_ptr() for w in W_qs]),
+            pointer_array([s.data_ptr() for s in s_ws]),
+            pointer_array([None if b is None else b.data_ptr() for b in biases]),
+            (ctypes.c_int64 * n)(*Ns), pointer_array([o.data_ptr() for o in outs]), _stream_handle(stream))
+    _check(st, "tfq_scaled_fp8_linear_multi")
+    return outs
 
 
 def tfq_quant_scaled_fp8_linear_workspace_bytes(M: int) -> int:

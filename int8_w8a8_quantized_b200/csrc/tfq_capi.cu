@@ -280,6 +280,26 @@ tfq_status tfq_scaled_fp8_linear(const void* A_q, const float* s_a, const void* 
                                   static_cast<cudaStream_t>(stream), ds);
 }
 
+tfq_status tfq_scaled_fp8_linear_multi(const void* A_q, const float* s_a, int64_t M, int64_t K, int n,
+                                       const void* const* W_q, const float* const* s_w, const void* const* bias_bf16,
+                                       const int64_t* N, void* const* out_bf16, void* stream) {
+    if (n < 1 || n > TFQ_MULTI_MAX_LINEARS)
+        return fail(TFQ_EINVAL, "n=%d outside [1, %d]", n, TFQ_MULTI_MAX_LINEARS);
+    if (W_q == nullptr || s_w == nullptr || N == nullptr || out_bf16 == nullptr)
+        return fail(TFQ_EINVAL, "null array");
+    for (int i = 0; i < n; ++i) {
+        const tfq_status st = check_gemm_args(A_q, s_a, W_q[i], s_w[i], bias_bf16 != nullptr ? bias_bf16[i] : nullptr,
+                                              M, N[i], K, out_bf16[i]);
+        if (st != TFQ_OK) return st;
+    }
+    if (M == 0) return TFQ_OK;
+    tfq_status st;
+    DeviceState* ds = current_device_state(&st);
+    if (ds == nullptr) return st;
+    return launch_scaled_fp8_gemm_multi(A_q, s_a, M, K, n, W_q, s_w, bias_bf16, N, out_bf16,
+                                        static_cast<cudaStream_t>(stream), ds);
+}
+
 size_t tfq_quant_scaled_fp8_linear_workspace_bytes(int64_t M) {
     return M < 0 ? 0 : quant_gemm_workspace_bytes(M);
 }

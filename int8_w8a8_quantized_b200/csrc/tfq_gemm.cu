@@ -322,11 +322,29 @@ __device__ __forceinline__ void quantize_rows_for_gemm(const GemmArgs& p, int la
     }
 }
 
+// Tensor maps of the CTA-pair kernel per Linear (see GemmArgs::n_lin): the
+// weight with 128-row boxes (b) and 64-row boxes (bq, the half-width tiles of
+// a split last round), and the output (y).
+struct PairMaps {
+    CUtensorMap b[kMaxLinears];
+    CUtensorMap bq[kMaxLinears];
+    CUtensorMap y[kMaxLinears];
+};
+
+// One Linear's operands on the host side: weight codes [N, K], column scales,
+// bias (may be null), N, output [M, N].
+struct LinearOperands {
+    const void* W;
+    const float* s_w;
+    const void* bias;
+    int64_t N;
+    void* out;
+};
+
 template <int PBN, int kAcc, int kQuant = 0>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair_threads<kQuant>(), 1)
-    scaled_mm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                                const __grid_constant__ CUtensorMap tmBq, const __grid_constant__ CUtensorMap tmY,
-                                GemmArgs p) {
+    scaled_mm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ PairMaps maps,
+                          GemmArgs p) {
     using C = PairCfg<PBN>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -362,9 +380,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair_threads<kQuant>
         *abort_flag = 0;
         fence_mbar_init();
         prefetch_tensormap(&tmA);
-        prefetch_tensormap(&tmB);
-        if (p.tail_halves) prefetch_tensormap(&tmBq);
-        prefetch_tensormap(&tmY);
+        for (int i = 0; i < p.n_lin; ++i) {
+            prefetch_tensormap(&maps.b[i]);
+            if (p.tail_halves) prefetch_tensormap(&maps.bq[i]);
+            prefetch_tensormap(&maps.y[i]);
+        }
     }
     if (warp == 1) {
         tmem_alloc_pair(tmem_slot, C::kTmemCols);
@@ -390,11 +410,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair_threads<kQuant>
             for (int w = cluster; ok && pair_work_item(w, total_tiles, n_clusters, p.tail_halves, t, half);
                  w += n_clusters, ++round) {
                 if (rank == 0) pace_round(p.round_ctr, round, total_tiles, n_clusters);
-                int tm, tn;
-                pair_tile_coords(t, m_tiles, p.n_tiles, p.group_m, p.band_n, tm, tn);
-                // a half tile: PBN / 2 columns, PBN / 4 B rows per CTA (tmBq's box)
+                int tm, tn_all, lin, tn;
+                pair_tile_coords(t, m_tiles, p.n_tiles, p.group_m, p.band_n, tm, tn_all);
+                split_linear_tile(p, tn_all, lin, tn);
+                // a half tile: PBN / 2 columns, PBN / 4 B rows per CTA (bq's box)
                 const int b_rows = half < 0 ? C::kBHalf : C::kBHalf / 2;
-                const CUtensorMap* tmb = half < 0 ? &tmB : &tmBq;
+                const CUtensorMap* tmb = half < 0 ? &maps.b[lin] : &maps.bq[lin];
                 const uint32_t stage_tx = 2 * static_cast<uint32_t>(C::kAStage + b_rows * BK);
                 const int a_row = tm * 256 + static_cast<int>(rank) * 128;
                 const int b_row = tn * PBN + (half > 0 ? PBN / 2 : 0) + static_cast<int>(rank) * b_rows;
@@ -483,10 +504,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair_threads<kQuant>
         int tcount = 0, t, half;
         for (int w = cluster; pair_work_item(w, total_tiles, n_clusters, p.tail_halves, t, half);
              w += n_clusters, ++tcount) {
-            int tm, tn;
-            pair_tile_coords(t, m_tiles, p.n_tiles, p.group_m, p.band_n, tm, tn);
+            int tm, tn_all, lin, tn;
+            pair_tile_coords(t, m_tiles, p.n_tiles, p.group_m, p.band_n, tm, tn_all);
+            split_linear_tile(p, tn_all, lin, tn);
+            const GemmArgs pl = linear_args(p, lin);
             const int n0 = tn * PBN + (half > 0 ? PBN / 2 : 0);
-            stage_col_params<PBN>(p, colp, n0, lane);
+            stage_col_params<PBN>(pl, colp, n0, lane);
             const int row0 = tm * 256 + static_cast<int>(rank) * 128 + quarter * 32;
             const int m = row0 + lane;
             float sa;
@@ -514,7 +537,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair_threads<kQuant>
             tc_fence_after();
             const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
                                    static_cast<uint32_t>(buf * PBN);
-            store_tile_rows<PBN, kAcc>(p, tmY, t_row, ebuf, colp, n0, row0, sa, lane, half < 0 ? PBN : PBN / 2);
+            store_tile_rows<PBN, kAcc>(pl, maps.y[lin], t_row, ebuf, colp, n0, row0, sa, lane,
+                                       half < 0 ? PBN : PBN / 2);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(buf == 0 ? tmem_empty_leader0 : tmem_empty_leader1);
@@ -555,10 +579,94 @@ __global__ void wait_selftest_kernel(uint64_t limit_ns, uint32_t* err) {
     if (threadIdx.x == 0 && !mbar_wait(&bar, 0, &abort_flag, limit_ns)) atomicOr(err, kErrSelfTest);
 }
 
+// Opt-in shared memory of the scaled GEMM kernels of one accumulator kind (once per device).
+template <int kAcc>
+tfq_status set_gemm_attributes(DeviceState* ds) {
+    if (ds->gemm_attr_set[kAcc]) return TFQ_OK;
+    cudaError_t e = cudaFuncSetAttribute(scaled_mm_kernel<kAcc>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(SMEM_BYTES));
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(scaled_mm_pair_kernel<256, kAcc>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(PairCfg<256>::kSmem));
+    if (e != cudaSuccess) return fail(TFQ_ECUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+    ds->gemm_attr_set[kAcc] = true;
+    return TFQ_OK;
+}
+
+// The tensor maps and the Linear table of the CTA-pair kernel for n Linears
+// that share A (their N tiles concatenated in order).
+tfq_status pair_linear_setup(const LinearOperands* lins, int n, int64_t M, int64_t K, PairMaps& maps,
+                             GemmArgs& a) {
+    constexpr int kPBN = 256;
+    using C = PairCfg<kPBN>;
+    int tiles = 0;
+    for (int i = 0; i < n; ++i) {
+        const LinearOperands& l = lins[i];
+        tfq_status st = encode_tensor_map_2d(&maps.b[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, l.W, K, l.N, K, BK,
+                                             C::kBHalf, CU_TENSOR_MAP_SWIZZLE_128B);
+        if (st == TFQ_OK)
+            st = encode_tensor_map_2d(&maps.bq[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, l.W, K, l.N, K, BK, C::kBHalf / 2,
+                                      CU_TENSOR_MAP_SWIZZLE_128B);
+        if (st == TFQ_OK)
+            st = encode_tensor_map_2d(&maps.y[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, l.out, l.N, M, l.N * 2, EPI_COLS,
+                                      32, CU_TENSOR_MAP_SWIZZLE_128B);
+        if (st != TFQ_OK) return st;
+        a.lin_tile0[i] = tiles;
+        a.lin_s_w[i] = l.s_w;
+        a.lin_bias[i] = static_cast<const uint16_t*>(l.bias);
+        a.lin_N[i] = static_cast<int>(l.N);
+        tiles += static_cast<int>((l.N + kPBN - 1) / kPBN);
+    }
+    for (int i = n; i <= kMaxLinears; ++i) a.lin_tile0[i] = tiles;
+    a.n_lin = n;
+    a.n_tiles = tiles;
+    a.s_w = lins[0].s_w;
+    a.bias = static_cast<const uint16_t*>(lins[0].bias);
+    a.N = static_cast<int>(lins[0].N);
+    return TFQ_OK;
+}
+
+// n Linears that share A (n = 1: the plain GEMM) as one launch of the
+// CTA-pair kernel (M >= TFQ_GEMM_PAIR_MIN_M).
+template <int kAcc>
+tfq_status launch_pair_linears(const void* A, const float* s_a, int64_t M, int64_t K, const LinearOperands* lins,
+                               int n, cudaStream_t stream, DeviceState* ds) {
+    tfq_status st = set_gemm_attributes<kAcc>(ds);
+    if (st != TFQ_OK) return st;
+    CUtensorMap tmA;
+    st = encode_tensor_map_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, A, K, M, K, BK, BM, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (st != TFQ_OK) return st;
+    PairMaps maps = {};
+    GemmArgs a;
+    st = pair_linear_setup(lins, n, M, K, maps, a);
+    if (st != TFQ_OK) return st;
+    a.s_a = s_a;
+    a.M = static_cast<int>(M);
+    a.K = static_cast<int>(K);
+    a.m_tiles = static_cast<int>((M + BM - 1) / BM);
+    a.k_blocks = static_cast<int>((K + BK - 1) / BK);
+    choose_raster(K, 256, a.band_n, a.group_m);
+    a.err = ds->err_word;
+    const int64_t pair_tiles = ((M + 255) / 256) * static_cast<int64_t>(a.n_tiles);
+    if (pair_tiles > INT32_MAX) return fail(TFQ_EUNSUPPORTED, "too many output tiles");
+    const int clusters = static_cast<int>(std::min<int64_t>(pair_tiles, ds->sm_count / 2));
+    a.tail_halves = choose_tail_halves(pair_tiles, clusters);
+    a.round_ctr = take_round_counter(ds);
+    const cudaError_t el = launch_kernel(scaled_mm_pair_kernel<256, kAcc>, dim3(2 * clusters), dim3(THREADS),
+                                         PairCfg<256>::kSmem, stream, tmA, maps, a);
+    if (el != cudaSuccess) return fail(TFQ_ECUDA, "GEMM launch: %s", cudaGetErrorString(el));
+    const cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? TFQ_OK : fail(TFQ_ECUDA, "GEMM launch: %s", cudaGetErrorString(e));
+}
+
 template <int kAcc>
 tfq_status launch_scaled_mm(const void* A, const float* s_a, const void* W, const float* s_w, const void* bias,
                             int64_t M, int64_t N, int64_t K, void* out, cudaStream_t stream, DeviceState* ds) {
     if (M == 0 || N == 0) return TFQ_OK;
+    if (use_pair_kernel(M, ds->sm_count)) {
+        const LinearOperands lin = {W, s_w, bias, N, out};
+        return launch_pair_linears<kAcc>(A, s_a, M, K, &lin, 1, stream, ds);
+    }
     CUtensorMap tmA, tmY;
     tfq_status st = encode_tensor_map_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, A, K, M, K, BK, BM,
                                          CU_TENSOR_MAP_SWIZZLE_128B);
@@ -566,16 +674,8 @@ tfq_status launch_scaled_mm(const void* A, const float* s_a, const void* W, cons
     st = encode_tensor_map_2d(&tmY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, out, N, M, N * 2, EPI_COLS, 32,
                               CU_TENSOR_MAP_SWIZZLE_128B);
     if (st != TFQ_OK) return st;
-    const int attr_idx = kAcc;
-    if (!ds->gemm_attr_set[attr_idx]) {
-        cudaError_t e = cudaFuncSetAttribute(scaled_mm_kernel<kAcc>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             static_cast<int>(SMEM_BYTES));
-        if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(scaled_mm_pair_kernel<256, kAcc>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     static_cast<int>(PairCfg<256>::kSmem));
-        if (e != cudaSuccess) return fail(TFQ_ECUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
-        ds->gemm_attr_set[attr_idx] = true;
-    }
+    st = set_gemm_attributes<kAcc>(ds);
+    if (st != TFQ_OK) return st;
     GemmArgs a;
     a.s_a = s_a;
     a.s_w = s_w;
@@ -586,36 +686,18 @@ tfq_status launch_scaled_mm(const void* A, const float* s_a, const void* W, cons
     a.m_tiles = static_cast<int>((M + BM - 1) / BM);
     a.n_tiles = static_cast<int>((N + BN - 1) / BN);
     a.k_blocks = static_cast<int>((K + BK - 1) / BK);
-    choose_raster(K, use_pair_kernel(M, ds->sm_count) ? 256 : BN, a.band_n, a.group_m);
+    choose_raster(K, BN, a.band_n, a.group_m);
     a.err = ds->err_word;
     a.round_ctr = nullptr;
     const int64_t tiles = static_cast<int64_t>(a.m_tiles) * a.n_tiles;
     if (tiles > INT32_MAX) return fail(TFQ_EUNSUPPORTED, "too many output tiles");
-    if (use_pair_kernel(M, ds->sm_count)) {
-        CUtensorMap tmBh, tmBq;
-        st = encode_tensor_map_2d(&tmBh, CU_TENSOR_MAP_DATA_TYPE_UINT8, W, K, N, K, BK, PairCfg<256>::kBHalf,
-                                  CU_TENSOR_MAP_SWIZZLE_128B);
-        if (st != TFQ_OK) return st;
-        st = encode_tensor_map_2d(&tmBq, CU_TENSOR_MAP_DATA_TYPE_UINT8, W, K, N, K, BK, PairCfg<256>::kBHalf / 2,
-                                  CU_TENSOR_MAP_SWIZZLE_128B);
-        if (st != TFQ_OK) return st;
-        const int64_t pair_tiles = ((M + 255) / 256) * static_cast<int64_t>(a.n_tiles);
-        const int clusters = static_cast<int>(std::min<int64_t>(pair_tiles, ds->sm_count / 2));
-        a.tail_halves = choose_tail_halves(pair_tiles, clusters);
-        a.round_ctr = take_round_counter(ds);
-        const cudaError_t el = launch_kernel(scaled_mm_pair_kernel<256, kAcc>, dim3(2 * clusters), dim3(THREADS),
-                                             PairCfg<256>::kSmem, stream, tmA, tmBh, tmBq, tmY, a);
-        if (el != cudaSuccess) return fail(TFQ_ECUDA, "GEMM launch: %s", cudaGetErrorString(el));
-    } else {
-        CUtensorMap tmB;
-        st = encode_tensor_map_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, W, K, N, K, BK, BN,
-                                  CU_TENSOR_MAP_SWIZZLE_128B);
-        if (st != TFQ_OK) return st;
-        const int grid = static_cast<int>(std::min<int64_t>(tiles, ds->sm_count));
-        const cudaError_t el = launch_kernel(scaled_mm_kernel<kAcc>, dim3(grid), dim3(THREADS), SMEM_BYTES, stream,
-                                             tmA, tmB, tmY, a);
-        if (el != cudaSuccess) return fail(TFQ_ECUDA, "GEMM launch: %s", cudaGetErrorString(el));
-    }
+    CUtensorMap tmB;
+    st = encode_tensor_map_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, W, K, N, K, BK, BN, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (st != TFQ_OK) return st;
+    const int grid = static_cast<int>(std::min<int64_t>(tiles, ds->sm_count));
+    const cudaError_t el = launch_kernel(scaled_mm_kernel<kAcc>, dim3(grid), dim3(THREADS), SMEM_BYTES, stream, tmA,
+                                         tmB, tmY, a);
+    if (el != cudaSuccess) return fail(TFQ_ECUDA, "GEMM launch: %s", cudaGetErrorString(el));
     const cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? TFQ_OK : fail(TFQ_ECUDA, "GEMM launch: %s", cudaGetErrorString(e));
 }
@@ -649,18 +731,14 @@ tfq_status launch_quant_scaled_fp8_gemm(const void* x, int64_t M, int64_t K, flo
     // start at zero.
     cudaError_t e = cudaMemsetAsync(workspace, 0, quant_gemm_workspace_bytes(M), stream);
     if (e != cudaSuccess) return fail(TFQ_ECUDA, "clearing the workspace: %s", cudaGetErrorString(e));
-    CUtensorMap tmA, tmY, tmBh, tmBq;
+    CUtensorMap tmA;
     tfq_status st = encode_tensor_map_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, A, K, M, K, BK, BM,
                                          CU_TENSOR_MAP_SWIZZLE_128B);
-    if (st == TFQ_OK)
-        st = encode_tensor_map_2d(&tmY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, out, N, M, N * 2, EPI_COLS, 32,
-                                  CU_TENSOR_MAP_SWIZZLE_128B);
-    if (st == TFQ_OK)
-        st = encode_tensor_map_2d(&tmBh, CU_TENSOR_MAP_DATA_TYPE_UINT8, W, K, N, K, BK, C::kBHalf,
-                                  CU_TENSOR_MAP_SWIZZLE_128B);
-    if (st == TFQ_OK)
-        st = encode_tensor_map_2d(&tmBq, CU_TENSOR_MAP_DATA_TYPE_UINT8, W, K, N, K, BK, C::kBHalf / 2,
-                                  CU_TENSOR_MAP_SWIZZLE_128B);
+    if (st != TFQ_OK) return st;
+    PairMaps maps = {};
+    GemmArgs a;
+    const LinearOperands lin = {W, s_w, bias, N, out};
+    st = pair_linear_setup(&lin, 1, M, K, maps, a);
     if (st != TFQ_OK) return st;
     auto kernel = clamp ? scaled_mm_pair_kernel<kPBN, kAccF32, 2> : scaled_mm_pair_kernel<kPBN, kAccF32, 1>;
     if (!ds->gemm_attr_set[5]) {
@@ -672,15 +750,10 @@ tfq_status launch_quant_scaled_fp8_gemm(const void* x, int64_t M, int64_t K, flo
         if (e != cudaSuccess) return fail(TFQ_ECUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
         ds->gemm_attr_set[5] = true;
     }
-    GemmArgs a;
     a.s_a = s_a;
-    a.s_w = s_w;
-    a.bias = static_cast<const uint16_t*>(bias);
     a.M = static_cast<int>(M);
-    a.N = static_cast<int>(N);
     a.K = static_cast<int>(K);
     a.m_tiles = static_cast<int>((M + BM - 1) / BM);
-    a.n_tiles = static_cast<int>((N + BN - 1) / BN);
     a.k_blocks = static_cast<int>((K + BK - 1) / BK);
     choose_raster(K, kPBN, a.band_n, a.group_m);
     a.err = ds->err_word;
@@ -696,8 +769,7 @@ tfq_status launch_quant_scaled_fp8_gemm(const void* x, int64_t M, int64_t K, flo
     a.q_next_row = ws;
     a.q_share_rows = ws + 32;
     a.qmax = qmax;
-    e = launch_kernel(kernel, dim3(2 * clusters), dim3(pair_threads<1>()), C::kSmem, stream, tmA, tmBh, tmBq, tmY,
-                      a);
+    e = launch_kernel(kernel, dim3(2 * clusters), dim3(pair_threads<1>()), C::kSmem, stream, tmA, maps, a);
     if (e != cudaSuccess) return fail(TFQ_ECUDA, "GEMM launch: %s", cudaGetErrorString(e));
     e = cudaGetLastError();
     return e == cudaSuccess ? TFQ_OK : fail(TFQ_ECUDA, "GEMM launch: %s", cudaGetErrorString(e));
@@ -707,6 +779,26 @@ tfq_status launch_scaled_fp8_gemm(const void* A, const float* s_a, const void* W
                                   const void* bias, int64_t M, int64_t N, int64_t K, void* out,
                                   cudaStream_t stream, DeviceState* ds) {
     return launch_scaled_mm<kAccF32>(A, s_a, W, s_w, bias, M, N, K, out, stream, ds);
+}
+
+tfq_status launch_scaled_fp8_gemm_multi(const void* A, const float* s_a, int64_t M, int64_t K, int n,
+                                        const void* const* W, const float* const* s_w, const void* const* bias,
+                                        const int64_t* N, void* const* out, cudaStream_t stream, DeviceState* ds) {
+    if (M == 0) return TFQ_OK;
+    LinearOperands lins[kMaxLinears];
+    int m = 0;
+    for (int i = 0; i < n; ++i)
+        if (N[i] > 0) lins[m++] = {W[i], s_w[i], bias != nullptr ? bias[i] : nullptr, N[i], out[i]};
+    if (m == 0) return TFQ_OK;
+    if (!use_pair_kernel(M, ds->sm_count)) {  // one-CTA kernel, one launch per Linear
+        for (int i = 0; i < m; ++i) {
+            const tfq_status st = launch_scaled_mm<kAccF32>(A, s_a, lins[i].W, lins[i].s_w, lins[i].bias, M,
+                                                            lins[i].N, K, lins[i].out, stream, ds);
+            if (st != TFQ_OK) return st;
+        }
+        return TFQ_OK;
+    }
+    return launch_pair_linears<kAccF32>(A, s_a, M, K, lins, m, stream, ds);
 }
 
 tfq_status launch_scaled_fp8_gemm_f16acc(const void* A, const float* s_a, const void* W, const float* s_w,

@@ -52,6 +52,10 @@ constexpr uint32_t make_idesc(int m, int n) {
     return fmt | (static_cast<uint32_t>(n >> 3) << 17) | (static_cast<uint32_t>(m >> 4) << 24);
 }
 
+// Linears that share their activations (and so the A operand) may run as one
+// CTA-pair launch: at most this many.
+constexpr int kMaxLinears = TFQ_MULTI_MAX_LINEARS;
+
 struct GemmArgs {
     const float* s_a;
     const float* s_w;
@@ -96,7 +100,35 @@ struct GemmArgs {
     unsigned* q_next_row = nullptr;
     unsigned* q_share_rows = nullptr;
     float qmax = 0.0f;
+    // The CTA-pair kernel: n_lin Linears that share A, their N tiles
+    // concatenated (n_tiles counts them all); tile columns [lin_tile0[i],
+    // lin_tile0[i + 1]) belong to Linear i, whose column scales, bias and N
+    // are lin_s_w[i], lin_bias[i] and lin_N[i].  One Linear: lin_tile0 = {0,
+    // n_tiles} and the three equal s_w, bias and N above.
+    int n_lin = 1;
+    int lin_tile0[kMaxLinears + 1] = {};
+    const float* lin_s_w[kMaxLinears] = {};
+    const uint16_t* lin_bias[kMaxLinears] = {};
+    int lin_N[kMaxLinears] = {};
 };
+
+// The Linear a column of tiles belongs to, and the tile's column within it.
+__device__ __forceinline__ void split_linear_tile(const GemmArgs& p, int tn_all, int& lin, int& tn) {
+    lin = 0;
+#pragma unroll
+    for (int i = 1; i < kMaxLinears; ++i)
+        if (i < p.n_lin && tn_all >= p.lin_tile0[i]) lin = i;
+    tn = tn_all - p.lin_tile0[lin];
+}
+
+// The arguments of one tile's epilogue: those of its Linear.
+__device__ __forceinline__ GemmArgs linear_args(const GemmArgs& p, int lin) {
+    GemmArgs q = p;
+    q.s_w = p.lin_s_w[lin];
+    q.bias = p.lin_bias[lin];
+    q.N = p.lin_N[lin];
+    return q;
+}
 
 #ifndef TFQ_PACING_WAIT_NS
 #define TFQ_PACING_WAIT_NS 200000ull

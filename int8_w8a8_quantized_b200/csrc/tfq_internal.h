@@ -110,6 +110,14 @@ tfq_status launch_scaled_fp8_gemm(const void* A, const float* s_a, const void* W
                                   const void* bias, int64_t M, int64_t N, int64_t K, void* out,
                                   cudaStream_t stream, DeviceState* ds);
 
+// Scaled FP8 GEMMs of n <= 4 Linears that share A_q and s_a: one launch of
+// the CTA-pair kernel (their N tiles concatenated) from M = 512 rows up, one
+// launch per Linear below.  bias may be null (no bias for any), and so may
+// any bias[i]; Linears with N[i] == 0 are skipped.
+tfq_status launch_scaled_fp8_gemm_multi(const void* A, const float* s_a, int64_t M, int64_t K, int n,
+                                        const void* const* W, const float* const* s_w, const void* const* bias,
+                                        const int64_t* N, void* const* out, cudaStream_t stream, DeviceState* ds);
+
 // Bytes of the workspace of launch_quant_scaled_fp8_gemm for M rows.
 size_t quant_gemm_workspace_bytes(int64_t M);
 

@@ -40,6 +40,7 @@ def test_header_declarations_match_binding():
 def test_header_limits_match_binding():
     text = open(os.path.join(ROOT, "include", "tfq.h"), encoding="utf-8").read()
     assert re.search(r"#define TFQ_INT8_MAX_K (\d+)", text).group(1) == str(_capi.TFQ_INT8_MAX_K)
+    assert re.search(r"#define TFQ_MULTI_MAX_LINEARS (\d+)", text).group(1) == str(_capi.TFQ_MULTI_MAX_LINEARS)
     assert re.search(r"#define TFQ_QUANT_MAX_K \(1 << (\d+)\)", text).group(1) == str(_capi.TFQ_QUANT_MAX_K.bit_length() - 1)
 
 
@@ -269,3 +270,33 @@ def test_quant_scaled_linear_validation(lib):
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU behaviour")
 def test_quant_scaled_linear_without_gpu_fails_loudly(lib):
     assert _fused(lib) in (_capi.TFQ_ECUDA, _capi.TFQ_EUNSUPPORTED)
+
+
+def _multi(lib, n=3, M=1024, K=256, W=None, sw=None, b=None, N=None, out=None, A=ALIGNED, sa=ALIGNED):
+    W = [ALIGNED] * n if W is None else W
+    sw = [ALIGNED] * n if sw is None else sw
+    N = [256] * n if N is None else N
+    out = [ALIGNED] * n if out is None else out
+    arr = _capi.pointer_array
+    return lib.tfq_scaled_fp8_linear_multi(A, sa, M, K, n, arr(W) if W != "null" else None, arr(sw),
+                                           None if b is None else arr(b), (ctypes.c_int64 * len(N))(*N),
+                                           arr(out), None)
+
+
+def test_multi_linear_validation(lib):
+    """The multi-Linear GEMM checks n, its arrays and every Linear's
+    arguments on the host, before any device work."""
+    assert _multi(lib, n=0, W=[], sw=[], N=[], out=[]) == _capi.TFQ_EINVAL
+    assert _multi(lib, n=5) == _capi.TFQ_EINVAL
+    assert _multi(lib, W="null") == _capi.TFQ_EINVAL
+    assert _multi(lib, N=[256, 12, 256]) == _capi.TFQ_EINVAL                      # N % 8
+    assert _multi(lib, W=[ALIGNED, None, ALIGNED]) == _capi.TFQ_EINVAL             # a null weight
+    assert _multi(lib, out=[ALIGNED, ALIGNED, ALIGNED + 2]) == _capi.TFQ_EINVAL    # misaligned output
+    assert _multi(lib, b=[None, ALIGNED + 8, None]) == _capi.TFQ_EINVAL            # misaligned bias
+    assert _multi(lib, K=24) == _capi.TFQ_EINVAL
+    assert _multi(lib, M=0, A=None, sa=None) == _capi.TFQ_OK                       # empty: no-op
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU behaviour")
+def test_multi_linear_without_gpu_fails_loudly(lib):
+    assert _multi(lib) in (_capi.TFQ_ECUDA, _capi.TFQ_EUNSUPPORTED)
