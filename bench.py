@@ -4,7 +4,8 @@
 A step is one pass of the whole hot path over one DiT block: for every
 distinct activation of the block, per-token FP8 quantization (tfq kernel),
 then every Linear reading it as a scaled FP8 GEMM with the fused
-scale/bias/BF16 epilogue (tfq kernel).  Weights are quantized once per
+scale/bias/BF16 epilogue (tfq kernel; FP8 runs the Linears that read one
+activation, Q, K and V, as one launch unless --separate).  Weights are quantized once per
 channel before timing (the offline converter step).  The metric is the
 block's GEMM FLOPs divided by the step time, which includes the activation
 quantizers ("TFLOP/s incl. act quant").
@@ -19,6 +20,7 @@ data-path collective); time is the max over ranks.
 from __future__ import annotations
 
 import argparse
+import ctypes
 import json
 import os
 import statistics
@@ -70,6 +72,9 @@ def parse_args():
     ap.add_argument("--fused", action="store_true",
                     help="fp8 only: the first Linear of each activation quantizes it inside its GEMM "
                          "(tfq_quant_scaled_fp8_linear: one kernel); the other Linears of that input take its codes")
+    ap.add_argument("--separate", action="store_true",
+                    help="FP8: one GEMM launch per Linear (by default the Linears that read one activation, Q, K "
+                         "and V, run as one tfq_scaled_fp8_linear_multi launch)")
     ap.add_argument("--tokens", type=int, default=0,
                     help="run the workload's Linears over this many tokens instead of its M (for ncu captures on "
                          "a reduced case; never a benchmark figure)")
@@ -396,6 +401,16 @@ def gpu_arm(args, wl, rank, world, local_rank):
     # "fused" (the first Linear of each activation quantizes it inside its
     # GEMM; metadata = (M, N, K, quantizer bytes)).
     fused = getattr(args, "fused", False)
+    multi = getattr(args, "multi", False)
+
+    def multi_arrays(group, q):
+        """The array arguments of tfq_scaled_fp8_linear_multi for the Linears
+        of `group` (weights, scales, biases, N, outputs) and the stream."""
+        return (_capi.pointer_array([W.data_ptr() for _, W, _, _ in group]),
+                _capi.pointer_array([s.data_ptr() for _, _, s, _ in group]),
+                _capi.pointer_array([None if bb is None else bb.data_ptr() for _, _, _, bb in group]),
+                (ctypes.c_int64 * len(group))(*[l.N for l, _, _, _ in group]),
+                _capi.pointer_array([ys[(l.name, q)].data_ptr() for l, _, _, _ in group]), sh)
     wss = {name: torch.empty(lib.tfq_quant_scaled_fp8_linear_workspace_bytes(x.shape[0]), dtype=torch.uint8,
                              device=dev) for name, x in xs.items()} if fused else {}
     ops = []
@@ -421,6 +436,15 @@ def gpu_arm(args, wl, rank, world, local_rank):
                                                             sw.data_ptr(), bp, lin.N, A.data_ptr(), sa.data_ptr(),
                                                             y.data_ptr(), ws.data_ptr(), sh),
                             (wl.M, lin.N, lin.K, 3 * x.numel() + 4 * x.shape[0])))
+            elif multi and lin.x in seen:
+                pass  # launched with the first Linear that reads lin.x
+            elif multi:
+                group = [(l, W, s, bb) for l, W, s, bb in lins if l.x == lin.x]
+                arrs = multi_arrays(group, q)
+                ops.append(("gemm",
+                            lambda A=A, sa=sa, lin=lin, n=len(group), arrs=arrs:
+                            lib.tfq_scaled_fp8_linear_multi(A.data_ptr(), sa.data_ptr(), wl.M, lin.K, n, *arrs),
+                            (wl.M, sum(l.N for l, _, _, _ in group), lin.K)))
             else:
                 ops.append(("gemm",
                             lambda A=A, sa=sa, Wq=Wq, sw=sw, bp=bp, lin=lin, y=y:
@@ -474,7 +498,7 @@ def gpu_arm(args, wl, rank, world, local_rank):
     ms_per_step = ms / args.steps
 
     # one step's kernels (for the path floor), independent of which launches had events
-    step_shapes = [(wl.M, lin.N, lin.K) for q in qmaxes for lin, _, _, _ in lins]
+    step_shapes = [meta[:3] for kind, _, meta in ops if kind != "quant"]
     step_quant_bytes = [3 * x.numel() + (x.numel() // 32 if mx else 4 * x.shape[0]) for q in qmaxes for x in xs.values()]
 
     def gemm_step_bytes(m, n, k):
@@ -522,7 +546,7 @@ def gpu_arm(args, wl, rank, world, local_rank):
     e2e = None
     if not args.no_e2e:
         e2e = e2e_arm(args, wl, qmaxes, quant_fn, gemm_fn, xs, lins, aq, ys, stream, sh, check, lib=lib,
-                      wss=wss if fused else None)
+                      wss=wss if fused else None, multi_arrays=multi_arrays if multi else None)
     return out, e2e
 
 
@@ -565,7 +589,8 @@ def torch_scaled_mm_context(args, wl, lins, aq, ys, qmaxes, stream):
         return {"error": f"{type(e).__name__}: {str(e)[:200]}"}
 
 
-def e2e_arm(args, wl, qmaxes, quant_fn, gemm_fn, xs, lins, aq, ys, stream, sh, check, lib=None, wss=None):
+def e2e_arm(args, wl, qmaxes, quant_fn, gemm_fn, xs, lins, aq, ys, stream, sh, check, lib=None, wss=None,
+            multi_arrays=None):
     """Every step: H2D copy of each activation of the block from pinned host
     memory, the quantizers and GEMMs, D2H copy of every output into pinned
     host memory.  The copies run on two copy streams and overlap the
@@ -584,6 +609,7 @@ def e2e_arm(args, wl, qmaxes, quant_fn, gemm_fn, xs, lins, aq, ys, stream, sh, c
     for lin in lins:
         if lin[0].x not in order:
             order.append(lin[0].x)
+    multi = multi_arrays is not None
     x_read = {}   # event: the quantizers of the previous step finished reading x
     y_read = {}   # event: the D2H copy of the previous step finished reading y
 
@@ -609,6 +635,23 @@ def e2e_arm(args, wl, qmaxes, quant_fn, gemm_fn, xs, lins, aq, ys, stream, sh, c
             for q in qmaxes:
                 A, sa = aq[(n, q)]
                 first = True
+                if multi:  # the Linears that read x as one launch
+                    group = [(lin, Wq, sw, b) for lin, Wq, sw, b in lins if lin.x == n]
+                    for lin, _, _, _ in group:
+                        if (lin.name, q) in y_read:
+                            stream.wait_event(y_read[(lin.name, q)])
+                    check(lib.tfq_scaled_fp8_linear_multi(
+                        A.data_ptr(), sa.data_ptr(), wl.M, group[0][0].K, len(group),
+                        *multi_arrays(group, q)), "gemm")
+                    done = torch.cuda.Event()
+                    done.record(stream)
+                    copy_out.wait_event(done)
+                    for lin, _, _, _ in group:
+                        with torch.cuda.stream(copy_out):
+                            hy[(lin.name, q)].copy_(ys[(lin.name, q)], non_blocking=True)
+                        y_read[(lin.name, q)] = torch.cuda.Event()
+                        y_read[(lin.name, q)].record(copy_out)
+                    continue
                 for lin, Wq, sw, b in lins:
                     if lin.x != n:
                         continue
@@ -1110,6 +1153,8 @@ def main():
         wl = dataclasses.replace(wl, M=args.tokens)
     if args.fused and args.dtype != "fp8":
         raise SystemExit("--fused takes --dtype fp8")
+    # FP8 without --fused: the Linears that share an activation as one launch
+    args.multi = args.dtype == "fp8" and not args.fused and not args.separate
     cfg = {"workload": wl.name, "M": wl.M, "dtype": args.dtype,
            "linears": [f"{l.name}:{l.K}->{l.N}" for l in wl.linears],
            "act_qmax": list(act_qmaxes(wl, args.dtype)) if args.dtype != "mxfp8" else "none (E8M0 scale per 32 values)",
@@ -1120,6 +1165,8 @@ def main():
            "parallelism": f"replicas x{world}"}
     if args.fused:
         cfg["quantization"] = "inside the first GEMM of each activation (one kernel per Linear)"
+    if args.multi:
+        cfg["launches"] = "the Linears that read one activation (Q, K, V) as one GEMM launch"
     if args.tokens:
         cfg["reduced_tokens"] = f"M = {args.tokens} instead of the workload's M (a profiling case, not a benchmark)"
 

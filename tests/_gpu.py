@@ -74,8 +74,14 @@ def bf16_bits_np(t: torch.Tensor) -> np.ndarray:
     return t.detach().contiguous().cpu().view(torch.int16).numpy().view(np.uint16)
 
 
+# (what, outputs compared, E_max, E_rel, worst error / bound) of every GEMM
+# tolerance check of the session; printed as a table at the end of the run.
+PARITY_RECORDS: list = []
+
+
 def gemm_tolerance_check(y_gpu: torch.Tensor, y_ref: np.ndarray, what: str = ""):
-    """|y - y_ref| <= 2^-7 |y_ref| + 1e-3 rms(y_ref), element by element."""
+    """|y - y_ref| <= 2^-7 |y_ref| + 1e-3 rms(y_ref), element by element.
+    Returns (E_max, E_rel) and records them with the worst error / bound."""
     y = y_gpu.float().cpu().numpy().astype(np.float64)
     assert y.shape == y_ref.shape
     rms = float(np.sqrt(np.mean(y_ref ** 2))) if y_ref.size else 0.0
@@ -89,6 +95,8 @@ def gemm_tolerance_check(y_gpu: torch.Tensor, y_ref: np.ndarray, what: str = "")
                              f"gpu {y[tuple(i)]} ref {y_ref[tuple(i)]} bound {bound[tuple(i)]}")
     e_max = float(err.max()) if err.size else 0.0
     e_rel = float(np.linalg.norm(y - y_ref) / max(np.linalg.norm(y_ref), 1e-300))
+    worst = float((err / np.maximum(bound, 1e-300)).max()) if err.size else 0.0
+    PARITY_RECORDS.append((what, int(err.size), e_max, e_rel, worst))
     return e_max, e_rel
 
 
