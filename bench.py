@@ -4,8 +4,8 @@
 A step is one pass of the whole hot path over one DiT block: for every
 distinct activation of the block, per-token FP8 quantization (tfq kernel),
 then every Linear reading it as a scaled FP8 GEMM with the fused
-scale/bias/BF16 epilogue (tfq kernel; FP8 runs the Linears that read one
-activation, Q, K and V, as one launch unless --separate).  Weights are quantized once per
+scale/bias/BF16 epilogue (tfq kernel; FP8 and INT8 run the Linears that
+read one activation, Q, K and V, as one launch unless --separate).  Weights are quantized once per
 channel before timing (the offline converter step).  The metric is the
 block's GEMM FLOPs divided by the step time, which includes the activation
 quantizers ("TFLOP/s incl. act quant").
@@ -73,8 +73,8 @@ def parse_args():
                     help="fp8 only: the first Linear of each activation quantizes it inside its GEMM "
                          "(tfq_quant_scaled_fp8_linear: one kernel); the other Linears of that input take its codes")
     ap.add_argument("--separate", action="store_true",
-                    help="FP8: one GEMM launch per Linear (by default the Linears that read one activation, Q, K "
-                         "and V, run as one tfq_scaled_fp8_linear_multi launch)")
+                    help="FP8, INT8: one GEMM launch per Linear (by default the Linears that read one activation, "
+                         "Q, K and V, run as one multi-Linear launch)")
     ap.add_argument("--tokens", type=int, default=0,
                     help="run the workload's Linears over this many tokens instead of its M (for ncu captures on "
                          "a reduced case; never a benchmark figure)")
@@ -402,10 +402,11 @@ def gpu_arm(args, wl, rank, world, local_rank):
     # GEMM; metadata = (M, N, K, quantizer bytes)).
     fused = getattr(args, "fused", False)
     multi = getattr(args, "multi", False)
+    multi_fn = lib.tfq_scaled_int8_linear_multi if args.dtype == "int8" else lib.tfq_scaled_fp8_linear_multi
 
     def multi_arrays(group, q):
-        """The array arguments of tfq_scaled_fp8_linear_multi for the Linears
-        of `group` (weights, scales, biases, N, outputs) and the stream."""
+        """The array arguments of the multi-Linear GEMM for the Linears of
+        `group` (weights, scales, biases, N, outputs) and the stream."""
         return (_capi.pointer_array([W.data_ptr() for _, W, _, _ in group]),
                 _capi.pointer_array([s.data_ptr() for _, _, s, _ in group]),
                 _capi.pointer_array([None if bb is None else bb.data_ptr() for _, _, _, bb in group]),
@@ -443,7 +444,7 @@ def gpu_arm(args, wl, rank, world, local_rank):
                 arrs = multi_arrays(group, q)
                 ops.append(("gemm",
                             lambda A=A, sa=sa, lin=lin, n=len(group), arrs=arrs:
-                            lib.tfq_scaled_fp8_linear_multi(A.data_ptr(), sa.data_ptr(), wl.M, lin.K, n, *arrs),
+                            multi_fn(A.data_ptr(), sa.data_ptr(), wl.M, lin.K, n, *arrs),
                             (wl.M, sum(l.N for l, _, _, _ in group), lin.K)))
             else:
                 ops.append(("gemm",
@@ -546,7 +547,7 @@ def gpu_arm(args, wl, rank, world, local_rank):
     e2e = None
     if not args.no_e2e:
         e2e = e2e_arm(args, wl, qmaxes, quant_fn, gemm_fn, xs, lins, aq, ys, stream, sh, check, lib=lib,
-                      wss=wss if fused else None, multi_arrays=multi_arrays if multi else None)
+                      wss=wss if fused else None, multi=(multi_fn, multi_arrays) if multi else None)
     return out, e2e
 
 
@@ -590,7 +591,7 @@ def torch_scaled_mm_context(args, wl, lins, aq, ys, qmaxes, stream):
 
 
 def e2e_arm(args, wl, qmaxes, quant_fn, gemm_fn, xs, lins, aq, ys, stream, sh, check, lib=None, wss=None,
-            multi_arrays=None):
+            multi=None):
     """Every step: H2D copy of each activation of the block from pinned host
     memory, the quantizers and GEMMs, D2H copy of every output into pinned
     host memory.  The copies run on two copy streams and overlap the
@@ -609,7 +610,7 @@ def e2e_arm(args, wl, qmaxes, quant_fn, gemm_fn, xs, lins, aq, ys, stream, sh, c
     for lin in lins:
         if lin[0].x not in order:
             order.append(lin[0].x)
-    multi = multi_arrays is not None
+    multi_fn, multi_arrays = multi if multi is not None else (None, None)
     x_read = {}   # event: the quantizers of the previous step finished reading x
     y_read = {}   # event: the D2H copy of the previous step finished reading y
 
@@ -640,9 +641,8 @@ def e2e_arm(args, wl, qmaxes, quant_fn, gemm_fn, xs, lins, aq, ys, stream, sh, c
                     for lin, _, _, _ in group:
                         if (lin.name, q) in y_read:
                             stream.wait_event(y_read[(lin.name, q)])
-                    check(lib.tfq_scaled_fp8_linear_multi(
-                        A.data_ptr(), sa.data_ptr(), wl.M, group[0][0].K, len(group),
-                        *multi_arrays(group, q)), "gemm")
+                    check(multi_fn(A.data_ptr(), sa.data_ptr(), wl.M, group[0][0].K, len(group),
+                                   *multi_arrays(group, q)), "gemm")
                     done = torch.cuda.Event()
                     done.record(stream)
                     copy_out.wait_event(done)
@@ -1153,8 +1153,8 @@ def main():
         wl = dataclasses.replace(wl, M=args.tokens)
     if args.fused and args.dtype != "fp8":
         raise SystemExit("--fused takes --dtype fp8")
-    # FP8 without --fused: the Linears that share an activation as one launch
-    args.multi = args.dtype == "fp8" and not args.fused and not args.separate
+    # FP8 and INT8 without --fused: the Linears that share an activation as one launch
+    args.multi = args.dtype in ("fp8", "int8") and not args.fused and not args.separate
     cfg = {"workload": wl.name, "M": wl.M, "dtype": args.dtype,
            "linears": [f"{l.name}:{l.K}->{l.N}" for l in wl.linears],
            "act_qmax": list(act_qmaxes(wl, args.dtype)) if args.dtype != "mxfp8" else "none (E8M0 scale per 32 values)",

@@ -132,7 +132,7 @@ TFQ_API tfq_status tfq_scaled_fp8_linear(const void *A_q, const float *s_a, cons
                                  const float *s_w, const void *bias_bf16, int64_t M, int64_t N,
                                  int64_t K, void *out_bf16, void *stream);
 
-/* Most Linears tfq_scaled_fp8_linear_multi takes in one call. */
+/* Most Linears tfq_scaled_fp8_linear_multi and tfq_scaled_int8_linear_multi take in one call. */
 #define TFQ_MULTI_MAX_LINEARS 4
 
 /*
@@ -223,6 +223,19 @@ TFQ_API tfq_status tfq_quant_act_int8_per_token(const void *x_bf16, int64_t M, i
 TFQ_API tfq_status tfq_scaled_int8_linear(const void *A_q, const float *s_a, const void *W_q,
                                           const float *s_w, const void *bias_bf16, int64_t M, int64_t N,
                                           int64_t K, void *out_bf16, void *stream);
+
+/*
+ * tfq_scaled_int8_linear_multi: tfq_scaled_fp8_linear_multi with int8
+ * operands -- out[i] = the result of tfq_scaled_int8_linear(A_q, s_a,
+ * W_q[i], s_w[i], bias_bf16[i], M, N[i], K, out[i]) for i < n, the same bits,
+ * from M = 512 rows up as one launch of the INT8 CTA-pair kernel.  Arrays,
+ * preconditions and errors as in tfq_scaled_fp8_linear_multi, and K >=
+ * TFQ_INT8_MAX_K returns TFQ_EUNSUPPORTED.
+ */
+TFQ_API tfq_status tfq_scaled_int8_linear_multi(const void *A_q, const float *s_a, int64_t M, int64_t K, int n,
+                                                const void *const *W_q, const float *const *s_w,
+                                                const void *const *bias_bf16, const int64_t *N,
+                                                void *const *out_bf16, void *stream);
 
 /*
  * tfq_scaled_fp8_linear_f16acc: tfq_scaled_fp8_linear with the products

@@ -38,6 +38,7 @@ from ._capi import (  # noqa: F401
     tfq_scaled_fp8_linear_multi,
     tfq_scaled_fp8_linear_noalloc,
     tfq_scaled_int8_linear,
+    tfq_scaled_int8_linear_multi,
     w8a8_int8_linear,
     w8a8_linear,
 )
@@ -53,6 +54,7 @@ __all__ = [
     "tfq_scaled_fp8_linear_noalloc",
     "tfq_quant_act_int8_per_token",
     "tfq_scaled_int8_linear",
+    "tfq_scaled_int8_linear_multi",
     "w8a8_int8_linear",
     "tfq_device_error",
     "w8a8_linear",

@@ -39,6 +39,7 @@ SIGNATURES = {
     "tfq_quant_scaled_fp8_linear": (_I, [_P, _I64, _I64, _F, _P, _P, _P, _I64, _P, _P, _P, _P, _P]),
     "tfq_quant_act_int8_per_token": (_I, [_P, _I64, _I64, _F, _P, _P, _P]),
     "tfq_scaled_int8_linear": (_I, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _P]),
+    "tfq_scaled_int8_linear_multi": (_I, [_P, _P, _I64, _I64, _I, _P, _P, _P, _P, _P, _P]),
     "tfq_scaled_fp8_linear_f16acc": (_I, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _P]),
     "tfq_mxfp8_scale_bytes": (_I64, [_I64, _I64]),
     "tfq_quant_mxfp8": (_I, [_P, _I64, _I64, _P, _P, _P]),
@@ -367,15 +368,13 @@ def pointer_array(ptrs):
     return (ctypes.c_void_p * len(ptrs))(*ptrs)
 
 
-def tfq_scaled_fp8_linear_multi(A_q, s_a, W_qs, s_ws, biases=None, outs=None, stream=None):
-    """The Linears that share A_q, s_a: W_qs / s_ws / biases (lists, biases or
-    any entry None) -> [out bf16 [M, N_i]], as one launch of the CTA-pair
-    kernel from 512 rows up (same bits as separate tfq_scaled_fp8_linear calls)."""
+def _linear_multi(name, code_dtype, A_q, s_a, W_qs, s_ws, biases, outs, stream):
+    """The multi-Linear GEMM `name` on operands of `code_dtype`."""
     import torch
     n = len(W_qs)
     if not 1 <= n <= TFQ_MULTI_MAX_LINEARS or len(s_ws) != n or (biases is not None and len(biases) != n):
         raise ValueError(f"1 to {TFQ_MULTI_MAX_LINEARS} Linears with one weight, scale and bias entry each")
-    _require(A_q, torch.uint8, 2, "A_q")
+    _require(A_q, code_dtype, 2, "A_q")
     dev = A_q.device
     _require(s_a, torch.float32, 1, "s_a", dev)
     M, K = A_q.shape
@@ -385,7 +384,7 @@ def tfq_scaled_fp8_linear_multi(A_q, s_a, W_qs, s_ws, biases=None, outs=None, st
     outs = [None] * n if outs is None else list(outs)
     Ns = []
     for i in range(n):
-        _require(W_qs[i], torch.uint8, 2, "W_q", dev)
+        _require(W_qs[i], code_dtype, 2, "W_q", dev)
         _require(s_ws[i], torch.float32, 1, "s_w", dev)
         N, K2 = W_qs[i].shape
         if K2 != K or s_ws[i].shape[0] != N:
@@ -401,13 +400,28 @@ def tfq_scaled_fp8_linear_multi(A_q, s_a, W_qs, s_ws, biases=None, outs=None, st
             raise ValueError("out shape")
         Ns.append(N)
     with torch.cuda.device(dev):
-        st = raw.tfq_scaled_fp8_linear_multi(
+        st = getattr(raw, name)(
             A_q.data_ptr(), s_a.data_ptr(), M, K, n, pointer_array([w.data_ptr() for w in W_qs]),
             pointer_array([s.data_ptr() for s in s_ws]),
             pointer_array([None if b is None else b.data_ptr() for b in biases]),
             (ctypes.c_int64 * n)(*Ns), pointer_array([o.data_ptr() for o in outs]), _stream_handle(stream))
-    _check(st, "tfq_scaled_fp8_linear_multi")
+    _check(st, name)
     return outs
+
+
+def tfq_scaled_fp8_linear_multi(A_q, s_a, W_qs, s_ws, biases=None, outs=None, stream=None):
+    """The Linears that share A_q, s_a: W_qs / s_ws / biases (lists, biases or
+    any entry None) -> [out bf16 [M, N_i]], as one launch of the CTA-pair
+    kernel from 512 rows up (same bits as separate tfq_scaled_fp8_linear calls)."""
+    import torch
+    return _linear_multi("tfq_scaled_fp8_linear_multi", torch.uint8, A_q, s_a, W_qs, s_ws, biases, outs, stream)
+
+
+def tfq_scaled_int8_linear_multi(A_q, s_a, W_qs, s_ws, biases=None, outs=None, stream=None):
+    """tfq_scaled_fp8_linear_multi with int8 operands (same bits as separate
+    tfq_scaled_int8_linear calls)."""
+    import torch
+    return _linear_multi("tfq_scaled_int8_linear_multi", torch.int8, A_q, s_a, W_qs, s_ws, biases, outs, stream)
 
 
 def tfq_quant_scaled_fp8_linear_workspace_bytes(M: int) -> int:

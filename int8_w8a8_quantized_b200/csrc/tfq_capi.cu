@@ -197,6 +197,36 @@ tfq_status check_gemm_args(const void* A_q, const float* s_a, const void* W_q, c
     return TFQ_OK;
 }
 
+// The host checks of the multi-Linear GEMMs: n in [1, TFQ_MULTI_MAX_LINEARS],
+// the arrays present and every Linear's arguments valid.
+static tfq_status check_multi_args(const void* A_q, const float* s_a, int64_t M, int64_t K, int n,
+                                   const void* const* W_q, const float* const* s_w, const void* const* bias_bf16,
+                                   const int64_t* N, void* const* out_bf16) {
+    if (n < 1 || n > TFQ_MULTI_MAX_LINEARS)
+        return fail(TFQ_EINVAL, "n=%d outside [1, %d]", n, TFQ_MULTI_MAX_LINEARS);
+    if (W_q == nullptr || s_w == nullptr || N == nullptr || out_bf16 == nullptr)
+        return fail(TFQ_EINVAL, "null array");
+    for (int i = 0; i < n; ++i) {
+        const tfq_status st = check_gemm_args(A_q, s_a, W_q[i], s_w[i], bias_bf16 != nullptr ? bias_bf16[i] : nullptr,
+                                              M, N[i], K, out_bf16[i]);
+        if (st != TFQ_OK) return st;
+    }
+    return TFQ_OK;
+}
+
+using MultiLauncher = tfq_status (*)(const void*, const float*, int64_t, int64_t, int, const void* const*,
+                                     const float* const*, const void* const*, const int64_t*, void* const*,
+                                     cudaStream_t, DeviceState*);
+
+static tfq_status launch_multi(MultiLauncher launcher, const void* A_q, const float* s_a, int64_t M, int64_t K,
+                               int n, const void* const* W_q, const float* const* s_w, const void* const* bias_bf16,
+                               const int64_t* N, void* const* out_bf16, void* stream) {
+    tfq_status st;
+    DeviceState* ds = current_device_state(&st);
+    if (ds == nullptr) return st;
+    return launcher(A_q, s_a, M, K, n, W_q, s_w, bias_bf16, N, out_bf16, static_cast<cudaStream_t>(stream), ds);
+}
+
 }  // namespace tfq
 
 extern "C" {
@@ -283,21 +313,20 @@ tfq_status tfq_scaled_fp8_linear(const void* A_q, const float* s_a, const void* 
 tfq_status tfq_scaled_fp8_linear_multi(const void* A_q, const float* s_a, int64_t M, int64_t K, int n,
                                        const void* const* W_q, const float* const* s_w, const void* const* bias_bf16,
                                        const int64_t* N, void* const* out_bf16, void* stream) {
-    if (n < 1 || n > TFQ_MULTI_MAX_LINEARS)
-        return fail(TFQ_EINVAL, "n=%d outside [1, %d]", n, TFQ_MULTI_MAX_LINEARS);
-    if (W_q == nullptr || s_w == nullptr || N == nullptr || out_bf16 == nullptr)
-        return fail(TFQ_EINVAL, "null array");
-    for (int i = 0; i < n; ++i) {
-        const tfq_status st = check_gemm_args(A_q, s_a, W_q[i], s_w[i], bias_bf16 != nullptr ? bias_bf16[i] : nullptr,
-                                              M, N[i], K, out_bf16[i]);
-        if (st != TFQ_OK) return st;
-    }
-    if (M == 0) return TFQ_OK;
-    tfq_status st;
-    DeviceState* ds = current_device_state(&st);
-    if (ds == nullptr) return st;
-    return launch_scaled_fp8_gemm_multi(A_q, s_a, M, K, n, W_q, s_w, bias_bf16, N, out_bf16,
-                                        static_cast<cudaStream_t>(stream), ds);
+    const tfq_status st = check_multi_args(A_q, s_a, M, K, n, W_q, s_w, bias_bf16, N, out_bf16);
+    if (st != TFQ_OK || M == 0) return st;
+    return launch_multi(launch_scaled_fp8_gemm_multi, A_q, s_a, M, K, n, W_q, s_w, bias_bf16, N, out_bf16, stream);
+}
+
+tfq_status tfq_scaled_int8_linear_multi(const void* A_q, const float* s_a, int64_t M, int64_t K, int n,
+                                        const void* const* W_q, const float* const* s_w, const void* const* bias_bf16,
+                                        const int64_t* N, void* const* out_bf16, void* stream) {
+    const tfq_status st = check_multi_args(A_q, s_a, M, K, n, W_q, s_w, bias_bf16, N, out_bf16);
+    if (st != TFQ_OK) return st;
+    if (K >= TFQ_INT8_MAX_K) return fail(TFQ_EUNSUPPORTED, "K=%lld: the INT8 sum may exceed s32 (K < %d)",
+                                         (long long)K, TFQ_INT8_MAX_K);
+    if (M == 0) return st;
+    return launch_multi(launch_scaled_int8_gemm_multi, A_q, s_a, M, K, n, W_q, s_w, bias_bf16, N, out_bf16, stream);
 }
 
 size_t tfq_quant_scaled_fp8_linear_workspace_bytes(int64_t M) {

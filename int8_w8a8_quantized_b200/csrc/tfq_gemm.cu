@@ -781,9 +781,12 @@ tfq_status launch_scaled_fp8_gemm(const void* A, const float* s_a, const void* W
     return launch_scaled_mm<kAccF32>(A, s_a, W, s_w, bias, M, N, K, out, stream, ds);
 }
 
-tfq_status launch_scaled_fp8_gemm_multi(const void* A, const float* s_a, int64_t M, int64_t K, int n,
-                                        const void* const* W, const float* const* s_w, const void* const* bias,
-                                        const int64_t* N, void* const* out, cudaStream_t stream, DeviceState* ds) {
+namespace {
+
+template <int kAcc>
+tfq_status launch_gemm_multi(const void* A, const float* s_a, int64_t M, int64_t K, int n, const void* const* W,
+                             const float* const* s_w, const void* const* bias, const int64_t* N, void* const* out,
+                             cudaStream_t stream, DeviceState* ds) {
     if (M == 0) return TFQ_OK;
     LinearOperands lins[kMaxLinears];
     int m = 0;
@@ -792,13 +795,27 @@ tfq_status launch_scaled_fp8_gemm_multi(const void* A, const float* s_a, int64_t
     if (m == 0) return TFQ_OK;
     if (!use_pair_kernel(M, ds->sm_count)) {  // one-CTA kernel, one launch per Linear
         for (int i = 0; i < m; ++i) {
-            const tfq_status st = launch_scaled_mm<kAccF32>(A, s_a, lins[i].W, lins[i].s_w, lins[i].bias, M,
-                                                            lins[i].N, K, lins[i].out, stream, ds);
+            const tfq_status st = launch_scaled_mm<kAcc>(A, s_a, lins[i].W, lins[i].s_w, lins[i].bias, M, lins[i].N,
+                                                         K, lins[i].out, stream, ds);
             if (st != TFQ_OK) return st;
         }
         return TFQ_OK;
     }
-    return launch_pair_linears<kAccF32>(A, s_a, M, K, lins, m, stream, ds);
+    return launch_pair_linears<kAcc>(A, s_a, M, K, lins, m, stream, ds);
+}
+
+}  // namespace
+
+tfq_status launch_scaled_fp8_gemm_multi(const void* A, const float* s_a, int64_t M, int64_t K, int n,
+                                        const void* const* W, const float* const* s_w, const void* const* bias,
+                                        const int64_t* N, void* const* out, cudaStream_t stream, DeviceState* ds) {
+    return launch_gemm_multi<kAccF32>(A, s_a, M, K, n, W, s_w, bias, N, out, stream, ds);
+}
+
+tfq_status launch_scaled_int8_gemm_multi(const void* A, const float* s_a, int64_t M, int64_t K, int n,
+                                         const void* const* W, const float* const* s_w, const void* const* bias,
+                                         const int64_t* N, void* const* out, cudaStream_t stream, DeviceState* ds) {
+    return launch_gemm_multi<kAccS32>(A, s_a, M, K, n, W, s_w, bias, N, out, stream, ds);
 }
 
 tfq_status launch_scaled_fp8_gemm_f16acc(const void* A, const float* s_a, const void* W, const float* s_w,

@@ -118,6 +118,11 @@ tfq_status launch_scaled_fp8_gemm_multi(const void* A, const float* s_a, int64_t
                                         const void* const* W, const float* const* s_w, const void* const* bias,
                                         const int64_t* N, void* const* out, cudaStream_t stream, DeviceState* ds);
 
+// The same with int8 operands (S8 x S8 -> S32).
+tfq_status launch_scaled_int8_gemm_multi(const void* A, const float* s_a, int64_t M, int64_t K, int n,
+                                         const void* const* W, const float* const* s_w, const void* const* bias,
+                                         const int64_t* N, void* const* out, cudaStream_t stream, DeviceState* ds);
+
 // Bytes of the workspace of launch_quant_scaled_fp8_gemm for M rows.
 size_t quant_gemm_workspace_bytes(int64_t M);
 

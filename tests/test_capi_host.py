@@ -272,31 +272,46 @@ def test_quant_scaled_linear_without_gpu_fails_loudly(lib):
     assert _fused(lib) in (_capi.TFQ_ECUDA, _capi.TFQ_EUNSUPPORTED)
 
 
-def _multi(lib, n=3, M=1024, K=256, W=None, sw=None, b=None, N=None, out=None, A=ALIGNED, sa=ALIGNED):
+MULTI_ENTRIES = ("tfq_scaled_fp8_linear_multi", "tfq_scaled_int8_linear_multi")
+
+
+def _multi(lib, n=3, M=1024, K=256, W=None, sw=None, b=None, N=None, out=None, A=ALIGNED, sa=ALIGNED,
+           entry="tfq_scaled_fp8_linear_multi"):
     W = [ALIGNED] * n if W is None else W
     sw = [ALIGNED] * n if sw is None else sw
     N = [256] * n if N is None else N
     out = [ALIGNED] * n if out is None else out
     arr = _capi.pointer_array
-    return lib.tfq_scaled_fp8_linear_multi(A, sa, M, K, n, arr(W) if W != "null" else None, arr(sw),
-                                           None if b is None else arr(b), (ctypes.c_int64 * len(N))(*N),
-                                           arr(out), None)
+    return getattr(lib, entry)(A, sa, M, K, n, arr(W) if W != "null" else None, arr(sw),
+                               None if b is None else arr(b), (ctypes.c_int64 * len(N))(*N), arr(out), None)
 
 
-def test_multi_linear_validation(lib):
-    """The multi-Linear GEMM checks n, its arrays and every Linear's
+@pytest.mark.parametrize("entry", MULTI_ENTRIES)
+def test_multi_linear_validation(lib, entry):
+    """The multi-Linear GEMMs check n, their arrays and every Linear's
     arguments on the host, before any device work."""
-    assert _multi(lib, n=0, W=[], sw=[], N=[], out=[]) == _capi.TFQ_EINVAL
-    assert _multi(lib, n=5) == _capi.TFQ_EINVAL
-    assert _multi(lib, W="null") == _capi.TFQ_EINVAL
-    assert _multi(lib, N=[256, 12, 256]) == _capi.TFQ_EINVAL                      # N % 8
-    assert _multi(lib, W=[ALIGNED, None, ALIGNED]) == _capi.TFQ_EINVAL             # a null weight
-    assert _multi(lib, out=[ALIGNED, ALIGNED, ALIGNED + 2]) == _capi.TFQ_EINVAL    # misaligned output
-    assert _multi(lib, b=[None, ALIGNED + 8, None]) == _capi.TFQ_EINVAL            # misaligned bias
-    assert _multi(lib, K=24) == _capi.TFQ_EINVAL
-    assert _multi(lib, M=0, A=None, sa=None) == _capi.TFQ_OK                       # empty: no-op
+    def multi(**kw):
+        return _multi(lib, entry=entry, **kw)
+    assert multi(n=0, W=[], sw=[], N=[], out=[]) == _capi.TFQ_EINVAL
+    assert multi(n=5) == _capi.TFQ_EINVAL
+    assert multi(W="null") == _capi.TFQ_EINVAL
+    assert multi(N=[256, 12, 256]) == _capi.TFQ_EINVAL                      # N % 8
+    assert multi(W=[ALIGNED, None, ALIGNED]) == _capi.TFQ_EINVAL             # a null weight
+    assert multi(out=[ALIGNED, ALIGNED, ALIGNED + 2]) == _capi.TFQ_EINVAL    # misaligned output
+    assert multi(b=[None, ALIGNED + 8, None]) == _capi.TFQ_EINVAL            # misaligned bias
+    assert multi(K=24) == _capi.TFQ_EINVAL
+    assert multi(M=0, A=None, sa=None) == _capi.TFQ_OK                       # empty: no-op
+
+
+def test_int8_multi_k_limit(lib):
+    """Like tfq_scaled_int8_linear, the multi form refuses K whose s32 sum
+    could overflow, before any device work."""
+    K = _capi.TFQ_INT8_MAX_K
+    assert _multi(lib, K=K, entry="tfq_scaled_int8_linear_multi") == _capi.TFQ_EUNSUPPORTED
+    assert _multi(lib, K=K, M=0, A=None, sa=None, entry="tfq_scaled_int8_linear_multi") == _capi.TFQ_EUNSUPPORTED
 
 
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU behaviour")
-def test_multi_linear_without_gpu_fails_loudly(lib):
-    assert _multi(lib) in (_capi.TFQ_ECUDA, _capi.TFQ_EUNSUPPORTED)
+@pytest.mark.parametrize("entry", MULTI_ENTRIES)
+def test_multi_linear_without_gpu_fails_loudly(lib, entry):
+    assert _multi(lib, entry=entry) in (_capi.TFQ_ECUDA, _capi.TFQ_EUNSUPPORTED)

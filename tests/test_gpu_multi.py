@@ -1,10 +1,12 @@
-"""GPU parity of tfq_scaled_fp8_linear_multi: the scaled FP8 GEMMs of up to
-four Linears that share their input, as one launch of the CTA-pair kernel
-(their N tiles concatenated) from 512 rows up.
+"""GPU parity of tfq_scaled_fp8_linear_multi and tfq_scaled_int8_linear_multi:
+the scaled FP8 (INT8) GEMMs of up to four Linears that share their input, as
+one launch of the CTA-pair kernel (their N tiles concatenated) from 512 rows
+up.
 
 Each output must equal, bit for bit, the output of the separate
-tfq_scaled_fp8_linear call (the same tiles, the same arithmetic), and be
-within |y - y_ref| <= 2^-7 |y_ref| + 1e-3 rms(y_ref) of the oracle.
+tfq_scaled_fp8_linear (tfq_scaled_int8_linear) call -- the same tiles, the
+same arithmetic -- and be within |y - y_ref| <= 2^-7 |y_ref| + 1e-3 rms(y_ref)
+of the oracle.
 """
 import numpy as np
 import pytest
@@ -27,14 +29,14 @@ def _codes(g, shape):
     return (mag | (torch.randint(0, 2, shape, generator=g, dtype=torch.int32) << 7)).to(torch.uint8).cuda()
 
 
-def _multi(A, sa, Ws, sws, biases):
+def _multi(A, sa, Ws, sws, biases, entry="tfq_scaled_fp8_linear_multi"):
     """The raw C call, guard elements after every output."""
     M, K = A.shape
     n = len(Ws)
     outs = [_gpu.guarded(M * W.shape[0], torch.bfloat16, 12345.0) for W in Ws]
     arr = _capi.pointer_array
     import ctypes
-    st = _capi.raw.tfq_scaled_fp8_linear_multi(
+    st = getattr(_capi.raw, entry)(
         A.data_ptr(), sa.data_ptr(), M, K, n, arr([W.data_ptr() for W in Ws]), arr([s.data_ptr() for s in sws]),
         arr([None if b is None else b.data_ptr() for b in biases]), (ctypes.c_int64 * n)(*[W.shape[0] for W in Ws]),
         arr([o.data_ptr() for o in outs]), _gpu.stream_handle())
@@ -132,3 +134,53 @@ def test_video_dit_qkv_full_size():
         _gpu.gemm_tolerance_check(y[ridx], y_ref, f"video {lin.name}")
     del ys
     torch.cuda.empty_cache()
+
+
+def _int8_linear(A, sa, W, sw, b):
+    M, K = A.shape
+    N = W.shape[0]
+    out = _gpu.guarded(M * N, torch.bfloat16, 12345.0)
+    st = _capi.raw.tfq_scaled_int8_linear(A.data_ptr(), sa.data_ptr(), W.data_ptr(), sw.data_ptr(),
+                                          None if b is None else b.data_ptr(), M, N, K, out.data_ptr(),
+                                          _gpu.stream_handle())
+    assert st == _capi.TFQ_OK, _capi.last_error_message()
+    _gpu.check_device_error()
+    assert torch.all(out[M * N:] == 12345.0), "write past the end of the output"
+    return out[:M * N].view(M, N)
+
+
+@pytest.mark.parametrize("M,Ns,K,bias_mask", [
+    (6889, [3072, 3072, 3072], 3072, [True, True, True]),      # the image-DiT Q, K, V
+    (2600, [1032, 520, 264], 1024, [True, False, True]),       # ragged N, one Linear without bias
+    (1100, [8, 1864], 400, [False, True]),                     # tiny N, K tail
+    (300, [520, 264], 1024, [True, True]),                      # below 512 rows: one launch per Linear
+])
+def test_int8_multi_matches_single_calls_and_oracle(M, Ns, K, bias_mask):
+    seed = 7 * M + sum(Ns) + K
+    g = torch.Generator().manual_seed(seed)
+    A = torch.randint(-128, 128, (M, K), generator=g, dtype=torch.int8).cuda()
+    sa = (torch.rand(M, generator=g) * 1e-3 + 1e-5).cuda()
+    Ws = [torch.randint(-128, 128, (N, K), generator=g, dtype=torch.int8).cuda() for N in Ns]
+    sws = [(torch.rand(N, generator=g) * 1e-3 + 1e-5).cuda() for N in Ns]
+    biases = [(torch.randn(N, generator=g) * 0.5).to(torch.bfloat16).cuda() if use else None
+              for N, use in zip(Ns, bias_mask)]
+    ys = _multi(A, sa, Ws, sws, biases, entry="tfq_scaled_int8_linear_multi")
+    rows = _gpu.tile_sample_rows(M, seed=seed)
+    for i, (y, W, sw, b) in enumerate(zip(ys, Ws, sws, biases)):
+        y1 = _int8_linear(A, sa, W, sw, b)
+        assert torch.equal(y.view(torch.int16), y1.view(torch.int16)), f"INT8 Linear {i} differs from its own call"
+        y_ref = oracle.scaled_int8_linear(A.cpu().numpy(), sa.cpu().numpy(), W.cpu().numpy(), sw.cpu().numpy(),
+                                          None if b is None else _gpu.bf16_bits_np(b), rows=rows)
+        _gpu.gemm_tolerance_check(y[torch.as_tensor(rows, device="cuda")], y_ref, f"int8 multi M={M} #{i}")
+
+
+def test_int8_tensor_wrapper():
+    from int8_w8a8_quantized_b200 import tfq_scaled_int8_linear, tfq_scaled_int8_linear_multi
+    g = torch.Generator().manual_seed(11)
+    A = torch.randint(-128, 128, (1536, 512), generator=g, dtype=torch.int8).cuda()
+    sa = (torch.rand(1536, generator=g) * 1e-3).cuda()
+    Ws = [torch.randint(-128, 128, (N, 512), generator=g, dtype=torch.int8).cuda() for N in (768, 256)]
+    sws = [(torch.rand(W.shape[0], generator=g) * 1e-3).cuda() for W in Ws]
+    ys = tfq_scaled_int8_linear_multi(A, sa, Ws, sws)
+    for y, W, sw in zip(ys, Ws, sws):
+        assert torch.equal(y.view(torch.int16), tfq_scaled_int8_linear(A, sa, W, sw).view(torch.int16))
