@@ -52,6 +52,8 @@
  *    results never depend on it.
  *  - Non-finite inputs (inf, NaN) are outside the contract: the codes and
  *    scales of a row holding one are unspecified.
+ *  - An output buffer must not overlap any input or any other output of the
+ *    same call; the results are unspecified otherwise.
  */
 #ifndef TFQ_H_
 #define TFQ_H_

@@ -4,7 +4,8 @@
   after the other -- every output element is computed by one CTA in a fixed
   order, so the kernels are deterministic;
 * the quantizer and the GEMM calls captured into a CUDA graph (after the
-  device's one-time set-up) replay to the eager results on new inputs."""
+  device's one-time set-up) replay to the eager results on new inputs;
+* the same for the one-call quantizing Linear and the multi-Linear GEMMs."""
 import pytest
 import torch
 
@@ -229,5 +230,76 @@ def test_one_call_quant_linear_graph_and_concurrent_streams():
         call(c, main)
         torch.cuda.synchronize()
         assert torch.equal(y_graph, c[6])
+    del graph
+    _gpu.check_device_error()
+
+
+def test_multi_linear_graph_and_concurrent_streams():
+    """Q/K/V-like multi-Linear launches (FP8 and INT8) on two streams at once,
+    and one captured into a CUDA graph and replayed on new codes, give the
+    results of the same calls run eagerly one after the other."""
+    lib = _gpu.lib()
+    g = torch.Generator().manual_seed(23)
+    M, K, Ns = 2100, 1024, (1032, 520, 776)
+    arr = _capi.pointer_array
+    import ctypes
+
+    def operands(int8):
+        if int8:
+            A = torch.randint(-128, 128, (M, K), generator=g, dtype=torch.int8).cuda()
+            Ws = [torch.randint(-128, 128, (N, K), generator=g, dtype=torch.int8).cuda() for N in Ns]
+        else:
+            A, Ws = _codes(g, (M, K)), [_codes(g, (N, K)) for N in Ns]
+        sa = (torch.rand(M, generator=g) * 1e-3).cuda()
+        sws = [(torch.rand(N, generator=g) * 1e-3).cuda() for N in Ns]
+        bs = [torch.randn(N, generator=g).to(torch.bfloat16).cuda() for N in Ns]
+        ys = [torch.empty((M, N), dtype=torch.bfloat16, device="cuda") for N in Ns]
+        return A, sa, Ws, sws, bs, ys
+
+    def call(entry, ops, stream):
+        A, sa, Ws, sws, bs, ys = ops
+        st = getattr(lib, entry)(A.data_ptr(), sa.data_ptr(), M, K, len(Ns), arr([w.data_ptr() for w in Ws]),
+                                 arr([s.data_ptr() for s in sws]), arr([b.data_ptr() for b in bs]),
+                                 (ctypes.c_int64 * len(Ns))(*Ns), arr([y.data_ptr() for y in ys]),
+                                 int(stream.cuda_stream))
+        assert st == _capi.TFQ_OK, _capi.last_error_message()
+
+    cases = [("tfq_scaled_fp8_linear_multi", operands(False)), ("tfq_scaled_int8_linear_multi", operands(True))]
+    main = torch.cuda.current_stream()
+    for entry, ops in cases:
+        call(entry, ops, main)
+    torch.cuda.synchronize()
+    serial = [[y.clone() for y in ops[5]] for _, ops in cases]
+    streams = [torch.cuda.Stream() for _ in cases]
+    for _ in range(3):
+        for (_, ops) in cases:
+            for y in ops[5]:
+                y.zero_()
+        for (entry, ops), s in zip(cases, streams):
+            s.wait_stream(main)
+            call(entry, ops, s)
+        for s in streams:
+            main.wait_stream(s)
+        torch.cuda.synchronize()
+        for (_, ops), ref in zip(cases, serial):
+            for y, r in zip(ops[5], ref):
+                assert torch.equal(y, r)
+    entry, ops = cases[0]
+    graph = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream()
+    side.wait_stream(main)
+    with torch.cuda.stream(side):
+        with torch.cuda.graph(graph, stream=side):
+            call(entry, ops, side)
+    main.wait_stream(side)
+    for _ in range(2):
+        ops[0].copy_(_codes(g, (M, K)))
+        graph.replay()
+        torch.cuda.synchronize()
+        y_graph = [y.clone() for y in ops[5]]
+        call(entry, ops, main)
+        torch.cuda.synchronize()
+        for a, b in zip(y_graph, ops[5]):
+            assert torch.equal(a, b)
     del graph
     _gpu.check_device_error()
