@@ -198,10 +198,19 @@ class ClockSampler:
         pynvml, h = self.nvml
         reasons_fn = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
             pynvml.nvmlDeviceGetCurrentClocksThrottleReasons
+        fid = getattr(pynvml, "NVML_FI_DEV_POWER_INSTANT", None)
         while not self.stop_flag:
             try:
+                inst = None
+                if fid is not None:  # the board's instantaneous power (read only)
+                    try:
+                        fv = pynvml.nvmlDeviceGetFieldValues(h, [fid])[0]
+                        if fv.nvmlReturn == 0:
+                            inst = float(fv.value.uiVal) / 1000.0
+                    except Exception:
+                        fid = None
                 self.samples.append((pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM),
-                                     pynvml.nvmlDeviceGetPowerUsage(h) / 1000.0, int(reasons_fn(h))))
+                                     pynvml.nvmlDeviceGetPowerUsage(h) / 1000.0, int(reasons_fn(h)), inst))
             except Exception:
                 pass
             _t.sleep(0.01)
@@ -259,17 +268,25 @@ CLOCK_REASON_BITS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdo
 
 
 def summarize_nvml_samples(samples, sm_max, limit_w):
-    """Clock record from NVML samples (SM MHz, board watts, reason bit mask):
-    median SM clock and power, the peak power, and every reason that was
-    active in any sample.  None without samples."""
+    """Clock record from NVML samples (SM MHz, board watts as NVML's power
+    usage, reason bit mask[, instantaneous board watts or None]): median SM
+    clock and power, the peak power, and every reason that was active in any
+    sample.  None without samples."""
     if not samples:
         return None
-    reasons = sorted(n for n, bit in CLOCK_REASON_BITS.items() if any(r & bit for _, _, r in samples))
-    return {"sm_mhz": statistics.median(c for c, _, _ in samples), "sm_max_mhz": sm_max,
-            "power_w_max": max(p for _, p, _ in samples),
-            "power_w_median": statistics.median(p for _, p, _ in samples),
-            "power_limit_w": limit_w, "samples": len(samples),
-            "source": "nvml, 10 ms", "reasons": reasons}
+    reasons = sorted(n for n, bit in CLOCK_REASON_BITS.items() if any(smp[2] & bit for smp in samples))
+    rec = {"sm_mhz": statistics.median(smp[0] for smp in samples), "sm_max_mhz": sm_max,
+           "power_w_max": max(smp[1] for smp in samples),
+           "power_w_median": statistics.median(smp[1] for smp in samples),
+           "power_limit_w": limit_w, "samples": len(samples),
+           "source": "nvml, 10 ms", "reasons": reasons}
+    inst = [smp[3] for smp in samples if len(smp) > 3 and smp[3] is not None]
+    if inst:
+        rec["power_w_instant_median"] = statistics.median(inst)
+        rec["power_w_instant_max"] = max(inst)
+        rec["power_note"] = ("power_w_median/max: NVML power usage, averaged by the driver over a window that "
+                             "lags a short timed region; power_w_instant_*: the instantaneous board power")
+    return rec
 
 
 def summarize_smi_lines(lines):
@@ -1279,6 +1296,11 @@ def main():
     if e2e is not None:
         e2e["value"] = round(world * e2e["value"], 3)
         line["e2e"] = e2e
+    clk = res["clocks"] or {}
+    if clk.get("power_w_instant_median") and value > 0:
+        line["energy"] = {"pj_per_op": round(clk["power_w_instant_median"] / (value / world), 4),
+                          "what": "median instantaneous board power in the timed region / this GPU's rate "
+                                  "(W per TFLOP/s = pJ per FLOP or OP, quantizers included)"}
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wl, args.cpu_seconds, args.dtype,
                                             single_thread_seconds=max(2.0, args.cpu_seconds / 2))

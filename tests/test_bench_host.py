@@ -31,6 +31,12 @@ def test_summarize_nvml_samples():
     bad = bench.summarize_nvml_samples([(900, 500.0, 0x8 | 0x40), (950, 500.0, 0x20)], 1965.0, None)
     assert bad["reasons"] == ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown"]
     assert bench.summarize_nvml_samples([], 1965.0, 1000.0) is None
+    # with the instantaneous board power (None where the field read failed)
+    inst = bench.summarize_nvml_samples([(1200, 500.0, 0x4, 990.0), (1210, 520.0, 0x4, None),
+                                         (1220, 540.0, 0x4, 1010.0), (1230, 560.0, 0x4, 1000.0)], 1965.0, 1000.0)
+    assert inst["power_w_instant_median"] == 1000.0 and inst["power_w_instant_max"] == 1010.0
+    assert inst["power_w_median"] == 530.0 and "power_note" in inst
+    assert "power_w_instant_median" not in rec
 
 
 def test_summarize_smi_lines():
