@@ -90,3 +90,62 @@ def test_mxfp8_quantizer_and_gemm(i):
     y_ref = oracle.mxfp8_linear(A.cpu().numpy(), _gpu.mx_untile(sfa.cpu().numpy(), M, K), W.cpu().numpy(),
                                 _gpu.mx_untile(sfw.cpu().numpy(), N, K), _gpu.bf16_bits_np(b))
     _gpu.gemm_tolerance_check(y, y_ref, f"mx M={M} N={N} K={K}")
+
+
+MULTI_RNG = np.random.default_rng(20261203)
+MULTI_CASES = []
+while len(MULTI_CASES) < 12:
+    n = int(MULTI_RNG.integers(1, 5))
+    M = int(MULTI_RNG.integers(1, 3000))
+    Ns = [int(MULTI_RNG.integers(0, 160)) * 8 for _ in range(n)]
+    K = int(MULTI_RNG.integers(1, 120)) * 16
+    if sum(Ns) > 0 and M * sum(Ns) * K <= 2 ** 31:
+        MULTI_CASES.append((M, Ns, K, [bool(MULTI_RNG.integers(0, 2)) for _ in range(n)]))
+MULTI_CASES.append((1500, [264, 0, 520], 320, [True, False, True]))  # a zero-width Linear between two others
+
+
+@pytest.mark.parametrize("i", range(len(MULTI_CASES)))
+def test_multi_linear_gemms(i):
+    """FP8 and INT8 multi-Linear GEMMs on random shapes (N = 0 Linears, null
+    biases, rows below and above the CTA-pair threshold): every output equal
+    to its single call bit for bit, and within the tolerance of the oracle."""
+    import ctypes
+    M, Ns, K, with_bias = MULTI_CASES[i]
+    g = torch.Generator().manual_seed(4000 + i)
+    arr = _capi.pointer_array
+    for int8 in (False, True):
+        if int8:
+            A = torch.randint(-128, 128, (M, K), generator=g, dtype=torch.int8)
+            Ws = [torch.randint(-128, 128, (N, K), generator=g, dtype=torch.int8) for N in Ns]
+        else:
+            A, Ws = _codes(g, (M, K)), [_codes(g, (N, K)) for N in Ns]
+        sa = torch.rand(M, generator=g) * 1e-2 + 1e-4
+        sws = [torch.rand(N, generator=g) * 1e-2 + 1e-4 for N in Ns]
+        bs = [(torch.randn(N, generator=g) * 0.5).to(torch.bfloat16) if wb else None for N, wb in zip(Ns, with_bias)]
+        dA, dsa = A.cuda(), sa.cuda()
+        dWs, dsws = [w.cuda() for w in Ws], [s.cuda() for s in sws]
+        dbs = [None if b is None else b.cuda() for b in bs]
+        ys = [_gpu.guarded(M * N, torch.bfloat16, 12345.0) for N in Ns]
+        entry = "tfq_scaled_int8_linear_multi" if int8 else "tfq_scaled_fp8_linear_multi"
+        st = getattr(_capi.raw, entry)(dA.data_ptr(), dsa.data_ptr(), M, K, len(Ns), arr([w.data_ptr() for w in dWs]),
+                                       arr([s.data_ptr() for s in dsws]),
+                                       arr([None if b is None else b.data_ptr() for b in dbs]),
+                                       (ctypes.c_int64 * len(Ns))(*Ns), arr([y.data_ptr() for y in ys]),
+                                       _gpu.stream_handle())
+        assert st == _capi.TFQ_OK, _capi.last_error_message()
+        _gpu.check_device_error()
+        single = _capi.raw.tfq_scaled_int8_linear if int8 else _capi.raw.tfq_scaled_fp8_linear
+        ref_fn = oracle.scaled_int8_linear if int8 else oracle.scaled_fp8_linear
+        for j, (N, y) in enumerate(zip(Ns, ys)):
+            assert torch.all(y[M * N:] == 12345.0), "write past the end of an output"
+            if N == 0:
+                continue
+            y = y[:M * N].view(M, N)
+            y1 = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+            st = single(dA.data_ptr(), dsa.data_ptr(), dWs[j].data_ptr(), dsws[j].data_ptr(),
+                        None if dbs[j] is None else dbs[j].data_ptr(), M, N, K, y1.data_ptr(), _gpu.stream_handle())
+            assert st == _capi.TFQ_OK, _capi.last_error_message()
+            assert torch.equal(y.view(torch.int16), y1.view(torch.int16)), f"Linear {j} differs from its own call"
+            y_ref = ref_fn(A.numpy(), sa.numpy(), Ws[j].numpy(), sws[j].numpy(),
+                           None if bs[j] is None else _gpu.bf16_bits_np(bs[j]))
+            _gpu.gemm_tolerance_check(y, y_ref, f"{'int8' if int8 else 'fp8'} multi M={M} N={N} K={K} #{j}")
