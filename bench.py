@@ -432,6 +432,7 @@ def gpu_arm(args, wl, rank, world, local_rank):
     wss = {name: torch.empty(lib.tfq_quant_scaled_fp8_linear_workspace_bytes(x.shape[0]), dtype=torch.uint8,
                              device=dev) for name, x in xs.items()} if fused else {}
     ops = []
+    quant_inputs = {}  # op index -> the activation a quantizer launch reads
     # Block order, as a LinearFP8 forward runs: each activation is quantized
     # directly before the first Linear that reads it (Q, K and V share theirs).
     for q in qmaxes:
@@ -442,6 +443,7 @@ def gpu_arm(args, wl, rank, world, local_rank):
             bp = None if b is None else b.data_ptr()
             if not fused and lin.x not in seen:
                 x = xs[lin.x]
+                quant_inputs[len(ops)] = x
                 ops.append(("quant",
                             lambda x=x, q=q, A=A, sa=sa: quant_fn(x.data_ptr(), x.shape[0], x.shape[1], float(q),
                                                                   A.data_ptr(), sa.data_ptr(), sh),
@@ -515,6 +517,43 @@ def gpu_arm(args, wl, rank, world, local_rank):
     ms = max_over_ranks(t0.elapsed_time(t1), dev) if world > 1 else t0.elapsed_time(t1)
     ms_per_step = ms / args.steps
 
+    # What the step allows a stream of the quantizers' bytes: the same step with
+    # every quantizer launch replaced by a device copy of the same traffic (it
+    # reads and writes half of the launch's algorithmic bytes each), in its
+    # place between the GEMMs, timed the same way.  Context for quantizer.frac
+    # (the achievable bandwidth at the clock the GEMMs leave), not part of the metric.
+    copy_ref = None
+    if quant_inputs:
+        nbs = {k: ops[k][2] // 2 for k in quant_inputs}
+        dst = torch.empty(max(nbs.values()), dtype=torch.uint8, device=dev)
+        copy_ops = []
+        for k, (kind, launch, meta) in enumerate(ops):
+            if k in quant_inputs:
+                src = quant_inputs[k].view(-1).view(torch.uint8)[:nbs[k]]
+                copy_ops.append(("copy", lambda s=src, d=dst[:nbs[k]]: d.copy_(s), 2 * nbs[k]))
+            else:
+                copy_ops.append((kind, launch, meta))
+        cev = []
+        for i in range(2 + args.steps):
+            for k, (kind, launch, meta) in enumerate(copy_ops):
+                rec = i >= 2 and kind == "copy" and (k == i % len(copy_ops) or not sample_one)
+                if rec:
+                    e0 = torch.cuda.Event(enable_timing=True); e0.record(stream)
+                if kind == "copy":
+                    launch()
+                else:
+                    check(launch(), kind)
+                if rec:
+                    e1 = torch.cuda.Event(enable_timing=True); e1.record(stream)
+                    cev.append((e0, e1, meta))
+        torch.cuda.synchronize()
+        if cev:
+            cms = sum(a.elapsed_time(b) for a, b, _ in cev)
+            copy_ref = {"gbs": sum(m for _, _, m in cev) / (cms * 1e-3) / 1e9, "launches_timed": len(cev),
+                        "what": "the step with each quantizer launch replaced by a device copy of the same "
+                                "traffic (half read, half written), events as for the quantizers"}
+        del dst
+
     # one step's kernels (for the path floor), independent of which launches had events
     step_shapes = [meta[:3] for kind, _, meta in ops if kind != "quant"]
     step_quant_bytes = [3 * x.numel() + (x.numel() // 32 if mx else 4 * x.shape[0]) for q in qmaxes for x in xs.values()]
@@ -548,7 +587,7 @@ def gpu_arm(args, wl, rank, world, local_rank):
         "kernel_events": (f"each kernel bracketed in {args.steps // n_kernels}-{-(-args.steps // n_kernels)} of "
                           f"the {args.steps} timed steps (one kernel per step)") if sample_one
         else "every kernel of every timed step",
-        "gpu_launches": launches[0], "clocks": clk,
+        "gpu_launches": launches[0], "clocks": clk, "quant_copy_reference": copy_ref,
         "sm_count": torch.cuda.get_device_properties(dev).multi_processor_count,
         "per_linear": {},
     }
@@ -1284,6 +1323,9 @@ def main():
                                    res["quant_launches_per_step"] / res["ms_per_step"], 4),
             "traffic": recorded_traffic("quant", wl.name, args.dtype),
             "algorithmic_bytes_per_launch": round(res["quant_bytes_total"] / max(1, res["quant_launches"])),
+            "in_step_copy": None if not res.get("quant_copy_reference") or quant_gbs is None else dict(
+                res["quant_copy_reference"], gbs=round(res["quant_copy_reference"]["gbs"], 1),
+                frac=round(quant_gbs / res["quant_copy_reference"]["gbs"], 4)),
         },
         "path_roofline": path_roofline(res, args.steps, peaks, fp8_peak),
         "context": res.get("context"),
