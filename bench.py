@@ -22,6 +22,7 @@ from __future__ import annotations
 import argparse
 import ctypes
 import json
+import math
 import os
 import statistics
 import subprocess
@@ -78,7 +79,8 @@ def parse_args():
     ap.add_argument("--tokens", type=int, default=0,
                     help="run the workload's Linears over this many tokens instead of its M (for ncu captures on "
                          "a reduced case; never a benchmark figure)")
-    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--e2e-steps", type=int, default=0,
+                    help="steps of the e2e measurement (0: enough for about 0.5 s of copies)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-context", action="store_true", help="skip the torch._scaled_mm context line")
@@ -421,14 +423,16 @@ def gpu_arm(args, wl, rank, world, local_rank):
     multi = getattr(args, "multi", False)
     multi_fn = lib.tfq_scaled_int8_linear_multi if args.dtype == "int8" else lib.tfq_scaled_fp8_linear_multi
 
-    def multi_arrays(group, q):
+    def multi_arrays(group, q, outs=None):
         """The array arguments of the multi-Linear GEMM for the Linears of
-        `group` (weights, scales, biases, N, outputs) and the stream."""
+        `group` (weights, scales, biases, N, outputs from `outs`, default the
+        block's outputs) and the stream."""
+        outs = ys if outs is None else outs
         return (_capi.pointer_array([W.data_ptr() for _, W, _, _ in group]),
                 _capi.pointer_array([s.data_ptr() for _, _, s, _ in group]),
                 _capi.pointer_array([None if bb is None else bb.data_ptr() for _, _, _, bb in group]),
                 (ctypes.c_int64 * len(group))(*[l.N for l, _, _, _ in group]),
-                _capi.pointer_array([ys[(l.name, q)].data_ptr() for l, _, _, _ in group]), sh)
+                _capi.pointer_array([outs[(l.name, q)].data_ptr() for l, _, _, _ in group]), sh)
     wss = {name: torch.empty(lib.tfq_quant_scaled_fp8_linear_workspace_bytes(x.shape[0]), dtype=torch.uint8,
                              device=dev) for name, x in xs.items()} if fused else {}
     ops = []
@@ -651,9 +655,12 @@ def e2e_arm(args, wl, qmaxes, quant_fn, gemm_fn, xs, lins, aq, ys, stream, sh, c
     """Every step: H2D copy of each activation of the block from pinned host
     memory, the quantizers and GEMMs, D2H copy of every output into pinned
     host memory.  The copies run on two copy streams and overlap the
-    compute stream (events order each copy with the kernels that produce or
-    consume its buffer, also across steps); the timed region ends when the
-    last D2H copy has landed."""
+    compute stream; the device buffers (activations, codes, outputs) are
+    double-buffered, steps alternating between the two sets, so that a
+    step's H2D copies overlap the previous step's kernels and D2H copies.
+    Events order each copy with the kernels that produce or consume its
+    buffer, also across steps; the timed region ends when the last D2H copy
+    has landed."""
     import torch
     hx = {n: torch.empty(x.shape, dtype=x.dtype, pin_memory=True) for n, x in xs.items()}
     for n, x in xs.items():
@@ -661,68 +668,81 @@ def e2e_arm(args, wl, qmaxes, quant_fn, gemm_fn, xs, lins, aq, ys, stream, sh, c
     hy = {k: torch.empty(y.shape, dtype=y.dtype, pin_memory=True) for k, y in ys.items()}
     h2d = sum(t.numel() * t.element_size() for t in hx.values())
     d2h = sum(t.numel() * t.element_size() for t in hy.values())
+    # the second device set
+    sets = [(xs, aq, ys),
+            ({n: torch.empty_like(x) for n, x in xs.items()},
+             {k: tuple(torch.empty_like(t) for t in v) for k, v in aq.items()},
+             {k: torch.empty_like(y) for k, y in ys.items()})]
     copy_in, copy_out = torch.cuda.Stream(), torch.cuda.Stream()
     order = []  # activations in the order the block uses them
     for lin in lins:
         if lin[0].x not in order:
             order.append(lin[0].x)
     multi_fn, multi_arrays = multi if multi is not None else (None, None)
-    x_read = {}   # event: the quantizers of the previous step finished reading x
-    y_read = {}   # event: the D2H copy of the previous step finished reading y
+    x_read = {}   # (set, x): event, the quantizers of the set's previous step finished reading x
+    y_read = {}   # (set, y): event, the D2H copy of the set's previous step finished reading y
+    counter = [0]
 
     def step():
+        k = counter[0] % 2
+        counter[0] += 1
+        xk, aqk, ysk = sets[k]
         landed = {}
         for n in order:
-            if n in x_read:
-                copy_in.wait_event(x_read[n])
+            if (k, n) in x_read:
+                copy_in.wait_event(x_read[(k, n)])
             with torch.cuda.stream(copy_in):
-                xs[n].copy_(hx[n], non_blocking=True)
+                xk[n].copy_(hx[n], non_blocking=True)
             landed[n] = torch.cuda.Event()
             landed[n].record(copy_in)
+
+        def to_host(key):
+            with torch.cuda.stream(copy_out):
+                hy[key].copy_(ysk[key], non_blocking=True)
+            y_read[(k, key)] = torch.cuda.Event()
+            y_read[(k, key)].record(copy_out)
+
         for n in order:
             stream.wait_event(landed[n])
-            x = xs[n]
+            x = xk[n]
             if wss is None:
                 for q in qmaxes:
-                    A, sa = aq[(n, q)]
+                    A, sa = aqk[(n, q)]
                     check(quant_fn(x.data_ptr(), x.shape[0], x.shape[1], float(q), A.data_ptr(), sa.data_ptr(),
                                    sh), "quant")
-                x_read[n] = torch.cuda.Event()
-                x_read[n].record(stream)
+                x_read[(k, n)] = torch.cuda.Event()
+                x_read[(k, n)].record(stream)
             for q in qmaxes:
-                A, sa = aq[(n, q)]
+                A, sa = aqk[(n, q)]
                 first = True
-                if multi:  # the Linears that read x as one launch
+                if multi_fn is not None:  # the Linears that read x as one launch
                     group = [(lin, Wq, sw, b) for lin, Wq, sw, b in lins if lin.x == n]
                     for lin, _, _, _ in group:
-                        if (lin.name, q) in y_read:
-                            stream.wait_event(y_read[(lin.name, q)])
+                        if (k, (lin.name, q)) in y_read:
+                            stream.wait_event(y_read[(k, (lin.name, q))])
                     check(multi_fn(A.data_ptr(), sa.data_ptr(), wl.M, group[0][0].K, len(group),
-                                   *multi_arrays(group, q)), "gemm")
+                                   *multi_arrays(group, q, ysk)), "gemm")
                     done = torch.cuda.Event()
                     done.record(stream)
                     copy_out.wait_event(done)
                     for lin, _, _, _ in group:
-                        with torch.cuda.stream(copy_out):
-                            hy[(lin.name, q)].copy_(ys[(lin.name, q)], non_blocking=True)
-                        y_read[(lin.name, q)] = torch.cuda.Event()
-                        y_read[(lin.name, q)].record(copy_out)
+                        to_host((lin.name, q))
                     continue
                 for lin, Wq, sw, b in lins:
                     if lin.x != n:
                         continue
                     key = (lin.name, q)
-                    y = ys[key]
-                    if key in y_read:
-                        stream.wait_event(y_read[key])
+                    y = ysk[key]
+                    if (k, key) in y_read:
+                        stream.wait_event(y_read[(k, key)])
                     bp = None if b is None else b.data_ptr()
                     if wss is not None and first:  # quantizes x inside its GEMM
                         check(lib.tfq_quant_scaled_fp8_linear(x.data_ptr(), wl.M, lin.K, float(q), Wq.data_ptr(),
                                                               sw.data_ptr(), bp, lin.N, A.data_ptr(), sa.data_ptr(),
                                                               y.data_ptr(), wss[n].data_ptr(), sh), "fused")
                         if q == qmaxes[-1]:
-                            x_read[n] = torch.cuda.Event()
-                            x_read[n].record(stream)
+                            x_read[(k, n)] = torch.cuda.Event()
+                            x_read[(k, n)].record(stream)
                     else:
                         check(gemm_fn(A.data_ptr(), sa.data_ptr(), Wq.data_ptr(), sw.data_ptr(), bp, wl.M, lin.N,
                                       lin.K, y.data_ptr(), sh), "gemm")
@@ -730,25 +750,7 @@ def e2e_arm(args, wl, qmaxes, quant_fn, gemm_fn, xs, lins, aq, ys, stream, sh, c
                     done = torch.cuda.Event()
                     done.record(stream)
                     copy_out.wait_event(done)
-                    with torch.cuda.stream(copy_out):
-                        hy[key].copy_(y, non_blocking=True)
-                    y_read[key] = torch.cuda.Event()
-                    y_read[key].record(copy_out)
-
-    step()
-    torch.cuda.synchronize()
-    t0 = torch.cuda.Event(enable_timing=True)
-    t1 = torch.cuda.Event(enable_timing=True)
-    t0.record(stream)
-    copy_in.wait_stream(stream)  # no copy of the timed steps starts before t0
-    copy_out.wait_stream(stream)
-    for _ in range(args.e2e_steps):
-        step()
-    stream.wait_stream(copy_out)
-    stream.wait_stream(copy_in)
-    t1.record(stream)
-    torch.cuda.synchronize()
-    ms = t0.elapsed_time(t1) / args.e2e_steps
+                    to_host(key)
 
     # Floor of the step over PCIe: the same copies with no kernels, both
     # directions at once on the same two copy streams (same buffers, same
@@ -765,18 +767,36 @@ def e2e_arm(args, wl, qmaxes, quant_fn, gemm_fn, xs, lins, aq, ys, stream, sh, c
         stream.wait_stream(copy_in)
         stream.wait_stream(copy_out)
 
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+
+    def timed(fn, n):
+        torch.cuda.synchronize()
+        t0.record(stream)
+        copy_in.wait_stream(stream)  # no copy of the timed steps starts before t0
+        copy_out.wait_stream(stream)
+        for _ in range(n):
+            fn()
+        stream.wait_stream(copy_out)
+        stream.wait_stream(copy_in)
+        t1.record(stream)
+        torch.cuda.synchronize()
+        return t0.elapsed_time(t1) / n
+
     copies_only()
-    torch.cuda.synchronize()
-    t0.record(stream)
-    for _ in range(args.e2e_steps):
-        copies_only()
-    t1.record(stream)
-    torch.cuda.synchronize()
-    copy_ms = t0.elapsed_time(t1) / args.e2e_steps
+    # Steps timed: --e2e-steps, or (0, the default) enough for about 0.5 s of
+    # copies, so that filling and draining the copy pipeline (the first H2D
+    # before any kernel, the last D2H after them) is a small part of the region.
+    n_steps = args.e2e_steps or max(3, min(200, math.ceil(500.0 / max(timed(copies_only, 2), 1e-3))))
+    copy_ms = timed(copies_only, n_steps)
+    step()
+    step()  # both device sets once before timing
+    ms = timed(step, n_steps)
     flops = wl.flops() // len(wl.act_qmax) * len(qmaxes)
     return {"value": flops / (ms * 1e-3) / 1e12, "unit": unit_name(args.dtype), "ms_per_step": ms,
-            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": args.e2e_steps,
-            "host_buffers": "pinned", "overlap": "H2D and D2H on two copy streams, overlapping compute",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n_steps,
+            "host_buffers": "pinned",
+            "overlap": "H2D and D2H on two copy streams, overlapping compute; device buffers double-buffered",
             "copies_alone_ms": round(copy_ms, 3), "frac_of_copy_floor": round(copy_ms / ms, 4),
             "floor": "the step's H2D and D2H copies alone, both directions at once, no kernels"}
 
