@@ -57,6 +57,7 @@ def test_quantizer_line_keys():
 
 
 def test_reference_arm_line():
-    d = _line("--impl", "reference", "--workload", "tiny_w8a8_linear", "--steps", "3", "--warmup", "3")
+    # one step of oracle work (about 15 s on the host cores) keeps the test short
+    d = _line("--impl", "reference", "--workload", "tiny_w8a8_linear", "--steps", "1", "--warmup", "1")
     assert d["impl"] == "reference" and d["cpu_baseline"]["kind"] == "oracle" and _number(d["value"])
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["value"] == d["value"]
