@@ -184,3 +184,39 @@ def test_int8_tensor_wrapper():
     ys = tfq_scaled_int8_linear_multi(A, sa, Ws, sws)
     for y, W, sw in zip(ys, Ws, sws):
         assert torch.equal(y.view(torch.int16), tfq_scaled_int8_linear(A, sa, W, sw).view(torch.int16))
+
+
+def test_int8_video_dit_qkv_full_size():
+    """The INT8 bench's Q/K/V launch at full size: the video-DiT block's
+    attention input quantized to INT8 by the GPU quantizer, Q, K and V
+    (75600 x 5120 -> 3 x 5120, INT8 weights at 127) as one launch; every
+    output bit equal to its single call, and the tile-share sample within the
+    tolerance of the oracle's exact integer sums."""
+    wl = workloads.WORKLOADS["video_dit_block"]
+    x = wl.make_x("x_attn", device="cuda")
+    M, K = x.shape
+    A = torch.empty((M, K), dtype=torch.int8, device="cuda")
+    sa = torch.empty(M, device="cuda")
+    st = _capi.raw.tfq_quant_act_int8_per_token(x.data_ptr(), M, K, 127.0, A.data_ptr(), sa.data_ptr(),
+                                                 _gpu.stream_handle())
+    assert st == _capi.TFQ_OK, _capi.last_error_message()
+    del x
+    lins = [l for l in wl.linears if l.x == "x_attn"]
+    Ws, sws, bs = [], [], []
+    for lin in lins:
+        w = wl.make_w(lin, device="cuda")
+        Wq, sw = _gpu.quant_weight(w, _capi.TFQ_DTYPE_INT8, 127.0)
+        del w
+        Ws.append(Wq.view(torch.int8)), sws.append(sw), bs.append(wl.make_bias(lin, device="cuda"))
+    ys = _multi(A, sa, Ws, sws, bs, entry="tfq_scaled_int8_linear_multi")
+    rows = _gpu.tile_sample_rows(M, seed=19)
+    ridx = torch.as_tensor(rows, device="cuda")
+    for lin, y, W, sw, b in zip(lins, ys, Ws, sws, bs):
+        y1 = _int8_linear(A, sa, W, sw, b)
+        assert torch.equal(y.view(torch.int16), y1.view(torch.int16)), lin.name
+        del y1
+        y_ref = oracle.scaled_int8_linear(A.cpu().numpy(), sa.cpu().numpy(), W.cpu().numpy(), sw.cpu().numpy(),
+                                          _gpu.bf16_bits_np(b), rows=rows)
+        _gpu.gemm_tolerance_check(y[ridx], y_ref, f"int8 video {lin.name}")
+    del ys
+    torch.cuda.empty_cache()
