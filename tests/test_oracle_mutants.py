@@ -56,6 +56,8 @@ MUTANTS = {
     "fp8_quotient_by_reciprocal": [
         ("float t = bf16_bits_to_float(row[k]) / sc;\n            if (t > qmax)",
          "float t = bf16_bits_to_float(row[k]) * (1.0f / sc);\n            if (t > qmax)")],
+    "fp8_no_clamp": [("            if (t > qmax)\n                t = qmax;\n            if (t < -qmax)\n                t = -qmax;\n            q[r * K + k] = tfq_oracle_e4m3_encode(t);",
+                      "            q[r * K + k] = tfq_oracle_e4m3_encode(t);")],
     "int8_quotient_by_reciprocal": [
         ("float t = bf16_bits_to_float(row[k]) / sc;\n            double mag",
          "float t = bf16_bits_to_float(row[k]) * (1.0f / sc);\n            double mag")],

@@ -56,7 +56,7 @@ def _inputs():
     return out
 
 
-@pytest.mark.parametrize("qmax", [448.0, 14.0, 7.0])
+@pytest.mark.parametrize("qmax", [448.0, 14.0, 7.0, 21.0, 100.0])
 def test_fp8_invariants_and_recompute(qmax):
     for x in _inputs():
         bits = bf16_bits(x)
@@ -83,6 +83,25 @@ def test_fp8_invariants_and_recompute(qmax):
         tt = xf.astype(np.float64) / s[:, None].astype(np.float64)
         bound = e4m3_spacing(np.minimum(np.abs(tt), qmax)) / 2 * (1 + 2.0 ** -20)
         assert np.all(np.abs(dec - np.clip(tt, -qmax, qmax)) <= bound + 2.0 ** -10)
+
+
+@pytest.mark.parametrize("qmax,amax", [(21.0, 1.4140625), (100.0, 1.0234375)])
+def test_fp8_clamp_of_a_quotient_above_qmax(qmax, amax):
+    """A row whose absmax quotient fl32(amax / s) lands one ulp above qmax (a
+    qmax that is not an E4M3 value lies halfway between two codes): the clamp
+    brings it back to qmax, which ties to the even code, while the unclamped
+    quotient would round up to the next code."""
+    row = np.array([amax, -amax / 2, amax / 4], dtype=np.float32)
+    bits = _row_bits([float(v) for v in row])
+    s = np.float32(amax) / np.float32(qmax)
+    t = np.float32(amax) / s
+    assert t > np.float32(qmax)                       # the case this pins
+    clamped, unclamped = bruteforce_e4m3(np.array([qmax], dtype=np.float32))[0], bruteforce_e4m3(np.array([t]))[0]
+    assert clamped != unclamped
+    q, s_o = oracle.quant_rows_fp8(bits, qmax)
+    assert s_o[0] == s and int(q[0, 0]) == int(clamped)
+    q_neg, _ = oracle.quant_rows_fp8(_row_bits([float(-v) for v in row]), qmax)
+    assert int(q_neg[0, 0]) == int(clamped) | 0x80
 
 
 def test_fp8_zero_rows_and_negative_zero():
