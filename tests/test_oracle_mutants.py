@@ -51,6 +51,8 @@ MUTANTS = {
     "encode_log2_off_by_one": [("e = E - 1;          /* floor(log2(a)) */", "e = E;")],
     # per-row scale and quotient
     "scale_signed_max": [("float v = fabsf(bf16_bits_to_float(row[k]));", "float v = bf16_bits_to_float(row[k]);")],
+    "scale_skips_last_element": [("    for (k = 0; k < K; ++k) {\n        float v = fabsf(bf16_bits_to_float(row[k]));",
+                                  "    for (k = 0; k < K - 1; ++k) {\n        float v = fabsf(bf16_bits_to_float(row[k]));")],
     "scale_no_zero_floor": [("if (amax < 1e-12f)\n        amax = 1e-12f;", "")],
     "scale_by_reciprocal": [("return amax / qmax;", "return amax * (1.0f / qmax);")],
     "fp8_quotient_by_reciprocal": [
@@ -69,6 +71,10 @@ MUTANTS = {
     "fp8_gemm_no_weight_scale": [("acc = acc * (double)s_a[m] * (double)s_w[n];", "acc = acc * (double)s_a[m];")],
     "fp8_gemm_weight_scale_index": [("acc = acc * (double)s_a[m] * (double)s_w[n];",
                                      "acc = acc * (double)s_a[m] * (double)s_w[m % N];")],
+    "fp8_gemm_float_accumulator": [("            double acc = 0.0;\n            int64_t k;\n            for (k = 0; k < K; ++k)\n                acc += dec[a[k]] * dec[w[k]];",
+                                    "            float acc = 0.0f;\n            int64_t k;\n            for (k = 0; k < K; ++k)\n                acc += (float)(dec[a[k]] * dec[w[k]]);")],
+    "fp8_gemm_activation_scale_index": [("acc = acc * (double)s_a[m] * (double)s_w[n];",
+                                         "acc = acc * (double)s_a[i] * (double)s_w[n];")],
     "fp8_gemm_reversed_k": [("acc += dec[a[k]] * dec[w[k]];", "acc += dec[a[k]] * dec[w[K - 1 - k]];")],
     "fp8_gemm_no_bias": [("acc = acc * (double)s_a[m] * (double)s_w[n];\n            if (bias)\n",
                           "acc = acc * (double)s_a[m] * (double)s_w[n];\n            if (bias && 0)\n")],

@@ -49,6 +49,13 @@ def _inputs():
         x = workloads.activations(M, K, seed=100 + seed, outlier_cols=3, outlier_mult=30.0, zero_rows=2)
         out.append(x)
     out.append(workloads.activations(33, 160, seed=7, nu=3, amplitude=4.0))
+    # rows whose absmax is their last element (every other row) or their first: the row maximum must
+    # cover the whole row, ends included
+    ends = workloads.activations(8, 96, seed=9).to(torch.float32)
+    peak = ends.abs().amax(dim=1) * 3.0
+    for r in range(8):
+        ends[r, -1 if r % 2 == 0 else 0] = peak[r] * (1 if r % 4 < 2 else -1)
+    out.append(ends.to(torch.bfloat16))
     # tiny magnitudes (scale near the 1e-12 floor) and a row of negative zeros
     tiny = workloads.activations(4, 64, seed=8) * 1e-13
     tiny[3] = -0.0
