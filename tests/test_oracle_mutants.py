@@ -40,6 +40,7 @@ MUTANTS = {
     # E4M3FN decoding
     "decode_subnormal_exponent": [("mag = ldexp((double)m, -9);", "mag = ldexp((double)m, -10);")],
     "decode_exponent_bias": [("ldexp((double)(8 + m), e - 10)", "ldexp((double)(8 + m), e - 9)")],
+    "decode_ignores_sign": [("    return sign ? -mag : mag;\n}", "    (void)sign;\n    return mag;\n}")],
     "decode_nan_whole_top_binade": [("if (e == 15 && m == 7)", "if (e == 15)")],
     # E4M3FN encoding
     "encode_ties_away": [("return (fmod(f, 2.0) == 0.0) ? f : f + 1.0;", "return f + 1.0;")],
@@ -60,6 +61,8 @@ MUTANTS = {
          "float t = bf16_bits_to_float(row[k]) * (1.0f / sc);\n            if (t > qmax)")],
     "fp8_no_clamp": [("            if (t > qmax)\n                t = qmax;\n            if (t < -qmax)\n                t = -qmax;\n            q[r * K + k] = tfq_oracle_e4m3_encode(t);",
                       "            q[r * K + k] = tfq_oracle_e4m3_encode(t);")],
+    "fp8_clamp_upper_only": [("            if (t < -qmax)\n                t = -qmax;\n            q[r * K + k] = tfq_oracle_e4m3_encode(t);",
+                              "            q[r * K + k] = tfq_oracle_e4m3_encode(t);")],
     "int8_quotient_by_reciprocal": [
         ("float t = bf16_bits_to_float(row[k]) / sc;\n            double mag",
          "float t = bf16_bits_to_float(row[k]) * (1.0f / sc);\n            double mag")],
@@ -75,6 +78,10 @@ MUTANTS = {
                                     "            float acc = 0.0f;\n            int64_t k;\n            for (k = 0; k < K; ++k)\n                acc += (float)(dec[a[k]] * dec[w[k]]);")],
     "fp8_gemm_activation_scale_index": [("acc = acc * (double)s_a[m] * (double)s_w[n];",
                                          "acc = acc * (double)s_a[i] * (double)s_w[n];")],
+    "fp8_gemm_drops_last_k": [("            for (k = 0; k < K; ++k)\n                acc += dec[a[k]] * dec[w[k]];",
+                               "            for (k = 0; k < K - 1; ++k)\n                acc += dec[a[k]] * dec[w[k]];")],
+    "fp8_gemm_bias_index": [("                acc += (double)bf16_bits_to_float(bias[n]);\n            y[i * N + n] = acc;\n        }\n    }\n}\n\n/*\n * INT8",
+                             "                acc += (double)bf16_bits_to_float(bias[m % N]);\n            y[i * N + n] = acc;\n        }\n    }\n}\n\n/*\n * INT8")],
     "fp8_gemm_reversed_k": [("acc += dec[a[k]] * dec[w[k]];", "acc += dec[a[k]] * dec[w[K - 1 - k]];")],
     "fp8_gemm_no_bias": [("acc = acc * (double)s_a[m] * (double)s_w[n];\n            if (bias)\n",
                           "acc = acc * (double)s_a[m] * (double)s_w[n];\n            if (bias && 0)\n")],
@@ -85,6 +92,8 @@ MUTANTS = {
                                        "v = (double)acc * (double)s_w[n];")],
     "int8_gemm_unsigned_activation": [("acc += (int64_t)a[k] * (int64_t)w[k];",
                                        "acc += (int64_t)(uint8_t)a[k] * (int64_t)w[k];")],
+    "int8_gemm_drops_last_k": [("            for (k = 0; k < K; ++k)\n                acc += (int64_t)a[k] * (int64_t)w[k];",
+                                "            for (k = 0; k < K - 1; ++k)\n                acc += (int64_t)a[k] * (int64_t)w[k];")],
     "int8_gemm_bias_subtracted": [("v += (double)bf16_bits_to_float(bias[n]);",
                                    "v -= (double)bf16_bits_to_float(bias[n]);")],
     # MXFP8 quantization
@@ -96,6 +105,7 @@ MUTANTS = {
     # MXFP8 GEMM
     "mx_gemm_no_weight_scale": [("(int)sfa[m * nb + b] + (int)sfw[n * nb + b] - 254", "(int)sfa[m * nb + b] - 127")],
     "mx_gemm_first_block_scale": [("(int)sfw[n * nb + b]", "(int)sfw[n * nb]")],
+    "mx_gemm_first_row_scale": [("(int)sfa[m * nb + b] + (int)sfw[n * nb + b]", "(int)sfa[b] + (int)sfw[n * nb + b]")],
     "mx_gemm_first_block_codes": [("const uint8_t *w = W + n * K + b * 32;", "const uint8_t *w = W + n * K;")],
     "mx_gemm_bias_subtracted": [("- 254);\n            }\n            if (bias)\n                acc +=",
                                  "- 254);\n            }\n            if (bias)\n                acc -=")],
