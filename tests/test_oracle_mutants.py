@@ -101,6 +101,9 @@ MUTANTS = {
     "mx_zero_block_unit_scale": [("if (amax == 0.0f)\n        return 0;", "if (amax == 0.0f)\n        return 127;")],
     "mx_exponent_floor_minus_126": [("if (e < -127)\n        e = -127;", "if (e < -126)\n        e = -126;")],
     "mx_scale_bias": [("scale = ldexp(1.0, (int)code - 127);", "scale = ldexp(1.0, (int)code - 126);")],
+    "mx_block_max_skips_last": [("            for (k = 0; k < 32; ++k) {\n                float v = fabsf(bf16_bits_to_float(blk[k]));",
+                                 "            for (k = 0; k < 31; ++k) {\n                float v = fabsf(bf16_bits_to_float(blk[k]));")],
+    "mx_block_stride": [("const uint16_t *blk = x + r * K + b * 32;", "const uint16_t *blk = x + r * K + b * 16;")],
     "mx_signed_max": [("float v = fabsf(bf16_bits_to_float(blk[k]));", "float v = bf16_bits_to_float(blk[k]);")],
     # MXFP8 GEMM
     "mx_gemm_no_weight_scale": [("(int)sfa[m * nb + b] + (int)sfw[n * nb + b] - 254", "(int)sfa[m * nb + b] - 127")],
