@@ -7,6 +7,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 from int8_w8a8_quantized_b200 import _capi, workloads
 from tests import _gpu
 from tests._pins import load_hand_rows
@@ -123,6 +124,32 @@ def test_hand_rows(K):
         assert torch.all(q[0, n:] == 0)
         amax = max(abs(v) for v in xs)
         assert s.cpu().numpy()[0] == np.float32(max(amax, 1e-12)) / np.float32(qmax)
+
+
+@pytest.mark.parametrize("K", [16, 5120, 16384])
+def test_clamp_of_quotients_above_qmax(K):
+    """Rows whose absmax quotient fl32(amax / s) lies one ulp above a qmax that
+    is not an E4M3 value (21: between codes 20 and 22; 100: between 96 and
+    104), found by search over bf16 magnitudes, in both signs, zero-padded to
+    K (grouped, warp-per-row and staged kernels): the clamp brings the
+    quotient back to qmax, which ties to the even code; codes and scales are
+    compared with the oracle bit for bit."""
+    mags = torch.arange(0x3F80, 0x4780, dtype=torch.int32).to(torch.int16).view(torch.bfloat16).float().numpy()
+    for qmax in (21.0, 100.0):
+        s = (mags / np.float32(qmax)).astype(np.float32)
+        above = mags[(mags / s).astype(np.float32) > np.float32(qmax)][:24]
+        assert len(above) >= 8
+        x = torch.zeros(2 * len(above), K, dtype=torch.float32)
+        for i, a in enumerate(above):
+            x[2 * i, 0], x[2 * i, 1] = float(a), float(a) / 4
+            x[2 * i + 1, 0], x[2 * i + 1, 1] = -float(a), float(a) / 8
+        xd = x.to(torch.bfloat16).cuda()
+        q, sc = _gpu.quant_act_fp8(xd, qmax)
+        q_ref, s_ref = _gpu.oracle_quant_fp8(xd, qmax)
+        np.testing.assert_array_equal(sc.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
+        np.testing.assert_array_equal(q.cpu().numpy(), q_ref)
+        clamped = int(oracle.e4m3_encode(np.array([qmax], dtype=np.float32))[0])
+        assert np.all(q.cpu().numpy()[:, 0] & 0x7F == clamped)
 
 
 @pytest.mark.parametrize("K", [256, 5120, 16384])
