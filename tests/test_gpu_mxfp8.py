@@ -38,6 +38,19 @@ def _check_quant(x):
     return q, sf
 
 
+@pytest.mark.parametrize("R,K", [(7, 32), (130, 256), (9, 5120)])
+def test_block_absmax_at_block_ends(R, K):
+    """Blocks whose absmax is their first or their last element (either sign):
+    the block maximum, and with it the E8M0 scale, must cover the block's ends."""
+    x = workloads.activations(R, K, seed=R + K, nu=4).float()
+    xb = x.view(R, K // 32, 32)
+    peak = xb.abs().amax(dim=2) * 3.0
+    for b in range(K // 32):
+        pos = -1 if b % 2 == 0 else 0
+        xb[:, b, pos] = peak[:, b] * (1 if b % 4 < 2 else -1)
+    _check_quant(x.to(torch.bfloat16).cuda())
+
+
 @pytest.mark.parametrize("R,K", [(1, 32), (3, 96), (5, 160), (130, 256), (129, 5120), (300, 1056),
                                  (17, 13824), (2049, 128), (64, 4096)])
 def test_quant_ragged(R, K):

@@ -152,6 +152,24 @@ def test_clamp_of_quotients_above_qmax(K):
         assert np.all(q.cpu().numpy()[:, 0] & 0x7F == clamped)
 
 
+@pytest.mark.parametrize("K", [16, 48, 2048, 3072, 5120, 13824, 16384, 20480, 65536])
+def test_absmax_at_row_ends(K):
+    """Rows whose absmax is their first or their last element (positive or
+    negative), every kernel variant (grouped, warp-per-row of one or several
+    segments, staged): the row maximum must cover both ends of the row."""
+    x = workloads.activations(16, K, seed=K + 1, nu=4).float()
+    peak = x.abs().amax(dim=1) * 3.0
+    for r in range(16):
+        x[r, -1 if r % 2 == 0 else 0] = peak[r] * (1 if r % 4 < 2 else -1)
+    xd = x.to(torch.bfloat16).cuda()
+    for qmax in (448.0, 7.0, 21.0):
+        _assert_fp8_equal(xd, qmax)
+    q, sc = _gpu.quant_weight(xd, _capi.TFQ_DTYPE_INT8, 127.0)
+    q_ref, s_ref = _gpu.oracle_quant_int8(xd, 127.0)
+    np.testing.assert_array_equal(sc.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
+    np.testing.assert_array_equal(q.cpu().numpy().view(np.int8), q_ref)
+
+
 @pytest.mark.parametrize("K", [256, 5120, 16384])
 @pytest.mark.parametrize("qmax", [1.0, 2.0, 448.0])
 def test_huge_magnitude_rows(qmax, K):
