@@ -77,6 +77,23 @@ def test_int8_extreme_codes():
     _gpu.gemm_tolerance_check(y, y_ref, "int8 extreme")
 
 
+@pytest.mark.parametrize("M,N", [(3, 8), (512, 136)])
+def test_int8_sum_at_the_largest_k(M, N):
+    """K = TFQ_INT8_MAX_K - 16, the largest K the INT8 GEMM takes, with every
+    product at 128^2: |sum| = 16384 K = 2 147 221 504, just below 2^31, so
+    the s32 accumulator is still exact (one-CTA and CTA-pair kernels)."""
+    K = _capi.TFQ_INT8_MAX_K - 16
+    A = torch.full((M, K), -128, dtype=torch.int8)
+    W = torch.full((N, K), -128, dtype=torch.int8)
+    W[1::2] = 127                                   # rows of -128 * 127 products: sums of the other sign
+    sa = torch.full((M,), 1e-6)
+    sw = torch.full((N,), 2e-6)
+    y = _int8_linear(A.cuda(), sa.cuda(), W.cuda(), sw.cuda(), None)
+    y_ref = oracle.scaled_int8_linear(A.numpy(), sa.numpy(), W.numpy(), sw.numpy())
+    assert y_ref[0, 0] == 16384.0 * K * float(np.float32(1e-6)) * float(np.float32(2e-6))
+    _gpu.gemm_tolerance_check(y, y_ref, f"int8 K={K}")
+
+
 def test_int8_linear_end_to_end():
     x = workloads.activations(700, 1024, seed=21, nu=4, outlier_cols=10, outlier_mult=20.0, zero_rows=3,
                               device="cuda")
