@@ -152,6 +152,27 @@ def test_clamp_of_quotients_above_qmax(K):
         assert np.all(q.cpu().numpy()[:, 0] & 0x7F == clamped)
 
 
+@pytest.mark.parametrize("K", [32, 5120, 16384])
+def test_subnormal_inputs(K):
+    """bf16 subnormals (below 2^-126): a row of them only (the floored scale),
+    among a normal maximum, and next to the smallest normals -- every code 0
+    with the input's sign, scales bit-exact, in FP8 and INT8, each kernel."""
+    x = torch.zeros(4, K)
+    x[0, :4] = torch.tensor([1e-39, -3e-39, 5e-40, -1e-40])
+    x[1, :4] = torch.tensor([2.0, -1e-39, 3e-39, -1e-40])
+    x[1, -1] = -7e-39
+    x[2, :3] = torch.tensor([1e-38, -1.1e-38, 1.17e-38])
+    x[3, ::7] = -1e-40
+    xd = x.to(torch.bfloat16).cuda()
+    assert float(xd.float().abs()[0].max()) < 2.0 ** -126
+    for qmax in (448.0, 7.0, 21.0):
+        _assert_fp8_equal(xd, qmax)
+    q, sc = _gpu.quant_weight(xd, _capi.TFQ_DTYPE_INT8, 127.0)
+    q_ref, s_ref = _gpu.oracle_quant_int8(xd, 127.0)
+    np.testing.assert_array_equal(sc.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
+    np.testing.assert_array_equal(q.cpu().numpy().view(np.int8), q_ref)
+
+
 @pytest.mark.parametrize("K", [16, 48, 2048, 3072, 5120, 13824, 16384, 20480, 65536])
 def test_absmax_at_row_ends(K):
     """Rows whose absmax is their first or their last element (positive or
