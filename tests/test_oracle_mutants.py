@@ -85,6 +85,8 @@ MUTANTS = {
     "fp8_gemm_reversed_k": [("acc += dec[a[k]] * dec[w[k]];", "acc += dec[a[k]] * dec[w[K - 1 - k]];")],
     "fp8_gemm_no_bias": [("acc = acc * (double)s_a[m] * (double)s_w[n];\n            if (bias)\n",
                           "acc = acc * (double)s_a[m] * (double)s_w[n];\n            if (bias && 0)\n")],
+    "fp8_gemm_bias_before_scales": [("            acc = acc * (double)s_a[m] * (double)s_w[n];\n            if (bias)\n                acc += (double)bf16_bits_to_float(bias[n]);\n            y[i * N + n] = acc;",
+                                     "            if (bias)\n                acc += (double)bf16_bits_to_float(bias[n]);\n            acc = acc * (double)s_a[m] * (double)s_w[n];\n            y[i * N + n] = acc;")],
     "fp8_gemm_bias_subtracted": [("(double)s_w[n];\n            if (bias)\n                acc +=",
                                   "(double)s_w[n];\n            if (bias)\n                acc -=")],
     # scaled INT8 GEMM
@@ -104,6 +106,8 @@ MUTANTS = {
     "mx_block_max_skips_last": [("            for (k = 0; k < 32; ++k) {\n                float v = fabsf(bf16_bits_to_float(blk[k]));",
                                  "            for (k = 0; k < 31; ++k) {\n                float v = fabsf(bf16_bits_to_float(blk[k]));")],
     "mx_block_stride": [("const uint16_t *blk = x + r * K + b * 32;", "const uint16_t *blk = x + r * K + b * 16;")],
+    "mx_element_scale_multiplied": [("double t = (double)bf16_bits_to_float(blk[k]) / scale;",
+                                     "double t = (double)bf16_bits_to_float(blk[k]) * scale;")],
     "mx_signed_max": [("float v = fabsf(bf16_bits_to_float(blk[k]));", "float v = bf16_bits_to_float(blk[k]);")],
     # MXFP8 GEMM
     "mx_gemm_no_weight_scale": [("(int)sfa[m * nb + b] + (int)sfw[n * nb + b] - 254", "(int)sfa[m * nb + b] - 127")],
