@@ -181,7 +181,8 @@ def test_profile_commands_still_run_with_this_bench(monkeypatch):
     import glob
     import os
     import shlex
-    files = sorted(glob.glob(os.path.join(bench.ROOT, "profiles", "*.md")))
+    files = sorted(f for f in glob.glob(os.path.join(bench.ROOT, "profiles", "*.md"))
+                   if os.path.basename(f) != "README.md")  # the index names no command
     assert files
     for f in files:
         text = open(f, encoding="utf-8").read().replace("\\\n", " ")
