@@ -387,7 +387,8 @@ TFQ_API const char *tfq_status_string(int status);
 /* Thread-local text of the last error this thread's calls returned. */
 TFQ_API const char *tfq_last_error_message(void);
 
-/* ABI version: 100 * major + minor. */
+/* ABI version: 100 * major + minor.  1.1 (101) added tfq_quant_scaled_fp8_linear,
+ * tfq_scaled_fp8_linear_multi and tfq_scaled_int8_linear_multi to 1.0. */
 TFQ_API int tfq_version(void);
 
 #ifdef __cplusplus

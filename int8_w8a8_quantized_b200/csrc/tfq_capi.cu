@@ -394,6 +394,6 @@ const char* tfq_status_string(int status) {
 
 const char* tfq_last_error_message(void) { return g_last_error; }
 
-int tfq_version(void) { return 100; }
+int tfq_version(void) { return 101; }
 
 }  // extern "C"

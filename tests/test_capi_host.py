@@ -57,7 +57,7 @@ def test_status_strings(lib):
     assert _capi.status_string(0) == "TFQ_OK"
     assert _capi.status_string(4) == "TFQ_ETIMEOUT"
     assert _capi.status_string(99) == "unknown"
-    assert lib.tfq_version() == 100
+    assert lib.tfq_version() == 101
 
 
 ALIGNED = 0x10000  # a fake, 16-byte aligned address: never dereferenced by a rejected call
@@ -191,7 +191,7 @@ C_PROGRAM = r"""
 int main(void)
 {
     const void *p = (const void *)0x10000; /* aligned, never dereferenced: every call below is rejected */
-    if (tfq_version() != 100)
+    if (tfq_version() != 101)
         return 1;
     if (strcmp(tfq_status_string(TFQ_EINVAL), "TFQ_EINVAL") != 0)
         return 2;
